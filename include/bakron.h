@@ -1,0 +1,199 @@
+/*
+ * bakron.h -- C ABI of the B200 (sm_100a) BaKron two-sided adaptive-rounding
+ * solver.
+ *
+ * Method: "BaKron: Efficient Quantization with Kronecker-Factored Hessians"
+ * (arXiv 2608.06291; called "FastKron" in the arXiv abstract).  A weight
+ * matrix W (m x n; row i = output channel, column j = input channel) is
+ * rounded to a per-row integer grid so as to keep the proxy loss
+ *     l(V) = vec(W-V)^T (A (x) B) vec(W-V) = tr((W-V)^T B (W-V) A)
+ * small, where A (n x n, input side) and B (m x m, output side) are the SPD
+ * Kronecker factors of the Hessian.  GPTQ applied to vec(W) with that Hessian
+ * (the paper's Algorithm 2) is reorganised into anti-diagonal rounding steps
+ * and batched rank updates (Proposition 3.1, Theorem 3.2, Algorithm 6), for
+ * O(m+n) sequential depth and O(mn(m+n)) work.
+ *
+ * Conventions for every entry point
+ *   - All matrices are dense, row-major, float32 unless stated.  Pointers
+ *     named *_dev are CUDA device pointers, *_host are host pointers.  Every
+ *     device pointer must be 16-byte aligned (else BAKRON_ERR_ALIGNMENT).
+ *   - The caller owns every buffer.  The library never allocates device or
+ *     pinned memory, never frees or retains caller memory; all scratch lives
+ *     in the caller's workspace, whose size the *_workspace_size query gives.
+ *   - Calls are stream-ordered and asynchronous on `stream` (a cudaStream_t;
+ *     NULL = legacy default stream).  Argument errors are returned at once and
+ *     nothing is enqueued.  Errors found on the device (non-SPD pivot,
+ *     non-finite input, factor with non-positive diagonal, timed-out wait) are
+ *     recorded in a status block in the first 256 bytes of the workspace;
+ *     every call clears that block (stream-ordered) before its kernels run, so
+ *     bakron_get_status() reports the latest call on that workspace.  A fresh
+ *     workspace needs no initialisation.
+ *   - A workspace must not be used by two calls that overlap on the GPU.
+ *     Distinct workspaces on distinct streams are independent.
+ *   - The library uses the current CUDA device; buffers must live on it.
+ */
+#ifndef BAKRON_H
+#define BAKRON_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *bakron_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    BAKRON_OK = 0,
+    BAKRON_ERR_INVALID_ARG = 1,    /* bad size, null pointer, bad grid, bad config */
+    BAKRON_ERR_ALIGNMENT = 2,      /* a device pointer is not 16-byte aligned */
+    BAKRON_ERR_NOT_SPD = 3,        /* (device) a Cholesky pivot was <= 0 or not finite */
+    BAKRON_ERR_NONFINITE = 4,      /* (device) W, A or B holds NaN or Inf */
+    BAKRON_ERR_DEVICE_TIMEOUT = 5, /* (device) a bounded wait gave up */
+    BAKRON_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed */
+    BAKRON_ERR_WORKSPACE = 7,      /* workspace null or smaller than the query */
+    BAKRON_ERR_BAD_FACTOR = 8      /* (device) LA or LB has a non-positive or non-finite diagonal */
+} bakron_status_t;
+
+/* Fixed per-row integer grid (the base quantizer; the method is modular in
+ * it, per the arXiv abstract).  Row i has step s_i and codes in [qmin, qmax];
+ * the rounding decision is clamp(rint(Wt_ij / s_i)) in fp32, ties to even.
+ *   bits      2..8.
+ *   qmin,qmax both 0 selects the symmetric range qmax = 2^(bits-1)-1,
+ *             qmin = -qmax; otherwise -128 <= qmin < qmax <= 127.
+ *   row_scale NULL: s_i = max_j |W_ij| / qmax (fp32, IEEE division; a row of
+ *             zeros gets s_i = 1).  Non-NULL: device pointer to m positive
+ *             finite steps, used as given. */
+typedef struct {
+    int32_t bits;
+    int32_t qmin;
+    int32_t qmax;
+    const float *row_scale;
+} bakron_quantizer_t;
+
+/* Solver configuration (NULL = defaults; zero fields take defaults).
+ *   tile        side T of the square tiles whose anti-diagonals the recursion
+ *               cuts on: 128 (default; the only supported value).
+ *   gemm        0 = tcgen05 tensor-core 3xTF32 band GEMMs (default),
+ *               1 = FP32 CUDA-core band GEMMs (cross-check).
+ *   use_graph   reserved, must be 0.
+ *   timeout_ms  limit for device-side bounded waits (default 200).
+ *   wt_out      optional device pointer, m x n fp32: if not NULL it receives
+ *               every entry's pre-rounding value Wt_ij (diagnostics). */
+typedef struct {
+    int32_t tile;
+    int32_t gemm;
+    int32_t use_graph;
+    int32_t timeout_ms;
+    float *wt_out;
+    int32_t profile;  /* 1: time every kernel class with CUDA events on `stream`;
+                         the call then synchronises `stream` before returning and
+                         the durations are read with bakron_get_profile(). */
+} bakron_config_t;
+
+/* Per-kernel-class device time of the latest profiled bakron_solve on the
+ * calling host thread (sums of CUDA-event intervals around each launch). */
+typedef struct {
+    double prep_ms, leaf_ms, stage1_ms, stage2_ms, total_ms;
+    int64_t prep_launches, leaf_launches, stage1_launches, stage2_launches;
+} bakron_profile_t;
+bakron_status_t bakron_get_profile(bakron_profile_t *out);
+
+/* ---------------------------------------------------------------- factor */
+/* Bytes of workspace bakron_factor needs for factors of sizes n and m. */
+size_t bakron_factor_workspace_size(int64_t n, int64_t m);
+
+/* Lower Cholesky factors of the inverted Hessian factors ("What carries the
+ * argument": L^(A), L^(B) with L L^T = A^{-1}, B^{-1}):
+ *   LA_dev (n x n) <- chol(A^{-1}),  LB_dev (m x m) <- chol(B^{-1}),
+ * both lower triangular with positive diagonal; the strict upper triangle is
+ * written with zeros.  A_dev (n x n) and B_dev (m x m) are SPD; only their
+ * lower triangles are read.  Computed in FP64 (blocked Cholesky of the
+ * reversed matrix J A J, blocked triangular inverse, L = J C^{-T} J), rounded
+ * to fp32.  Either side may be skipped by passing n = 0 (resp. m = 0) and
+ * NULL pointers.  Device errors: BAKRON_ERR_NOT_SPD, BAKRON_ERR_NONFINITE. */
+bakron_status_t bakron_factor(const float *A_dev, int64_t n, const float *B_dev, int64_t m,
+                              float *LA_dev, float *LB_dev, void *ws_dev, size_t ws_bytes,
+                              bakron_stream_t stream);
+
+/* ----------------------------------------------------------------- solve */
+/* Bytes of workspace bakron_solve needs for an m x n solve. */
+size_t bakron_solve_workspace_size(int64_t m, int64_t n, const bakron_config_t *cfg);
+
+/* The BaKron solve (Algorithm 6 with Proposition 3.1's updates).
+ *   W_dev      m x n weights (read only).
+ *   LA_dev     n x n raw lower factor of A^{-1} (as bakron_factor writes it).
+ *   LB_dev     m x m raw lower factor of B^{-1}.  The solver normalises both
+ *              to unit diagonal itself; only lower triangles are read.
+ *   q          grid (see bakron_quantizer_t); host pointer.
+ *   V_dev      m x n out: quantised weights, V_ij = s_i * codes_ij (fp32).
+ *   codes_dev  m x n out: int8 codes.
+ *   scales_dev m out: the steps s_i used.
+ * Result: the unique code matrix of Theorem 3.2's intended output, computed
+ * with FP32 leaf arithmetic and 3xTF32 (or FP32) band updates.  m, n >= 1.
+ * Device errors: BAKRON_ERR_NONFINITE (W), BAKRON_ERR_BAD_FACTOR,
+ * BAKRON_ERR_DEVICE_TIMEOUT. */
+bakron_status_t bakron_solve(const float *W_dev, int64_t m, int64_t n, const float *LA_dev,
+                             const float *LB_dev, const bakron_quantizer_t *q, float *V_dev,
+                             int8_t *codes_dev, float *scales_dev, void *ws_dev, size_t ws_bytes,
+                             const bakron_config_t *cfg, bakron_stream_t stream);
+
+/* Bytes of device workspace bakron_solve_host needs (solve workspace plus
+ * device staging for W, LA, LB, V, codes and scales). */
+size_t bakron_solve_host_workspace_size(int64_t m, int64_t n, const bakron_config_t *cfg);
+
+/* bakron_solve on HOST buffers: copies W_host, LA_host, LB_host to device
+ * staging inside ws_dev, solves, and copies V, codes and scales back, all
+ * enqueued on `stream` (pinned host memory makes the copies asynchronous;
+ * the results are valid after the stream is synchronised).  q->row_scale,
+ * if not NULL, is a HOST pointer here. */
+bakron_status_t bakron_solve_host(const float *W_host, int64_t m, int64_t n, const float *LA_host,
+                                  const float *LB_host, const bakron_quantizer_t *q, float *V_host,
+                                  int8_t *codes_host, float *scales_host, void *ws_dev,
+                                  size_t ws_bytes, const bakron_config_t *cfg,
+                                  bakron_stream_t stream);
+
+/* ------------------------------------------------------------ proxy loss */
+/* Bytes of workspace bakron_proxy_loss needs. */
+size_t bakron_proxy_loss_workspace_size(int64_t m, int64_t n);
+
+/* Proxy loss l = tr((W-V)^T B (W-V) A) = ||B^{1/2}(V-W)A^{1/2}||_F^2
+ * (Corollary 3.4's distortion; the review's "||vec(W)-vec(V)||_H^2",
+ * H = A (x) B).  W_dev, V_dev m x n; A_dev n x n; B_dev m x m (symmetric).
+ * Products in FP32 on the GPU, final reduction in FP64.  The result is
+ * written to *out_dev (a device double) and, if out_host is not NULL, also
+ * to *out_host, in which case the call synchronises `stream`. */
+bakron_status_t bakron_proxy_loss(const float *W_dev, const float *V_dev, const float *A_dev,
+                                  const float *B_dev, int64_t m, int64_t n, double *out_dev,
+                                  double *out_host, void *ws_dev, size_t ws_bytes,
+                                  bakron_stream_t stream);
+
+/* ---------------------------------------------------------- diagnostics */
+/* Synchronises `stream` and returns the first device-detected error of the
+ * latest call on this workspace (BAKRON_OK if none), then clears it. */
+bakron_status_t bakron_get_status(void *ws_dev, size_t ws_bytes, bakron_stream_t stream);
+
+/* Static description of a status code. */
+const char *bakron_status_string(bakron_status_t status);
+
+/* Schedule statistics of an m x n solve with the given config: number of
+ * recursion nodes, leaf launches, and the algorithmic update FLOPs (2 x the
+ * structurally non-zero multiply-adds of the band products over the tile
+ * cut; the leaves' in-tile work excluded).  Host only; enqueues nothing. */
+typedef struct {
+    int64_t tiles_m, tiles_n, tile_diagonals;
+    int64_t nodes, leaves;
+    double update_flops;   /* algorithmic (tile-dense) FLOPs of all band products */
+    double stage1_flops, stage2_flops;
+} bakron_plan_stats_t;
+bakron_status_t bakron_plan_stats(int64_t m, int64_t n, const bakron_config_t *cfg,
+                                  bakron_plan_stats_t *out);
+
+/* Library version string. */
+const char *bakron_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BAKRON_H */

@@ -1,0 +1,153 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every
+function include/bakron.h declares, and its host-only entry points behave."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "bakron.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from two_sided_gptq_b200 import _native, build
+
+    build.build()
+    return _native.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bakron_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from two_sided_gptq_b200 import _native
+
+    names = declared_functions()
+    assert len(names) >= 12
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(_native.SIGNATURES), "binding signatures must mirror the header"
+
+
+def test_library_is_sm100a_build():
+    from two_sided_gptq_b200 import build
+
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.FLAGS)
+
+
+def test_host_only_queries(lib):
+    from two_sided_gptq_b200 import _native
+
+    assert lib.bakron_version().decode().startswith("bakron-b200")
+    assert lib.bakron_status_string(3).decode().startswith("matrix is not")
+    assert lib.bakron_solve_workspace_size(0, 5, None) == 0
+    ws = lib.bakron_solve_workspace_size(4096, 4096, None)
+    # Wt, D hi/lo, X^T hi/lo (5 x m n) + three copies of each factor
+    assert ws >= 4 * (5 * 4096 * 4096 + 6 * 4096 * 4096)
+    assert lib.bakron_solve_host_workspace_size(100, 70, None) > lib.bakron_solve_workspace_size(100, 70, None)
+    assert lib.bakron_factor_workspace_size(300, 200) >= 2 * 300 * 300 * 8
+    assert lib.bakron_proxy_loss_workspace_size(3, 4) == 256
+    bad = _native.Config(64, 0, 0, 0, None)  # unsupported tile
+    assert lib.bakron_solve_workspace_size(10, 10, ctypes.byref(bad)) == 0
+
+
+def test_argument_errors_return_before_any_device_work(lib):
+    from two_sided_gptq_b200 import _native
+
+    q = _native.Quantizer(4, 0, 0, None)
+    fake = 1 << 20  # aligned, never dereferenced: validation fails first
+    args = lambda W=fake, m=8, n=8, ws=fake, wsb=1 << 30: (W, m, n, fake, fake, ctypes.byref(q), fake, fake, fake,
+                                                           ws, wsb, None, None)
+    assert lib.bakron_solve(*args(m=0)) == _native.Status.ERR_INVALID_ARG
+    assert lib.bakron_solve(*args(n=-3)) == _native.Status.ERR_INVALID_ARG
+    assert lib.bakron_solve(*args(W=None)) == _native.Status.ERR_INVALID_ARG
+    assert lib.bakron_solve(*args(ws=None)) == _native.Status.ERR_WORKSPACE
+    assert lib.bakron_solve(*args(W=fake + 4)) == _native.Status.ERR_ALIGNMENT
+    assert lib.bakron_solve(*args(wsb=100)) == _native.Status.ERR_WORKSPACE
+    q_bad = _native.Quantizer(9, 0, 0, None)
+    a = list(args())
+    a[5] = ctypes.byref(q_bad)
+    assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
+    q_bad = _native.Quantizer(4, 3, -3, None)
+    a[5] = ctypes.byref(q_bad)
+    assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
+    cfg = _native.Config(0, 5, 0, 0, None)
+    a = list(args())
+    a[11] = ctypes.byref(cfg)
+    assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
+    assert lib.bakron_factor(fake, -1, fake, 4, fake, fake, fake, 1 << 30, None) == _native.Status.ERR_INVALID_ARG
+    assert lib.bakron_factor(fake, 4, fake, 4, fake + 8, fake, fake, 1 << 30, None) == _native.Status.ERR_ALIGNMENT
+    assert lib.bakron_factor(fake, 4, fake, 4, fake, fake, fake, 16, None) == _native.Status.ERR_WORKSPACE
+    assert lib.bakron_proxy_loss(fake, fake, fake, fake, 0, 4, fake, None, fake, 256, None) == \
+        _native.Status.ERR_INVALID_ARG
+
+
+def _brute_schedule_flops(Mt, Nt, T=128):
+    """Independent count of the tile-cut schedule's band-product FLOPs.
+
+    For every node of the midpoint recursion over tile diagonals, enumerate
+    all (source tile, target tile) pairs with source <= target; X(I, J') is
+    needed when some pair links row I to column J'; stage 1 costs one tile
+    product per source tile (I, J) with J <= J' for every needed X(I, J');
+    stage 2 one per needed X(I, J') with I <= I' for every target (I', J')."""
+    tiles = [(I, J) for I in range(Mt) for J in range(Nt)]
+    total = [0.0, 0.0]
+
+    def rec(k, l):
+        if l <= 1:
+            return
+        h = l // 2
+        rec(k, h)
+        src = [(I, J) for (I, J) in tiles if k <= I + J < k + h]
+        tgt = [(I, J) for (I, J) in tiles if k + h <= I + J < k + l]
+        need = set()
+        for (I, J) in src:
+            for (I2, J2) in tgt:
+                if I <= I2 and J <= J2:
+                    need.add((I, J2))
+        for (I, J2) in need:
+            total[0] += sum(1 for (a, b) in src if a == I and b <= J2)
+        for (I2, J2) in tgt:
+            total[1] += sum(1 for (I, Jx) in need if Jx == J2 and I <= I2)
+        rec(k + h, l - h)
+
+    rec(0, Mt + Nt - 1)
+    f = 2.0 * T ** 3
+    return total[0] * f, total[1] * f
+
+
+@pytest.mark.parametrize("shape", [(1, 1), (1, 5), (4, 1), (3, 3), (5, 8), (9, 4), (7, 11)])
+def test_plan_stats_matches_bruteforce_count(lib, shape):
+    from two_sided_gptq_b200 import _native
+
+    Mt, Nt = shape
+    s = _native.PlanStats()
+    assert lib.bakron_plan_stats(Mt * 128, Nt * 128, None, ctypes.byref(s)) == 0
+    f1, f2 = _brute_schedule_flops(Mt, Nt)
+    assert s.tiles_m == Mt and s.tiles_n == Nt and s.tile_diagonals == Mt + Nt - 1
+    assert s.leaves == Mt + Nt - 1 and s.nodes == Mt + Nt - 2
+    assert s.stage1_flops == pytest.approx(f1, rel=0, abs=0)
+    assert s.stage2_flops == pytest.approx(f2, rel=0, abs=0)
+
+
+def test_plan_stats_4096_cubic_work(lib):
+    """O(mn(m+n)) work: the update FLOPs at 4096^2 lie between the
+    mn(m+n) pull-form count and twice it, and grow ~8x per size doubling
+    (the pages' falsification test: cubic, not m^2 n^2)."""
+    from two_sided_gptq_b200 import _native
+
+    def flops(m, n):
+        s = _native.PlanStats()
+        assert lib.bakron_plan_stats(m, n, None, ctypes.byref(s)) == 0
+        return s.update_flops
+
+    f = flops(4096, 4096)
+    assert 4096 ** 2 * 8192 < f < 2 * 4096 ** 2 * 8192
+    r = flops(8192, 8192) / f
+    assert 7.0 < r < 9.0, r

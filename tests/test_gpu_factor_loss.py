@@ -1,0 +1,129 @@
+"""GPU parity of bakron_factor and bakron_proxy_loss, end-to-end solves with
+GPU factors, and device-detected errors (all raised on the host side: bad
+inputs are planted in the data, never a fault)."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from parity import LOSS_RTOL, TIE_EPS, tie_cap
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bk():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import two_sided_gptq_b200 as bk
+
+    return bk
+
+
+def _t(x):
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_factor_matches_oracle(bk, name):
+    W, A, B = workloads.generate(name)
+    LA, LB = bk.factor(_t(A), _t(B))
+    for L, M in ((LA, A), (LB, B)):
+        Lg = L.cpu().numpy().astype(np.float64)
+        Lo = oracle.factor(M)
+        rel = np.linalg.norm(Lg - Lo) / np.linalg.norm(Lo)
+        resid = np.abs(Lg @ Lg.T @ M.astype(np.float64) - np.eye(M.shape[0])).max()
+        print(name, "factor rel err", rel, "max |L L^T A - I|", resid)
+        assert np.all(np.triu(Lg, 1) == 0) and np.all(np.diag(Lg) > 0)
+        assert rel <= 1e-5
+
+
+@pytest.mark.parametrize("n", [1, 2, 63, 64, 65, 200, 513])
+def test_factor_sizes(bk, n):
+    _, A, _ = workloads.random_problem(2, n, seed=n)
+    LA, _ = bk.factor(_t(A), None)
+    Lg = LA.cpu().numpy().astype(np.float64)
+    Lo = oracle.factor(A)
+    assert np.linalg.norm(Lg - Lo) / np.linalg.norm(Lo) <= 1e-5
+
+
+def test_factor_not_spd(bk):
+    A = np.eye(70, dtype=np.float32)
+    A[40, 40] = -1.0
+    with pytest.raises(bk.BakronError) as e:
+        bk.factor(_t(A), None)
+    assert e.value.status == bk.Status.ERR_NOT_SPD
+
+
+def test_factor_nonfinite(bk):
+    A = np.eye(30, dtype=np.float32)
+    A[20, 3] = np.nan
+    with pytest.raises(bk.BakronError) as e:
+        bk.factor(_t(A), None)
+    assert e.value.status in (bk.Status.ERR_NONFINITE, bk.Status.ERR_NOT_SPD)
+
+
+def test_solve_device_errors(bk):
+    W, A, B = workloads.random_problem(50, 60, seed=1)
+    LA = oracle.factor(A).astype(np.float32)
+    LB = oracle.factor(B).astype(np.float32)
+    Wn = W.copy()
+    Wn[3, 7] = np.inf
+    with pytest.raises(bk.BakronError) as e:
+        bk.solve(_t(Wn), _t(LA), _t(LB))
+    assert e.value.status == bk.Status.ERR_NONFINITE
+    LAz = LA.copy()
+    LAz[10, 10] = 0.0
+    with pytest.raises(bk.BakronError) as e:
+        bk.solve(_t(W), _t(LAz), _t(LB))
+    assert e.value.status == bk.Status.ERR_BAD_FACTOR
+    # the status is cleared after it has been read: a good solve passes
+    bk.solve(_t(W), _t(LA), _t(LB))
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_proxy_loss_matches_oracle(bk, name):
+    W, A, B = workloads.generate(name)
+    LA = oracle.factor(A).astype(np.float32)
+    LB = oracle.factor(B).astype(np.float32)
+    Wd = _t(W)
+    V, codes, s = bk.solve(Wd, _t(LA), _t(LB), bits=4)
+    l_gpu = bk.proxy_loss(Wd, V, _t(A), _t(B))
+    l_or = oracle.proxy_loss(W, V.cpu().numpy(), A, B)
+    print(name, "loss gpu", l_gpu, "oracle", l_or)
+    assert abs(l_gpu - l_or) <= LOSS_RTOL * abs(l_or)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_end_to_end_gpu_factors(bk, name):
+    """factor and solve both on the GPU, checked against the oracle running
+    from its own FP64 factors: the fp32 factor rounding moves pre-rounding
+    values by far less than the tie window, so the same contract holds."""
+    W, A, B = workloads.generate(name)
+    LA, LB = bk.factor(_t(A), _t(B))
+    Wd = _t(W)
+    V, codes, s = bk.solve(Wd, LA, LB, bits=4)
+    qmin, qmax = oracle.grid(4)
+    s_or = oracle.scales(W, qmax)
+    LtA = oracle.normalize(oracle.factor(A))
+    LtB = oracle.normalize(oracle.factor(B))
+    r = oracle.forced_check(W, LtA, LtB, s_or, qmin, qmax, codes.cpu().numpy().astype(np.int32), tie_eps=TIE_EPS)
+    print(name, "e2e mismatches", r["mismatches"], "ties", r["ties"], "failures", r["failures"])
+    assert r["failures"] == 0 and r["ties"] <= tie_cap(W.size)
+
+
+def test_solve_host_buffers(bk):
+    import torch
+
+    W, A, B = workloads.random_problem(150, 270, seed=8)
+    LA = oracle.factor(A).astype(np.float32)
+    LB = oracle.factor(B).astype(np.float32)
+    Vh, ch, sh = bk.solve_host(torch.from_numpy(W), torch.from_numpy(LA), torch.from_numpy(LB), bits=4)
+    Vd, cd, sd = bk.solve(_t(W), _t(LA), _t(LB), bits=4)
+    assert np.array_equal(ch.numpy(), cd.cpu().numpy())
+    assert np.array_equal(Vh.numpy(), Vd.cpu().numpy())
+    assert np.array_equal(sh.numpy(), sd.cpu().numpy())

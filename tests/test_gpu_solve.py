@@ -1,0 +1,102 @@
+"""GPU parity of the BaKron solve against the oracle (calls the C ABI through
+the Python binding).  See tests/parity.py for the contract."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from parity import check_solve, gpu_solve, oracle_factors
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import two_sided_gptq_b200 as bk
+
+    bk._lib()
+
+
+_cache = {}
+
+
+def named(name):
+    if name not in _cache:
+        W, A, B = workloads.generate(name)
+        LA, LB = oracle_factors(A, B)
+        _cache[name] = (W, A, B, LA, LB)
+    return _cache[name]
+
+
+@pytest.mark.parametrize("gemm", [0, 1])
+@pytest.mark.parametrize("name", ["tiny", "tiny_bI", "mid"])
+def test_named_workloads(name, gemm):
+    W, A, B, LA, LB = named(name)
+    check_solve(W, LA, LB, workloads.WORKLOADS[name].bits, gemm=gemm, label=f"{name}/gemm{gemm}")
+
+
+def test_tiny_B_identity_equals_gptq():
+    """B = I: the GPU codes equal one-sided GPTQ's (oracle, GPTQ's own form)."""
+    W, A, B, LA, LB = named("tiny_bI")
+    _, codes, s, _ = gpu_solve(W, LA, LB, 4)
+    qmin, qmax = oracle.grid(4)
+    assert np.array_equal(codes, oracle.gptq(W, A, s, qmin, qmax))
+
+
+# ragged shapes: several tiles and a ragged tail in either direction, plus
+# degenerate single-row / single-column / single-entry problems
+RAGGED = [(1, 1), (1, 300), (300, 1), (129, 257), (257, 129), (200, 333), (384, 640), (77, 1000)]
+
+
+@pytest.mark.parametrize("gemm", [0, 1])
+@pytest.mark.parametrize("shape", RAGGED)
+def test_ragged_shapes(shape, gemm):
+    m, n = shape
+    W, A, B = workloads.random_problem(m, n, seed=m * 1000 + n)
+    LA, LB = oracle_factors(A, B)
+    check_solve(W, LA, LB, 4, gemm=gemm, label=f"{m}x{n}/gemm{gemm}")
+
+
+@pytest.mark.parametrize("bits", [2, 3, 8])
+def test_other_grids(bits):
+    W, A, B = workloads.random_problem(300, 260, seed=bits)
+    LA, LB = oracle_factors(A, B)
+    check_solve(W, LA, LB, bits, label=f"int{bits}")
+
+
+def test_zero_row_and_user_scales():
+    W, A, B = workloads.random_problem(140, 150, seed=3)
+    W[5] = 0.0
+    LA, LB = oracle_factors(A, B)
+    r = check_solve(W, LA, LB, 4, label="zero-row")
+    rs = np.full(140, 0.004, np.float32)
+    check_solve(W, LA, LB, 4, row_scale=rs, label="user-scales")
+    del r
+
+
+def test_deterministic():
+    W, A, B, LA, LB = named("mid")
+    a = gpu_solve(W, LA, LB, 4)
+    b = gpu_solve(W, LA, LB, 4)
+    assert np.array_equal(a[1], b[1]) and np.array_equal(a[3], b[3])
+
+
+def test_tensor_core_and_fp32_paths_agree():
+    """The 3xTF32 tensor-core band products and the FP32 CUDA-core ones give
+    pre-rounding values within FP32-level error of each other."""
+    W, A, B, LA, LB = named("mid")
+    _, c0, _, wt0 = gpu_solve(W, LA, LB, 4, gemm=0)
+    _, c1, _, wt1 = gpu_solve(W, LA, LB, 4, gemm=1)
+    err = np.abs(wt0.astype(np.float64) - wt1).max()
+    print("tc vs simt max |dWt| =", err, " code mismatches =", int((c0 != c1).sum()))
+    assert err < 1e-5 * np.abs(W).max() * 10
+
+
+@pytest.mark.slow
+def test_bench_workload_4096():
+    W, A, B, LA, LB = named("bench")
+    check_solve(W, LA, LB, 4, label="bench4096")

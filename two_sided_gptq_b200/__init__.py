@@ -1,0 +1,191 @@
+"""B200-native BaKron two-sided adaptive-rounding solver (Python binding).
+
+Thin marshalling layer over the C ABI in ``include/bakron.h``: every step of
+the computation runs in the library's CUDA kernels.  PyTorch supplies device
+memory and streams only.
+
+    LA, LB = factor(A, B)                       # chol(A^-1), chol(B^-1), FP64 inside
+    V, codes, scales = solve(W, LA, LB, bits=4) # BaKron (Algorithm 6)
+    loss = proxy_loss(W, V, A, B)               # tr((W-V)^T B (W-V) A)
+
+Method: "BaKron: Efficient Quantization with Kronecker-Factored Hessians"
+(arXiv 2608.06291).
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _native
+from ._native import BakronError, Config, PlanStats, Profile, Quantizer, Status, check
+
+__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile", "workspace", "get_status",
+           "BakronError", "Status", "version", "library_path"]
+
+
+def _lib():
+    return _native.load()
+
+
+def library_path() -> str:
+    return _native.LIB_PATH
+
+
+def version() -> str:
+    return _lib().bakron_version().decode()
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _ptr(t) -> int:
+    return t.data_ptr() if t is not None else 0
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev_f32(x, name):
+    torch = _torch()
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous float32 CUDA tensor")
+    return x
+
+
+def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False):
+    return Config(0, int(gemm), 0, int(timeout_ms), _ptr(wt_out), 1 if profile else 0)
+
+
+def workspace(nbytes: int, device=None):
+    """A device byte buffer usable as a workspace (torch owns the memory)."""
+    torch = _torch()
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def get_status(ws, stream=None) -> Status:
+    """Synchronise and return (and clear) the device status recorded in ``ws``."""
+    return Status(_lib().bakron_get_status(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def factor(A, B=None, *, stream=None, ws=None, check_status=True):
+    """``(LA, LB)`` with ``LA LA^T = A^{-1}``, ``LB LB^T = B^{-1}`` (lower, fp32)."""
+    torch = _torch()
+    lib = _lib()
+    n = 0 if A is None else A.shape[0]
+    m = 0 if B is None else B.shape[0]
+    if A is not None:
+        _dev_f32(A, "A")
+    if B is not None:
+        _dev_f32(B, "B")
+    dev = (A if A is not None else B).device
+    LA = torch.empty((n, n), dtype=torch.float32, device=dev) if n else None
+    LB = torch.empty((m, m), dtype=torch.float32, device=dev) if m else None
+    need = lib.bakron_factor_workspace_size(n, m)
+    if ws is None:
+        ws = workspace(need, dev)
+    st = _stream(stream)
+    check(lib.bakron_factor(_ptr(A), n, _ptr(B), m, _ptr(LA), _ptr(LB), _ptr(ws), ws.numel(), st), "bakron_factor")
+    if check_status:
+        check(lib.bakron_get_status(_ptr(ws), ws.numel(), st), "bakron_factor (device)")
+    return LA, LB
+
+
+def solve_workspace_size(m: int, n: int, gemm: int = 0) -> int:
+    return int(_lib().bakron_solve_workspace_size(m, n, ctypes.byref(_config(gemm))))
+
+
+def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None, out=None, stream=None,
+          wt_out=None, check_status=True, timeout_ms=0, profile=False):
+    """BaKron solve on device tensors.  Returns ``(V, codes, scales)``.
+
+    ``gemm=0`` uses the tcgen05 3xTF32 band products, ``gemm=1`` the FP32
+    CUDA-core ones.  ``out`` may supply ``(V, codes, scales)`` buffers and
+    ``ws`` a workspace; ``check_status=False`` skips the synchronising status
+    read (for timing).
+    """
+    torch = _torch()
+    lib = _lib()
+    _dev_f32(W, "W"), _dev_f32(LA, "LA"), _dev_f32(LB, "LB")
+    m, n = W.shape
+    if LA.shape != (n, n) or LB.shape != (m, m):
+        raise ValueError("LA must be n x n and LB m x m")
+    cfg = _config(gemm, timeout_ms, wt_out, profile)
+    if out is None:
+        V = torch.empty((m, n), dtype=torch.float32, device=W.device)
+        codes = torch.empty((m, n), dtype=torch.int8, device=W.device)
+        scales = torch.empty((m,), dtype=torch.float32, device=W.device)
+    else:
+        V, codes, scales = out
+    if ws is None:
+        ws = workspace(lib.bakron_solve_workspace_size(m, n, ctypes.byref(cfg)), W.device)
+    q = Quantizer(int(bits), int(qmin), int(qmax), _ptr(row_scale))
+    st = _stream(stream)
+    check(lib.bakron_solve(_ptr(W), m, n, _ptr(LA), _ptr(LB), ctypes.byref(q), _ptr(V), _ptr(codes), _ptr(scales),
+                           _ptr(ws), ws.numel(), ctypes.byref(cfg), st), "bakron_solve")
+    if check_status:
+        check(lib.bakron_get_status(_ptr(ws), ws.numel(), st), "bakron_solve (device)")
+    return V, codes, scales
+
+
+def solve_host_workspace_size(m: int, n: int, gemm: int = 0) -> int:
+    return int(_lib().bakron_solve_host_workspace_size(m, n, ctypes.byref(_config(gemm))))
+
+
+def solve_host(W, LA, LB, bits=4, *, V=None, codes=None, scales=None, gemm=0, ws=None, stream=None,
+               synchronize=True):
+    """BaKron solve on HOST buffers (torch CPU tensors, ideally pinned): the
+    library stages them through ``ws`` on the device and copies the results
+    back.  Returns ``(V, codes, scales)`` host tensors."""
+    torch = _torch()
+    lib = _lib()
+    m, n = W.shape
+    for t, name in ((W, "W"), (LA, "LA"), (LB, "LB")):
+        if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous float32 CPU tensor")
+    V = torch.empty((m, n), dtype=torch.float32, pin_memory=True) if V is None else V
+    codes = torch.empty((m, n), dtype=torch.int8, pin_memory=True) if codes is None else codes
+    scales = torch.empty((m,), dtype=torch.float32, pin_memory=True) if scales is None else scales
+    cfg = _config(gemm)
+    if ws is None:
+        ws = workspace(lib.bakron_solve_host_workspace_size(m, n, ctypes.byref(cfg)))
+    q = Quantizer(int(bits), 0, 0, 0)
+    st = _stream(stream)
+    check(lib.bakron_solve_host(_ptr(W), m, n, _ptr(LA), _ptr(LB), ctypes.byref(q), _ptr(V), _ptr(codes),
+                                _ptr(scales), _ptr(ws), ws.numel(), ctypes.byref(cfg), st), "bakron_solve_host")
+    if synchronize:
+        check(lib.bakron_get_status(_ptr(ws), ws.numel(), st), "bakron_solve_host (device)")
+    return V, codes, scales
+
+
+def proxy_loss(W, V, A, B, *, stream=None) -> float:
+    """``tr((W-V)^T B (W-V) A)`` computed on the device (FP32 products, FP64 sum)."""
+    torch = _torch()
+    lib = _lib()
+    m, n = W.shape
+    out = torch.zeros((1,), dtype=torch.float64, device=W.device)
+    ws = workspace(lib.bakron_proxy_loss_workspace_size(m, n), W.device)
+    host = ctypes.c_double(0.0)
+    check(lib.bakron_proxy_loss(_ptr(W), _ptr(V), _ptr(A), _ptr(B), m, n, _ptr(out), ctypes.byref(host), _ptr(ws),
+                                ws.numel(), _stream(stream)), "bakron_proxy_loss")
+    return float(host.value)
+
+
+def last_profile() -> dict:
+    """Per-kernel-class device times (ms) of the latest ``solve(..., profile=True)``
+    on this thread."""
+    pr = Profile()
+    check(_lib().bakron_get_profile(ctypes.byref(pr)), "bakron_get_profile")
+    return {f: getattr(pr, f) for f, _ in Profile._fields_}
+
+
+def plan_stats(m: int, n: int) -> dict:
+    """Schedule statistics of an m x n solve (host only)."""
+    s = PlanStats()
+    check(_lib().bakron_plan_stats(m, n, None, ctypes.byref(s)), "bakron_plan_stats")
+    return {f: getattr(s, f) for f, _ in PlanStats._fields_}

@@ -1,0 +1,461 @@
+// api.cu -- the C ABI (include/bakron.h): argument checks, workspace layout
+// and the solve schedule.
+//
+// Schedule (Algorithm 6, "antidiag k+l/2 : l" in the referee report): the
+// recursion runs over ranges of tile diagonals key(I, J) = I + J of the
+// T x T tile grid, [0, Mt + Nt - 1).  solve(k, l): a range of one tile
+// diagonal is a leaf (leaf.cu); otherwise h = floor(l / 2), solve(k, h), the
+// two band products of the node (src keys [k, k+h) -> tgt keys [k+h, k+l)),
+// then solve(k + h, l - h).  Cutting on tile diagonals instead of entry
+// diagonals keeps every band product a sum of dense T x T tile products; it
+// is a valid order because tile diagonals are a coarsening of the product
+// order and Theorem 3.2 makes the result order independent.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace bakron;
+
+namespace {
+
+constexpr const char *kVersion = "bakron-b200 0.1";
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct Config {
+    int tile = kTile, gemm = 0, use_graph = 0, timeout_ms = 200, profile = 0;
+    float *wt_out = nullptr;
+};
+
+// Event-pair timing of kernel classes (profile mode): kind 0 prep, 1 leaf,
+// 2 stage 1, 3 stage 2.
+struct Profiler {
+    bool on = false;
+    cudaStream_t stream = nullptr;
+    std::vector<cudaEvent_t> pool;
+    std::vector<int> kinds;
+    size_t used = 0;
+    cudaEvent_t next()
+    {
+        if (used == pool.size()) {
+            cudaEvent_t e;
+            if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+            pool.push_back(e);
+        }
+        return pool[used++];
+    }
+    void begin(int kind)
+    {
+        if (!on) return;
+        kinds.push_back(kind);
+        cudaEvent_t e = next();
+        if (e) cudaEventRecord(e, stream);
+    }
+    void end()
+    {
+        if (!on) return;
+        cudaEvent_t e = next();
+        if (e) cudaEventRecord(e, stream);
+    }
+};
+thread_local Profiler t_prof;
+thread_local bakron_profile_t t_last_profile = {};
+
+bakron_status_t read_config(const bakron_config_t *c, Config &out)
+{
+    out = Config();
+    if (!c) return BAKRON_OK;
+    if (c->tile != 0 && c->tile != kTile) return BAKRON_ERR_INVALID_ARG;
+    if (c->gemm < 0 || c->gemm > 1) return BAKRON_ERR_INVALID_ARG;
+    out.gemm = c->gemm;
+    if (c->use_graph != 0) return BAKRON_ERR_INVALID_ARG;
+    if (c->timeout_ms < 0) return BAKRON_ERR_INVALID_ARG;
+    if (c->timeout_ms > 0) out.timeout_ms = c->timeout_ms;
+    out.wt_out = c->wt_out;
+    out.profile = c->profile ? 1 : 0;
+    return BAKRON_OK;
+}
+
+bakron_status_t read_grid(const bakron_quantizer_t *q, int &qmin, int &qmax)
+{
+    if (!q) return BAKRON_ERR_INVALID_ARG;
+    if (q->bits < 2 || q->bits > 8) return BAKRON_ERR_INVALID_ARG;
+    if (q->qmin == 0 && q->qmax == 0) {
+        qmax = (1 << (q->bits - 1)) - 1;
+        qmin = -qmax;
+    } else {
+        qmin = q->qmin;
+        qmax = q->qmax;
+        if (qmin >= qmax || qmin < -128 || qmax > 127) return BAKRON_ERR_INVALID_ARG;
+        if (qmax - qmin + 1 > (1 << q->bits)) return BAKRON_ERR_INVALID_ARG;
+    }
+    return BAKRON_OK;
+}
+
+// Largest supported side: tile counts must fit the grids' y dimension and
+// every element index fits int64.
+constexpr int64_t kMaxSide = (int64_t)kTile * 65535;
+
+std::mutex g_cfg_mu;
+bool g_configured[64] = {};
+
+cudaError_t configure_device()
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(g_cfg_mu);
+    if (dev >= 0 && dev < 64 && g_configured[dev]) return cudaSuccess;
+    if ((e = leaf_configure()) != cudaSuccess) return e;
+    if ((e = band_tc_configure()) != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) g_configured[dev] = true;
+    return cudaSuccess;
+}
+
+struct SolveCtx {
+    LeafArgs leaf;
+    GemmArgs s1, s2;
+    TcMaps m1, m2;
+    int gemm;
+    cudaStream_t stream;
+};
+
+cudaError_t run_band(const SolveCtx &c, int stage, const NodeParams &np)
+{
+    const GemmArgs &g = stage == 1 ? c.s1 : c.s2;
+    t_prof.begin(stage + 1);
+    cudaError_t e = c.gemm == 1 ? launch_band_simt(stage, np, g, c.stream)
+                                : launch_band_tc(stage, np, g, stage == 1 ? c.m1 : c.m2, c.stream);
+    t_prof.end();
+    return e;
+}
+
+cudaError_t run_schedule(const SolveCtx &c, int k, int l)
+{
+    if (l <= 1) {
+        t_prof.begin(1);
+        cudaError_t e = launch_leaf(c.leaf, k, c.stream);
+        t_prof.end();
+        return e;
+    }
+    const int h = l / 2;
+    cudaError_t e = run_schedule(c, k, h);
+    if (e != cudaSuccess) return e;
+    NodeParams np{k, h, l, c.leaf.Mt, c.leaf.Nt};
+    if ((e = run_band(c, 1, np)) != cudaSuccess) return e;
+    if ((e = run_band(c, 2, np)) != cudaSuccess) return e;
+    return run_schedule(c, k + h, l - h);
+}
+
+bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *LA, const float *LB,
+                             const bakron_quantizer_t *q, float *V, int8_t *codes, float *scales,
+                             void *ws, size_t ws_bytes, const bakron_config_t *cfg,
+                             cudaStream_t stream, bool user_scales_on_device)
+{
+    if (m < 1 || n < 1 || m > kMaxSide || n > kMaxSide) return BAKRON_ERR_INVALID_ARG;
+    if (!W || !LA || !LB || !V || !codes || !scales) return BAKRON_ERR_INVALID_ARG;
+    if (!ws) return BAKRON_ERR_WORKSPACE;
+    if (!aligned16(W) || !aligned16(LA) || !aligned16(LB) || !aligned16(V) || !aligned16(codes) ||
+        !aligned16(scales) || !aligned16(ws))
+        return BAKRON_ERR_ALIGNMENT;
+    Config conf;
+    bakron_status_t s = read_config(cfg, conf);
+    if (s != BAKRON_OK) return s;
+    if (conf.wt_out && !aligned16(conf.wt_out)) return BAKRON_ERR_ALIGNMENT;
+    int qmin = 0, qmax = 0;
+    if ((s = read_grid(q, qmin, qmax)) != BAKRON_OK) return s;
+    if (q->row_scale && !aligned16(q->row_scale) && user_scales_on_device) return BAKRON_ERR_ALIGNMENT;
+    SolveLayout L;
+    L.compute(m, n, kTile);
+    if (ws_bytes < L.total) return BAKRON_ERR_WORKSPACE;
+    if (configure_device() != cudaSuccess) return BAKRON_ERR_CUDA;
+
+    char *w = (char *)ws;
+    DeviceStatus *st = (DeviceStatus *)(w + L.status);
+    if (cudaMemsetAsync(st, 0, kStatusBytes, stream) != cudaSuccess) return BAKRON_ERR_CUDA;
+    t_prof.on = conf.profile != 0;
+    t_prof.stream = stream;
+    t_prof.used = 0;
+    t_prof.kinds.clear();
+    t_prof.begin(0);
+    if (launch_prep(W, m, n, LA, LB, qmax, q->row_scale, scales, L, w, stream) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
+    t_prof.end();
+
+    SolveCtx c;
+    c.gemm = conf.gemm;
+    c.stream = stream;
+    c.leaf.LA32 = (const float *)(w + L.LA32);
+    c.leaf.LB32 = (const float *)(w + L.LB32);
+    c.leaf.scales = scales;
+    c.leaf.Wt = (float *)(w + L.Wt);
+    c.leaf.Dhi = (float *)(w + L.Dhi);
+    c.leaf.Dlo = (float *)(w + L.Dlo);
+    c.leaf.V = V;
+    c.leaf.codes = codes;
+    c.leaf.m = m; c.leaf.n = n; c.leaf.Mp = L.Mp; c.leaf.Np = L.Np;
+    c.leaf.Mt = (int)L.Mt; c.leaf.Nt = (int)L.Nt;
+    c.leaf.qmin = qmin; c.leaf.qmax = qmax;
+    c.leaf.st = st;
+    c.leaf.wt_out = conf.wt_out;
+    // stage 1: X^T (Np x Mp) = LtA (Np x Np) . Delta (Mp x Np)^T over tile columns
+    c.s1 = GemmArgs{(const float *)(w + L.LAhi), (const float *)(w + L.LAlo),
+                    (const float *)(w + L.Dhi), (const float *)(w + L.Dlo), L.Np, L.Np,
+                    (float *)(w + L.XThi), (float *)(w + L.XTlo), nullptr, L.Mp, st, conf.timeout_ms};
+    // stage 2: Wt (Mp x Np) -= LtB (Mp x Mp) . X^T (Np x Mp)^T
+    c.s2 = GemmArgs{(const float *)(w + L.LBhi), (const float *)(w + L.LBlo),
+                    (const float *)(w + L.XThi), (const float *)(w + L.XTlo), L.Mp, L.Mp,
+                    nullptr, nullptr, (float *)(w + L.Wt), L.Np, st, conf.timeout_ms};
+    if (c.gemm == 0 && (!make_tc_maps(1, c.leaf.Mt, c.leaf.Nt, c.s1, &c.m1) ||
+                        !make_tc_maps(2, c.leaf.Mt, c.leaf.Nt, c.s2, &c.m2)))
+        return BAKRON_ERR_CUDA;
+    const int keys = (int)(L.Mt + L.Nt - 1);
+    if (run_schedule(c, 0, keys) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (t_prof.on) {
+        t_prof.on = false;
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return BAKRON_ERR_CUDA;
+        bakron_profile_t pr = {};
+        double *ms[4] = {&pr.prep_ms, &pr.leaf_ms, &pr.stage1_ms, &pr.stage2_ms};
+        int64_t *cnt[4] = {&pr.prep_launches, &pr.leaf_launches, &pr.stage1_launches, &pr.stage2_launches};
+        for (size_t i = 0; i < t_prof.kinds.size() && 2 * i + 1 < t_prof.used; ++i) {
+            float dt = 0.f;
+            cudaEventElapsedTime(&dt, t_prof.pool[2 * i], t_prof.pool[2 * i + 1]);
+            *ms[t_prof.kinds[i]] += dt;
+            *cnt[t_prof.kinds[i]] += 1;
+        }
+        pr.prep_launches *= 4;  // scales, padded copy, two factor normalisations
+        float tot = 0.f;
+        if (t_prof.used >= 2) cudaEventElapsedTime(&tot, t_prof.pool[0], t_prof.pool[t_prof.used - 1]);
+        pr.total_ms = tot;
+        t_last_profile = pr;
+    }
+    return BAKRON_OK;
+}
+
+void count_schedule(int k, int l, int Mt, int Nt, bakron_plan_stats_t *o)
+{
+    if (l <= 1) {
+        o->leaves++;
+        return;
+    }
+    const int h = l / 2;
+    count_schedule(k, h, Mt, Nt, o);
+    NodeParams np{k, h, l, Mt, Nt};
+    const double t3 = 2.0 * kTile * (double)kTile * kTile;  // FLOPs of one T x T x T tile product
+    for (int I = 0; I < Mt; ++I)
+        for (int x = 0; x < l; ++x) {
+            Item it = stage1_item(np, x, I);
+            if (it.valid) o->stage1_flops += t3 * (it.k1 - it.k0);
+        }
+    for (int I = 0; I < Mt; ++I)
+        for (int x = 0; x < l - h; ++x) {
+            Item it = stage2_item(np, x, I);
+            if (it.valid) o->stage2_flops += t3 * (it.k1 - it.k0);
+        }
+    o->nodes++;
+    count_schedule(k + h, l - h, Mt, Nt, o);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *bakron_version(void) { return kVersion; }
+
+const char *bakron_status_string(bakron_status_t s)
+{
+    switch (s) {
+    case BAKRON_OK: return "ok";
+    case BAKRON_ERR_INVALID_ARG: return "invalid argument";
+    case BAKRON_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case BAKRON_ERR_NOT_SPD: return "matrix is not symmetric positive definite (Cholesky pivot <= 0)";
+    case BAKRON_ERR_NONFINITE: return "input holds NaN or Inf";
+    case BAKRON_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+    case BAKRON_ERR_CUDA: return "CUDA runtime error";
+    case BAKRON_ERR_WORKSPACE: return "workspace missing or too small";
+    case BAKRON_ERR_BAD_FACTOR: return "factor has a non-positive or non-finite diagonal";
+    }
+    return "unknown status";
+}
+
+size_t bakron_solve_workspace_size(int64_t m, int64_t n, const bakron_config_t *cfg)
+{
+    Config conf;
+    if (m < 1 || n < 1 || m > kMaxSide || n > kMaxSide || read_config(cfg, conf) != BAKRON_OK) return 0;
+    SolveLayout L;
+    L.compute(m, n, kTile);
+    return L.total;
+}
+
+bakron_status_t bakron_solve(const float *W_dev, int64_t m, int64_t n, const float *LA_dev,
+                             const float *LB_dev, const bakron_quantizer_t *q, float *V_dev,
+                             int8_t *codes_dev, float *scales_dev, void *ws_dev, size_t ws_bytes,
+                             const bakron_config_t *cfg, bakron_stream_t stream)
+{
+    return solve_device(W_dev, m, n, LA_dev, LB_dev, q, V_dev, codes_dev, scales_dev, ws_dev, ws_bytes,
+                        cfg, (cudaStream_t)stream, true);
+}
+
+// Host-buffer variant: staging buffers follow the solve workspace.
+namespace {
+struct HostLayout {
+    size_t solve, W, LA, LB, V, codes, scales, uscales, total;
+    void compute(int64_t m, int64_t n, size_t solve_bytes)
+    {
+        size_t o = 0;
+        auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+        solve = take(solve_bytes);
+        W = take((size_t)m * n * 4); LA = take((size_t)n * n * 4); LB = take((size_t)m * m * 4);
+        V = take((size_t)m * n * 4); codes = take((size_t)m * n); scales = take((size_t)m * 4);
+        uscales = take((size_t)m * 4);
+        total = o;
+    }
+};
+}  // namespace
+
+size_t bakron_solve_host_workspace_size(int64_t m, int64_t n, const bakron_config_t *cfg)
+{
+    size_t s = bakron_solve_workspace_size(m, n, cfg);
+    if (!s) return 0;
+    HostLayout H;
+    H.compute(m, n, s);
+    return H.total;
+}
+
+bakron_status_t bakron_solve_host(const float *W_host, int64_t m, int64_t n, const float *LA_host,
+                                  const float *LB_host, const bakron_quantizer_t *q, float *V_host,
+                                  int8_t *codes_host, float *scales_host, void *ws_dev,
+                                  size_t ws_bytes, const bakron_config_t *cfg,
+                                  bakron_stream_t stream)
+{
+    if (!W_host || !LA_host || !LB_host || !V_host || !codes_host || !scales_host || !q)
+        return BAKRON_ERR_INVALID_ARG;
+    size_t sb = bakron_solve_workspace_size(m, n, cfg);
+    if (!sb) return BAKRON_ERR_INVALID_ARG;
+    if (!ws_dev) return BAKRON_ERR_WORKSPACE;
+    if (!aligned16(ws_dev)) return BAKRON_ERR_ALIGNMENT;
+    HostLayout H;
+    H.compute(m, n, sb);
+    if (ws_bytes < H.total) return BAKRON_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    char *w = (char *)ws_dev;
+    auto h2d = [&](size_t off, const void *src, size_t bytes) {
+        return cudaMemcpyAsync(w + off, src, bytes, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    };
+    if (!h2d(H.W, W_host, (size_t)m * n * 4) || !h2d(H.LA, LA_host, (size_t)n * n * 4) ||
+        !h2d(H.LB, LB_host, (size_t)m * m * 4))
+        return BAKRON_ERR_CUDA;
+    bakron_quantizer_t qd = *q;
+    if (q->row_scale) {
+        if (!h2d(H.uscales, q->row_scale, (size_t)m * 4)) return BAKRON_ERR_CUDA;
+        qd.row_scale = (const float *)(w + H.uscales);
+    }
+    bakron_status_t r = solve_device((const float *)(w + H.W), m, n, (const float *)(w + H.LA),
+                                     (const float *)(w + H.LB), &qd, (float *)(w + H.V),
+                                     (int8_t *)(w + H.codes), (float *)(w + H.scales), w + H.solve, sb,
+                                     cfg, s, true);
+    if (r != BAKRON_OK) return r;
+    if (cudaMemcpyAsync(V_host, w + H.V, (size_t)m * n * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(codes_host, w + H.codes, (size_t)m * n, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(scales_host, w + H.scales, (size_t)m * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
+    return BAKRON_OK;
+}
+
+size_t bakron_factor_workspace_size(int64_t n, int64_t m)
+{
+    if (n < 0 || m < 0 || (n == 0 && m == 0)) return 0;
+    int64_t d = std::max(n, m);
+    return align_up(kStatusBytes) + align_up((size_t)2 * d * d * sizeof(double));
+}
+
+bakron_status_t bakron_factor(const float *A_dev, int64_t n, const float *B_dev, int64_t m,
+                              float *LA_dev, float *LB_dev, void *ws_dev, size_t ws_bytes,
+                              bakron_stream_t stream)
+{
+    if (n < 0 || m < 0 || (n == 0 && m == 0) || n > kMaxSide || m > kMaxSide) return BAKRON_ERR_INVALID_ARG;
+    if ((n > 0 && (!A_dev || !LA_dev)) || (m > 0 && (!B_dev || !LB_dev))) return BAKRON_ERR_INVALID_ARG;
+    if (!ws_dev) return BAKRON_ERR_WORKSPACE;
+    if ((n > 0 && (!aligned16(A_dev) || !aligned16(LA_dev))) ||
+        (m > 0 && (!aligned16(B_dev) || !aligned16(LB_dev))) || !aligned16(ws_dev))
+        return BAKRON_ERR_ALIGNMENT;
+    if (ws_bytes < bakron_factor_workspace_size(n, m)) return BAKRON_ERR_WORKSPACE;
+    char *w = (char *)ws_dev;
+    DeviceStatus *st = (DeviceStatus *)w;
+    double *work = (double *)(w + align_up(kStatusBytes));
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemsetAsync(st, 0, kStatusBytes, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (n > 0 && launch_factor(A_dev, n, LA_dev, work, st, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (m > 0 && launch_factor(B_dev, m, LB_dev, work, st, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    return BAKRON_OK;
+}
+
+size_t bakron_proxy_loss_workspace_size(int64_t m, int64_t n)
+{
+    if (m < 1 || n < 1) return 0;
+    return kStatusBytes;
+}
+
+bakron_status_t bakron_proxy_loss(const float *W_dev, const float *V_dev, const float *A_dev,
+                                  const float *B_dev, int64_t m, int64_t n, double *out_dev,
+                                  double *out_host, void *ws_dev, size_t ws_bytes,
+                                  bakron_stream_t stream)
+{
+    if (m < 1 || n < 1 || m > kMaxSide || n > kMaxSide) return BAKRON_ERR_INVALID_ARG;
+    if (!W_dev || !V_dev || !A_dev || !B_dev || !out_dev) return BAKRON_ERR_INVALID_ARG;
+    if (!ws_dev || ws_bytes < kStatusBytes) return BAKRON_ERR_WORKSPACE;
+    if (!aligned16(W_dev) || !aligned16(V_dev) || !aligned16(A_dev) || !aligned16(B_dev) ||
+        ((uintptr_t)out_dev & 7u))
+        return BAKRON_ERR_ALIGNMENT;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemsetAsync(ws_dev, 0, kStatusBytes, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (launch_proxy_loss(W_dev, V_dev, A_dev, B_dev, m, n, out_dev, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (out_host) {
+        if (cudaMemcpyAsync(out_host, out_dev, sizeof(double), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return BAKRON_ERR_CUDA;
+    }
+    return BAKRON_OK;
+}
+
+bakron_status_t bakron_get_status(void *ws_dev, size_t ws_bytes, bakron_stream_t stream)
+{
+    if (!ws_dev || ws_bytes < kStatusBytes) return BAKRON_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    DeviceStatus h;
+    if (cudaMemcpy(&h, ws_dev, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (h.code != 0 && cudaMemset(ws_dev, 0, sizeof(h)) != cudaSuccess) return BAKRON_ERR_CUDA;
+    return (bakron_status_t)h.code;
+}
+
+bakron_status_t bakron_get_profile(bakron_profile_t *out)
+{
+    if (!out) return BAKRON_ERR_INVALID_ARG;
+    *out = t_last_profile;
+    return BAKRON_OK;
+}
+
+bakron_status_t bakron_plan_stats(int64_t m, int64_t n, const bakron_config_t *cfg, bakron_plan_stats_t *out)
+{
+    Config conf;
+    if (!out || m < 1 || n < 1 || m > kMaxSide || n > kMaxSide) return BAKRON_ERR_INVALID_ARG;
+    if (read_config(cfg, conf) != BAKRON_OK) return BAKRON_ERR_INVALID_ARG;
+    std::memset(out, 0, sizeof(*out));
+    out->tiles_m = (m + kTile - 1) / kTile;
+    out->tiles_n = (n + kTile - 1) / kTile;
+    out->tile_diagonals = out->tiles_m + out->tiles_n - 1;
+    count_schedule(0, (int)out->tile_diagonals, (int)out->tiles_m, (int)out->tiles_n, out);
+    out->update_flops = out->stage1_flops + out->stage2_flops;
+    return BAKRON_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,344 @@
+// band_tc.cu -- the band products of Algorithm 6 on the 5th-generation tensor
+// cores (tcgen05, sm_100a), 3xTF32.
+//
+// Each CTA computes one T x T output tile D = sum_k A[ra rows, k] B[rb rows, k]^T
+// over a contiguous range of tile columns (stage 1: X^T = LtA . Delta^T,
+// stage 2: Wt -= LtB . X).  Both operands are K-major in global memory, so
+// TMA loads 128-row x 32-column fp32 boxes with 128-byte swizzle straight into
+// the canonical UMMA layout.  Operands are pre-split into TF32 hi/lo parts;
+// every K=8 step issues hi*hi + hi*lo + lo*hi into one FP32 TMEM accumulator
+// (the low*low term is below FP32 resolution).
+//
+// Warp roles (192 threads): warp 0 lane 0 issues TMA into a 3-stage ring;
+// warp 1 owns TMEM and lane 0 issues the MMAs; warps 2..5 read the
+// accumulator back (tcgen05.ld, 32 lanes each) and write the tile.
+// Every mbarrier wait is bounded by a %globaltimer deadline; on expiry the
+// kernel records BAKRON_ERR_DEVICE_TIMEOUT, drains what it issued and exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace bakron {
+
+namespace {
+constexpr int T = kTile;
+constexpr int KB = 32;                    // fp32 columns per stage (128 bytes)
+constexpr int kStages = 3;
+constexpr int kTileBytes = T * KB * 4;    // 16 KB per operand part
+constexpr int kStageBytes = 4 * kTileBytes;
+constexpr int kThreads = 192;
+constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t kTmemCols = 128;
+
+// Instruction descriptor: D fp32, A/B tf32, K-major both, N = 128, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(T >> 3) << 17) |
+                            ((uint32_t)(T >> 4) << 24);
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint64_t now_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: false if the deadline passed first.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t deadline)
+{
+    while (!mbar_try_wait(bar, parity))
+        if (now_ns() > deadline) return false;
+    return true;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"((uint64_t)map), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+// UMMA shared-memory descriptor, K-major, 128-byte swizzle: 8-row atoms of
+// 128 B rows, atoms 1024 B apart (SBO), LBO unused (1), version 1.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+__device__ __forceinline__ void umma_tf32(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate));
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+}  // namespace
+
+template <int STAGE>
+__global__ void __launch_bounds__(kThreads, 1)
+band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
+{
+    const Item it = STAGE == 1 ? stage1_item(np, blockIdx.x, blockIdx.y)
+                               : stage2_item(np, blockIdx.x, blockIdx.y);
+    if (!it.valid) return;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t *bars = (uint64_t *)(smem + kStages * kStageBytes);
+    // bars[0..S) full, bars[S..2S) empty, bars[2S] accumulator ready, bars[2S+1] drain
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+    const uint32_t acc_bar = bar0 + 8u * (2 * kStages), drain_bar = acc_bar + 8u;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(acc_bar, 1);
+        mbar_init(drain_bar, 1);
+        abort_sh = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&tmem_base_sh)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = tmem_base_sh;
+
+    const int nk = (it.k1 - it.k0) * (T / KB);
+    const int kbase = it.k0 * T;
+    const uint64_t deadline = now_ns() + (uint64_t)g.timeout_ms * 1000000ull;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------- TMA producer
+        int issued = 0;
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % kStages;
+            if (kb >= kStages && !mbar_wait(empty_bar(s), ((kb / kStages) - 1) & 1, deadline)) {
+                record_error(g.st, BAKRON_ERR_DEVICE_TIMEOUT, 1000 + STAGE);
+                atomicExch(&abort_sh, 1);
+                break;
+            }
+            if (*(volatile int *)&abort_sh) break;
+            const uint32_t base = smem_u32(smem + s * kStageBytes);
+            mbar_expect_tx(full_bar(s), kStageBytes);
+            const int x = kbase + kb * KB;
+            tma_load_2d(base, &maps.a_hi, x, it.ra * T, full_bar(s));
+            tma_load_2d(base + kTileBytes, &maps.a_lo, x, it.ra * T, full_bar(s));
+            tma_load_2d(base + 2 * kTileBytes, &maps.b_hi, x, it.rb * T, full_bar(s));
+            tma_load_2d(base + 3 * kTileBytes, &maps.b_lo, x, it.rb * T, full_bar(s));
+            issued = kb + 1;
+        }
+        // make sure every issued copy has landed before the CTA can exit
+        for (int kb = max(0, issued - kStages); kb < issued; ++kb)
+            mbar_wait(full_bar(kb % kStages), (kb / kStages) & 1, deadline + 50000000ull);
+    } else if (warp == 1 && lane == 0) {
+        // ---------------- MMA issuer
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % kStages;
+            if (!mbar_wait(full_bar(s), (kb / kStages) & 1, deadline)) {
+                record_error(g.st, BAKRON_ERR_DEVICE_TIMEOUT, 2000 + STAGE);
+                atomicExch(&abort_sh, 1);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t base = smem_u32(smem + s * kStageBytes);
+#pragma unroll
+            for (int k8 = 0; k8 < KB / 8; ++k8) {
+                const uint32_t off = k8 * 32;  // 8 tf32 = 32 bytes along K inside the swizzle atom
+                const uint64_t ah = umma_desc(base + off), al = umma_desc(base + kTileBytes + off);
+                const uint64_t bh = umma_desc(base + 2 * kTileBytes + off), bl = umma_desc(base + 3 * kTileBytes + off);
+                umma_tf32(tmem_d, al, bh, (kb | k8) != 0);
+                umma_tf32(tmem_d, ah, bl, 1);
+                umma_tf32(tmem_d, ah, bh, 1);
+            }
+            umma_commit(empty_bar(s));
+        }
+        umma_commit(ok ? acc_bar : drain_bar);
+        if (!ok) mbar_wait(drain_bar, 0, deadline + 50000000ull);
+    } else if (warp >= 2) {
+        // ---------------- epilogue: TMEM -> registers -> global
+        const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
+        int go = 0;
+        if (lane == 0) {
+            const bool ok = mbar_wait(acc_bar, 0, deadline);
+            if (!ok) {
+                record_error(g.st, BAKRON_ERR_DEVICE_TIMEOUT, 3000 + STAGE);
+                atomicExch(&abort_sh, 1);
+            }
+            go = ok && !*(volatile int *)&abort_sh;
+        }
+        go = __shfl_sync(0xffffffffu, go, 0);  // warp-uniform: tcgen05.ld is .sync.aligned
+        if (go) {
+            tc_fence_after();
+            const int r = quad * 32 + lane;
+            const int64_t orow = (int64_t)it.ra * T + r;
+            const int64_t ocol = (int64_t)it.rb * T;
+#pragma unroll 1
+            for (int c0 = 0; c0 < T; c0 += 32) {
+                float v[32];
+                tmem_ld32(tmem_d + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+                if (STAGE == 1) {
+                    float4 *hi = (float4 *)(g.out_hi + orow * g.ldo + ocol + c0);
+                    float4 *lo = (float4 *)(g.out_lo + orow * g.ldo + ocol + c0);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float4 h, l;
+                        split_tf32(v[4 * q + 0], h.x, l.x);
+                        split_tf32(v[4 * q + 1], h.y, l.y);
+                        split_tf32(v[4 * q + 2], h.z, l.z);
+                        split_tf32(v[4 * q + 3], h.w, l.w);
+                        hi[q] = h;
+                        lo[q] = l;
+                    }
+                } else {
+                    float4 *o = (float4 *)(g.out_acc + orow * g.ldo + ocol + c0);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float4 w = o[q];
+                        w.x -= v[4 * q + 0];
+                        w.y -= v[4 * q + 1];
+                        w.z -= v[4 * q + 2];
+                        w.w -= v[4 * q + 3];
+                        o[q] = w;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(kTmemCols));
+    }
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode()
+{
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+// rows x cols fp32 row-major matrix with row stride ld (elements); box 32 x 128.
+bool make_map(CUtensorMap *map, const float *base, int64_t rows, int64_t cols, int64_t ld)
+{
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+    cuuint32_t box[2] = {(cuuint32_t)KB, (cuuint32_t)T};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, (void *)base, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t band_tc_configure()
+{
+    cudaError_t e = cudaFuncSetAttribute(band_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(band_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+}
+
+bool make_tc_maps(int stage, int Mt, int Nt, const GemmArgs &g, TcMaps *maps)
+{
+    // stage 1: A = LtA (Np x Np), B = Delta (Mp x Np); stage 2: A = LtB (Mp x Mp),
+    // B = X^T (Np x Mp).  In both, an operand's column count equals its row stride.
+    const int64_t Mp = (int64_t)Mt * T, Np = (int64_t)Nt * T;
+    const int64_t a_rows = stage == 1 ? Np : Mp, b_rows = stage == 1 ? Mp : Np;
+    return make_map(&maps->a_hi, g.Ahi, a_rows, g.lda, g.lda) && make_map(&maps->a_lo, g.Alo, a_rows, g.lda, g.lda) &&
+           make_map(&maps->b_hi, g.Bhi, b_rows, g.ldb, g.ldb) && make_map(&maps->b_lo, g.Blo, b_rows, g.ldb, g.ldb);
+}
+
+cudaError_t launch_band_tc(int stage, const NodeParams &np, const GemmArgs &g, const TcMaps &maps,
+                           cudaStream_t stream)
+{
+    if (stage == 1) {
+        band_tc_kernel<1><<<dim3(np.l, np.Mt), kThreads, kSmem, stream>>>(maps, np, g);
+    } else {
+        band_tc_kernel<2><<<dim3(np.l - np.h, np.Mt), kThreads, kSmem, stream>>>(maps, np, g);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace bakron

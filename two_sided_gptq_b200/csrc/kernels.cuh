@@ -1,0 +1,62 @@
+// kernels.cuh -- launch interfaces between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace bakron {
+
+struct LeafArgs {
+    const float *LA32, *LB32, *scales;
+    float *Wt, *Dhi, *Dlo, *V;
+    int8_t *codes;
+    int64_t m, n, Mp, Np;
+    int Mt, Nt, qmin, qmax;
+    DeviceStatus *st;
+    float *wt_out;  // optional m x n pre-rounding values
+};
+
+// Operands of the band products.  Stage 1: A = LtA (Np x Np), B = Delta
+// (Mp x Np), out = X^T (Np x Mp, hi/lo).  Stage 2: A = LtB (Mp x Mp),
+// B = X^T (Np x Mp), out = Wt (Mp x Np) -= D.
+struct GemmArgs {
+    const float *Ahi, *Alo, *Bhi, *Blo;
+    int64_t lda, ldb;    // row strides (elements) of A and B
+    float *out_hi, *out_lo;  // stage 1 outputs (ld = ldo)
+    float *out_acc;          // stage 2 output (ld = ldo), out -= D
+    int64_t ldo;
+    DeviceStatus *st;
+    int timeout_ms;
+};
+
+cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, const float *LB,
+                        int qmax, const float *user_scales, float *scales, const SolveLayout &L,
+                        char *ws, cudaStream_t stream);
+
+cudaError_t leaf_configure();
+cudaError_t launch_leaf(const LeafArgs &p, int K, cudaStream_t stream);
+
+// FP32 CUDA-core band products (reference kernels for the tensor-core path).
+cudaError_t launch_band_simt(int stage, const NodeParams &np, const GemmArgs &g, cudaStream_t stream);
+
+// tcgen05 3xTF32 band products.  The TMA descriptors of a stage's four
+// operand parts depend only on the workspace, so they are encoded once per
+// solve.
+struct TcMaps {
+    CUtensorMap a_hi, a_lo, b_hi, b_lo;
+};
+cudaError_t band_tc_configure();
+bool make_tc_maps(int stage, int Mt, int Nt, const GemmArgs &g, TcMaps *maps);
+cudaError_t launch_band_tc(int stage, const NodeParams &np, const GemmArgs &g, const TcMaps &maps,
+                           cudaStream_t stream);
+
+// Proxy loss (FP32 products, FP64 reduction) into *out (device double).
+cudaError_t launch_proxy_loss(const float *W, const float *V, const float *A, const float *B,
+                              int64_t m, int64_t n, double *out, cudaStream_t stream);
+
+// FP64 factorisation: L (n x n, fp32) = chol(A^{-1}); work = n*n doubles.
+cudaError_t launch_factor(const float *A, int64_t n, float *L, double *work, DeviceStatus *st,
+                          cudaStream_t stream);
+
+}  // namespace bakron
