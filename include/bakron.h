@@ -154,6 +154,40 @@ bakron_status_t bakron_solve_host(const float *W_host, int64_t m, int64_t n, con
                                   size_t ws_bytes, const bakron_config_t *cfg,
                                   bakron_stream_t stream);
 
+/* ------------------------------------------------ allocation-free solve */
+/* No counterpart in the paper: this is a service of the library, not a step
+ * of the method.
+ *
+ * Some callers may not allocate device memory at the moment they need a
+ * solve: plug-ins whose execution hook must not allocate (an inference
+ * engine's enqueue step, for example), and services that reserve all their
+ * memory at start-up and forbid allocation afterwards so that their footprint
+ * stays fixed.  They cannot obtain the workspace bakron_solve asks for.  This
+ * entry point runs the same solve with its workspace in a device array that
+ * the library itself declares: BAKRON_NOALLOC_SCRATCH_BYTES bytes, reserved
+ * on every GPU that loads the library and held until the process exits.
+ *
+ *   Arguments as bakron_solve, without ws/ws_bytes.  The problem must fit
+ *   the array: bakron_solve_workspace_size(m, n, cfg) <=
+ *   BAKRON_NOALLOC_SCRATCH_BYTES (true for any m, n <= 512); larger problems
+ *   return BAKRON_ERR_WORKSPACE and nothing is enqueued.  cfg->profile must be
+ *   0 (BAKRON_ERR_INVALID_ARG otherwise).
+ *   device_status_host: NULL keeps the call asynchronous (device-detected
+ *   errors are then not reported); otherwise the call synchronises `stream`
+ *   and stores the device status (a bakron_status_t value) there.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.  The library calls no cudaMalloc or cudaFree here.
+ *   Every call on a device shares the one array and leaves its contents
+ *   behind; the solve clears what must start at zero.  Calls that overlap on
+ *   the GPU (other streams, other host threads) race on the array: issue them
+ *   one after another. */
+#define BAKRON_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+bakron_status_t bakron_solve_noalloc(const float *W_dev, int64_t m, int64_t n, const float *LA_dev,
+                                     const float *LB_dev, const bakron_quantizer_t *q, float *V_dev,
+                                     int8_t *codes_dev, float *scales_dev, const bakron_config_t *cfg,
+                                     bakron_stream_t stream, int32_t *device_status_host);
+
 /* ------------------------------------------------------------ proxy loss */
 /* Bytes of workspace bakron_proxy_loss needs. */
 size_t bakron_proxy_loss_workspace_size(int64_t m, int64_t n);

@@ -73,6 +73,8 @@ SIGNATURES = {
     "bakron_plan_stats": (ctypes.c_int, [_i64, _i64, ctypes.POINTER(Config), ctypes.POINTER(PlanStats)]),
     "bakron_version": (ctypes.c_char_p, []),
     "bakron_get_profile": (ctypes.c_int, [ctypes.POINTER(Profile)]),
+    "bakron_solve_noalloc": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, ctypes.POINTER(Quantizer), _vp, _vp, _vp,
+                                            ctypes.POINTER(Config), _vp, ctypes.POINTER(ctypes.c_int32)]),
 }
 
 _lib = None
