@@ -90,6 +90,10 @@ typedef struct {
     int32_t profile;  /* 1: time every kernel class with CUDA events on `stream`;
                          the call then synchronises `stream` before returning and
                          the durations are read with bakron_get_profile(). */
+    int32_t leaf;     /* leaf sweep structure: 0 = default (3); 1 = each tile as
+                         2 x 2 sub-tiles of 64 swept by the whole CTA; 2 = one
+                         anti-diagonal sweep over the whole 128 x 128 tile; 3 =
+                         4 x 4 sub-tiles of 32, each swept by one warp. */
 } bakron_config_t;
 
 /* Per-kernel-class device time of the latest profiled bakron_solve on the

@@ -41,7 +41,7 @@ def oracle_factors(A, B):
     return LA, LB
 
 
-def gpu_solve(W, LA32, LB32, bits, gemm=0, row_scale=None):
+def gpu_solve(W, LA32, LB32, bits, gemm=0, row_scale=None, leaf=0):
     import torch
 
     import two_sided_gptq_b200 as bk
@@ -52,17 +52,17 @@ def gpu_solve(W, LA32, LB32, bits, gemm=0, row_scale=None):
     LBd = torch.from_numpy(np.ascontiguousarray(LB32)).to(dev)
     wt = torch.empty_like(Wd)
     rs = None if row_scale is None else torch.from_numpy(np.asarray(row_scale, np.float32)).to(dev)
-    V, codes, scales = bk.solve(Wd, LAd, LBd, bits=bits, gemm=gemm, wt_out=wt, row_scale=rs)
+    V, codes, scales = bk.solve(Wd, LAd, LBd, bits=bits, gemm=gemm, wt_out=wt, row_scale=rs, leaf=leaf)
     torch.cuda.synchronize()
     return V.cpu().numpy(), codes.cpu().numpy().astype(np.int32), scales.cpu().numpy(), wt.cpu().numpy()
 
 
-def check_solve(W, LA32, LB32, bits, gemm=0, row_scale=None, label=""):
+def check_solve(W, LA32, LB32, bits, gemm=0, row_scale=None, label="", leaf=0):
     """Run the GPU solve on (W, LA32, LB32) and check it teacher-forced
     against the oracle using the same fp32 factors (widened to FP64).
     Returns the report dict (asserts the contract)."""
     qmin, qmax = oracle.grid(bits)
-    V, codes, s_gpu, wt_gpu = gpu_solve(W, LA32, LB32, bits, gemm, row_scale)
+    V, codes, s_gpu, wt_gpu = gpu_solve(W, LA32, LB32, bits, gemm, row_scale, leaf)
     s = oracle.scales(W, qmax) if row_scale is None else np.asarray(row_scale, np.float32)
     assert np.array_equal(s_gpu.view(np.uint32), s.view(np.uint32)), f"{label}: steps differ"
     LtA = oracle.normalize(LA32.astype(np.float64))

@@ -58,8 +58,8 @@ def _dev_f32(x, name):
     return x
 
 
-def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False):
-    return Config(0, int(gemm), 0, int(timeout_ms), _ptr(wt_out), 1 if profile else 0)
+def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False, leaf=0):
+    return Config(0, int(gemm), 0, int(timeout_ms), _ptr(wt_out), 1 if profile else 0, int(leaf))
 
 
 def workspace(nbytes: int, device=None):
@@ -101,11 +101,12 @@ def solve_workspace_size(m: int, n: int, gemm: int = 0) -> int:
 
 
 def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None, out=None, stream=None,
-          wt_out=None, check_status=True, timeout_ms=0, profile=False):
+          wt_out=None, check_status=True, timeout_ms=0, profile=False, leaf=0):
     """BaKron solve on device tensors.  Returns ``(V, codes, scales)``.
 
     ``gemm=0`` uses the tcgen05 3xTF32 band products, ``gemm=1`` the FP32
-    CUDA-core ones.  ``out`` may supply ``(V, codes, scales)`` buffers and
+    CUDA-core ones; ``leaf`` selects the leaf sweep structure (0 default,
+    1 two-level CTA-wide, 2 single-level, 3 warp per 32 x 32 sub-tile).  ``out`` may supply ``(V, codes, scales)`` buffers and
     ``ws`` a workspace; ``check_status=False`` skips the synchronising status
     read (for timing).
     """
@@ -115,7 +116,7 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     m, n = W.shape
     if LA.shape != (n, n) or LB.shape != (m, m):
         raise ValueError("LA must be n x n and LB m x m")
-    cfg = _config(gemm, timeout_ms, wt_out, profile)
+    cfg = _config(gemm, timeout_ms, wt_out, profile, leaf)
     if out is None:
         V = torch.empty((m, n), dtype=torch.float32, device=W.device)
         codes = torch.empty((m, n), dtype=torch.int8, device=W.device)

@@ -31,7 +31,7 @@ constexpr const char *kVersion = "bakron-b200 0.1";
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 struct Config {
-    int tile = kTile, gemm = 0, use_graph = 0, timeout_ms = 200, profile = 0;
+    int tile = kTile, gemm = 0, use_graph = 0, timeout_ms = 200, profile = 0, leaf = 2;
     float *wt_out = nullptr;
 };
 
@@ -81,6 +81,8 @@ bakron_status_t read_config(const bakron_config_t *c, Config &out)
     if (c->timeout_ms > 0) out.timeout_ms = c->timeout_ms;
     out.wt_out = c->wt_out;
     out.profile = c->profile ? 1 : 0;
+    if (c->leaf < 0 || c->leaf > 3) return BAKRON_ERR_INVALID_ARG;
+    if (c->leaf != 0) out.leaf = c->leaf - 1;  // 0 keeps the default
     return BAKRON_OK;
 }
 
@@ -124,7 +126,7 @@ struct SolveCtx {
     LeafArgs leaf;
     GemmArgs s1, s2;
     TcMaps m1, m2;
-    int gemm;
+    int gemm, leaf_variant;
     cudaStream_t stream;
 };
 
@@ -142,7 +144,7 @@ cudaError_t run_schedule(const SolveCtx &c, int k, int l)
 {
     if (l <= 1) {
         t_prof.begin(1);
-        cudaError_t e = launch_leaf(c.leaf, k, c.stream);
+        cudaError_t e = launch_leaf(c.leaf, k, c.leaf_variant, c.stream);
         t_prof.end();
         return e;
     }
@@ -192,6 +194,7 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
 
     SolveCtx c;
     c.gemm = conf.gemm;
+    c.leaf_variant = conf.leaf;
     c.stream = stream;
     c.leaf.LA32 = (const float *)(w + L.LA32);
     c.leaf.LB32 = (const float *)(w + L.LB32);

@@ -18,6 +18,7 @@ __global__ void __launch_bounds__(256) band_simt_kernel(NodeParams np, GemmArgs 
     const Item it = STAGE == 1 ? stage1_item(np, blockIdx.x, blockIdx.y)
                                : stage2_item(np, blockIdx.x, blockIdx.y);
     if (!it.valid) return;
+    pdl_wait();
     __shared__ float As[BK][T + 4];
     __shared__ float Bs[BK][T + 4];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -70,14 +71,8 @@ __global__ void __launch_bounds__(256) band_simt_kernel(NodeParams np, GemmArgs 
 
 cudaError_t launch_band_simt(int stage, const NodeParams &np, const GemmArgs &g, cudaStream_t stream)
 {
-    if (stage == 1) {
-        dim3 grid(np.l, np.Mt);
-        band_simt_kernel<1><<<grid, 256, 0, stream>>>(np, g);
-    } else {
-        dim3 grid(np.l - np.h, np.Mt);
-        band_simt_kernel<2><<<grid, 256, 0, stream>>>(np, g);
-    }
-    return cudaGetLastError();
+    if (stage == 1) return launch_pdl(band_simt_kernel<1>, dim3(np.l, np.Mt), dim3(256), 0, stream, np, g);
+    return launch_pdl(band_simt_kernel<2>, dim3(np.l - np.h, np.Mt), dim3(256), 0, stream, np, g);
 }
 
 // --------------------------------------------------------------------------

@@ -29,7 +29,7 @@ constexpr int kTileBytes = T * KB * 4;    // 16 KB per operand part
 constexpr int kStageBytes = 4 * kTileBytes;
 constexpr int kThreads = 192;
 constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kTmemCols = 2 * T;  // two accumulator buffers
 
 // Instruction descriptor: D fp32, A/B tf32, K-major both, N = 128, M = 128.
 constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(T >> 3) << 17) |
@@ -133,7 +133,8 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t *bars = (uint64_t *)(smem + kStages * kStageBytes);
-    // bars[0..S) full, bars[S..2S) empty, bars[2S] accumulator ready, bars[2S+1] drain
+    // bars: [0,S) stage full, [S,2S) stage empty, 2S+{0,1} accumulator full,
+    // 2S+{2,3} accumulator empty, 2S+4 drain
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
 
@@ -141,14 +142,23 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-    const uint32_t acc_bar = bar0 + 8u * (2 * kStages), drain_bar = acc_bar + 8u;
+    auto accf_bar = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
+    auto acce_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
 
     if (threadIdx.x == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&maps.a_hi) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&maps.a_lo) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&maps.b_hi) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&maps.b_lo) : "memory");
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        mbar_init(acc_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(accf_bar(b), 1);
+            mbar_init(acce_bar(b), 4);  // one arrive per epilogue warp
+        }
         mbar_init(drain_bar, 1);
         abort_sh = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -162,9 +172,16 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_d = tmem_base_sh;
+    const uint32_t tmem_base = tmem_base_sh;
+    pdl_wait();  // operands and the output tile were written by earlier kernels
 
-    const int nk = (it.k1 - it.k0) * (T / KB);
+    // The contraction runs over nchunk chunks of one tile (T = 128 columns) each.
+    // Chunk c accumulates from zero in TMEM buffer c & 1 (columns 128 (c&1) ..);
+    // the epilogue warps add every finished chunk into FP32 registers, which
+    // keeps the tensor cores' accumulation to 128-long sums.
+    constexpr int KB_PER_CHUNK = T / KB;
+    const int nchunk = it.k1 - it.k0;
+    const int nk = nchunk * KB_PER_CHUNK;
     const int kbase = it.k0 * T;
     const uint64_t deadline = now_ns() + (uint64_t)g.timeout_ms * 1000000ull;
 
@@ -188,67 +205,105 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
             tma_load_2d(base + 3 * kTileBytes, &maps.b_lo, x, it.rb * T, full_bar(s));
             issued = kb + 1;
         }
+        pdl_trigger();
         // make sure every issued copy has landed before the CTA can exit
         for (int kb = max(0, issued - kStages); kb < issued; ++kb)
             mbar_wait(full_bar(kb % kStages), (kb / kStages) & 1, deadline + 50000000ull);
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % kStages;
-            if (!mbar_wait(full_bar(s), (kb / kStages) & 1, deadline)) {
-                record_error(g.st, BAKRON_ERR_DEVICE_TIMEOUT, 2000 + STAGE);
-                atomicExch(&abort_sh, 1);
+        for (int c = 0; c < nchunk && ok; ++c) {
+            const int buf = c & 1;
+            if (c >= 2 && !mbar_wait(acce_bar(buf), ((c >> 1) - 1) & 1, deadline)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t base = smem_u32(smem + s * kStageBytes);
+            const uint32_t tmem_d = tmem_base + (uint32_t)(buf * T);
+            for (int kc = 0; kc < KB_PER_CHUNK; ++kc) {
+                const int kb = c * KB_PER_CHUNK + kc;
+                const int s = kb % kStages;
+                if (!mbar_wait(full_bar(s), (kb / kStages) & 1, deadline)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t base = smem_u32(smem + s * kStageBytes);
 #pragma unroll
-            for (int k8 = 0; k8 < KB / 8; ++k8) {
-                const uint32_t off = k8 * 32;  // 8 tf32 = 32 bytes along K inside the swizzle atom
-                const uint64_t ah = umma_desc(base + off), al = umma_desc(base + kTileBytes + off);
-                const uint64_t bh = umma_desc(base + 2 * kTileBytes + off), bl = umma_desc(base + 3 * kTileBytes + off);
-                umma_tf32(tmem_d, al, bh, (kb | k8) != 0);
-                umma_tf32(tmem_d, ah, bl, 1);
-                umma_tf32(tmem_d, ah, bh, 1);
+                for (int k8 = 0; k8 < KB / 8; ++k8) {
+                    const uint32_t off = k8 * 32;  // 8 tf32 = 32 bytes along K inside the swizzle atom
+                    const uint64_t ah = umma_desc(base + off), al = umma_desc(base + kTileBytes + off);
+                    const uint64_t bh = umma_desc(base + 2 * kTileBytes + off),
+                                   bl = umma_desc(base + 3 * kTileBytes + off);
+                    umma_tf32(tmem_d, al, bh, (kc | k8) != 0);
+                    umma_tf32(tmem_d, ah, bl, 1);
+                    umma_tf32(tmem_d, ah, bh, 1);
+                }
+                umma_commit(empty_bar(s));
             }
-            umma_commit(empty_bar(s));
+            if (ok) umma_commit(accf_bar(buf));
         }
-        umma_commit(ok ? acc_bar : drain_bar);
-        if (!ok) mbar_wait(drain_bar, 0, deadline + 50000000ull);
-    } else if (warp >= 2) {
-        // ---------------- epilogue: TMEM -> registers -> global
+        if (!ok) {
+            record_error(g.st, BAKRON_ERR_DEVICE_TIMEOUT, 2000 + STAGE);
+            atomicExch(&abort_sh, 1);
+            umma_commit(drain_bar);  // let issued MMAs finish before TMEM is released
+            mbar_wait(drain_bar, 0, deadline + 50000000ull);
+        }
+        pdl_trigger();
+    } else if (warp < 2) {
+        pdl_trigger();  // idle lanes of the producer and MMA warps
+    } else {
+        // ---------------- epilogue: per-chunk promotion TMEM -> FP32 registers, then store
         const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
-        int go = 0;
-        if (lane == 0) {
-            const bool ok = mbar_wait(acc_bar, 0, deadline);
-            if (!ok) {
-                record_error(g.st, BAKRON_ERR_DEVICE_TIMEOUT, 3000 + STAGE);
-                atomicExch(&abort_sh, 1);
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        float acc[T];
+#pragma unroll
+        for (int i = 0; i < T; ++i) acc[i] = 0.f;
+        bool good = true;
+        for (int c = 0; c < nchunk; ++c) {
+            const int buf = c & 1;
+            int go = 0;
+            if (lane == 0) {
+                const bool ok = mbar_wait(accf_bar(buf), (c >> 1) & 1, deadline);
+                if (!ok) {
+                    record_error(g.st, BAKRON_ERR_DEVICE_TIMEOUT, 3000 + STAGE);
+                    atomicExch(&abort_sh, 1);
+                }
+                go = ok && !*(volatile int *)&abort_sh;
             }
-            go = ok && !*(volatile int *)&abort_sh;
-        }
-        go = __shfl_sync(0xffffffffu, go, 0);  // warp-uniform: tcgen05.ld is .sync.aligned
-        if (go) {
+            go = __shfl_sync(0xffffffffu, go, 0);  // warp-uniform: tcgen05.ld is .sync.aligned
+            if (!go) {
+                good = false;
+                break;
+            }
             tc_fence_after();
-            const int r = quad * 32 + lane;
-            const int64_t orow = (int64_t)it.ra * T + r;
-            const int64_t ocol = (int64_t)it.rb * T;
-#pragma unroll 1
+#pragma unroll
             for (int c0 = 0; c0 < T; c0 += 32) {
                 float v[32];
-                tmem_ld32(tmem_d + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+                tmem_ld32(tmem_base + lane_off + (uint32_t)(buf * T + c0), v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[c0 + i] += v[i];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce_bar(buf)) : "memory");
+        }
+        pdl_trigger();
+        if (good) {
+            const int64_t orow = (int64_t)it.ra * T + quad * 32 + lane;
+            const int64_t ocol = (int64_t)it.rb * T;
+#pragma unroll
+            for (int c0 = 0; c0 < T; c0 += 32) {
                 if (STAGE == 1) {
                     float4 *hi = (float4 *)(g.out_hi + orow * g.ldo + ocol + c0);
                     float4 *lo = (float4 *)(g.out_lo + orow * g.ldo + ocol + c0);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         float4 h, l;
-                        split_tf32(v[4 * q + 0], h.x, l.x);
-                        split_tf32(v[4 * q + 1], h.y, l.y);
-                        split_tf32(v[4 * q + 2], h.z, l.z);
-                        split_tf32(v[4 * q + 3], h.w, l.w);
+                        split_tf32(acc[c0 + 4 * q + 0], h.x, l.x);
+                        split_tf32(acc[c0 + 4 * q + 1], h.y, l.y);
+                        split_tf32(acc[c0 + 4 * q + 2], h.z, l.z);
+                        split_tf32(acc[c0 + 4 * q + 3], h.w, l.w);
                         hi[q] = h;
                         lo[q] = l;
                     }
@@ -257,10 +312,10 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         float4 w = o[q];
-                        w.x -= v[4 * q + 0];
-                        w.y -= v[4 * q + 1];
-                        w.z -= v[4 * q + 2];
-                        w.w -= v[4 * q + 3];
+                        w.x -= acc[c0 + 4 * q + 0];
+                        w.y -= acc[c0 + 4 * q + 1];
+                        w.z -= acc[c0 + 4 * q + 2];
+                        w.w -= acc[c0 + 4 * q + 3];
                         o[q] = w;
                     }
                 }
@@ -271,7 +326,7 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(kTmemCols));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
     }
 }
 
@@ -333,12 +388,8 @@ bool make_tc_maps(int stage, int Mt, int Nt, const GemmArgs &g, TcMaps *maps)
 cudaError_t launch_band_tc(int stage, const NodeParams &np, const GemmArgs &g, const TcMaps &maps,
                            cudaStream_t stream)
 {
-    if (stage == 1) {
-        band_tc_kernel<1><<<dim3(np.l, np.Mt), kThreads, kSmem, stream>>>(maps, np, g);
-    } else {
-        band_tc_kernel<2><<<dim3(np.l - np.h, np.Mt), kThreads, kSmem, stream>>>(maps, np, g);
-    }
-    return cudaGetLastError();
+    if (stage == 1) return launch_pdl(band_tc_kernel<1>, dim3(np.l, np.Mt), dim3(kThreads), kSmem, stream, maps, np, g);
+    return launch_pdl(band_tc_kernel<2>, dim3(np.l - np.h, np.Mt), dim3(kThreads), kSmem, stream, maps, np, g);
 }
 
 }  // namespace bakron

@@ -4,7 +4,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/bakron.h"
+#include <utility>
+
+#include "bakron.h"
 
 namespace bakron {
 
@@ -28,6 +30,33 @@ __device__ __forceinline__ void record_error(DeviceStatus *st, int code, int whe
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// Programmatic dependent launch: every kernel of the solve is launched with
+// programmatic stream serialisation, so the next kernel's CTAs may start
+// (their prologue overlapping this kernel's tail) once every CTA of this one
+// has called pdl_trigger(); each kernel calls pdl_wait() before it touches
+// memory written by an earlier kernel, which blocks until the earlier grid
+// has completed and its writes are visible.  Both are no-ops for a kernel
+// launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 constexpr size_t kAlign = 1024;
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }

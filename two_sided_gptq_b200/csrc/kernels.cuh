@@ -35,7 +35,7 @@ cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, c
                         char *ws, cudaStream_t stream);
 
 cudaError_t leaf_configure();
-cudaError_t launch_leaf(const LeafArgs &p, int K, cudaStream_t stream);
+cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stream);
 
 // FP32 CUDA-core band products (reference kernels for the tensor-core path).
 cudaError_t launch_band_simt(int stage, const NodeParams &np, const GemmArgs &g, cudaStream_t stream);

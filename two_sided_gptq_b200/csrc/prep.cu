@@ -12,6 +12,8 @@ __global__ void scales_kernel(const float *__restrict__ W, int64_t m, int64_t n,
                               const float *__restrict__ user, float *__restrict__ s,
                               DeviceStatus *st)
 {
+    pdl_wait();
+    pdl_trigger();
     int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     int lane = threadIdx.x & 31;
     if (row >= m) return;
@@ -48,6 +50,8 @@ __global__ void pad_copy_kernel(const float *__restrict__ W, int64_t m, int64_t 
                                 int64_t Mp, float *__restrict__ Wt, float *__restrict__ Dhi,
                                 float *__restrict__ Dlo)
 {
+    pdl_wait();
+    pdl_trigger();
     int64_t total = Mp * Np;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
@@ -64,6 +68,8 @@ __global__ void normalize_split_kernel(const float *__restrict__ L, int64_t n, i
                                        float *__restrict__ L32, float *__restrict__ Lhi,
                                        float *__restrict__ Llo, DeviceStatus *st)
 {
+    pdl_wait();
+    pdl_trigger();
     int64_t total = Np * Np;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
@@ -98,14 +104,19 @@ cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, c
                         char *ws, cudaStream_t stream)
 {
     DeviceStatus *st = (DeviceStatus *)(ws + L.status);
-    scales_kernel<<<(unsigned)((m + 7) / 8), 256, 0, stream>>>(W, m, n, qmax, user_scales, scales, st);
-    pad_copy_kernel<<<grid_for(L.Mp * L.Np, 256), 256, 0, stream>>>(
-        W, m, n, L.Np, L.Mp, (float *)(ws + L.Wt), (float *)(ws + L.Dhi), (float *)(ws + L.Dlo));
-    normalize_split_kernel<<<grid_for(L.Np * L.Np, 256), 256, 0, stream>>>(
-        LA, n, L.Np, (float *)(ws + L.LA32), (float *)(ws + L.LAhi), (float *)(ws + L.LAlo), st);
-    normalize_split_kernel<<<grid_for(L.Mp * L.Mp, 256), 256, 0, stream>>>(
-        LB, m, L.Mp, (float *)(ws + L.LB32), (float *)(ws + L.LBhi), (float *)(ws + L.LBlo), st);
-    return cudaGetLastError();
+    cudaError_t e;
+    if ((e = launch_pdl(scales_kernel, dim3((unsigned)((m + 7) / 8)), dim3(256), 0, stream, W, m, n, qmax,
+                        user_scales, scales, st)) != cudaSuccess)
+        return e;
+    if ((e = launch_pdl(pad_copy_kernel, dim3(grid_for(L.Mp * L.Np, 256)), dim3(256), 0, stream, W, m, n, L.Np,
+                        L.Mp, (float *)(ws + L.Wt), (float *)(ws + L.Dhi), (float *)(ws + L.Dlo))) != cudaSuccess)
+        return e;
+    if ((e = launch_pdl(normalize_split_kernel, dim3(grid_for(L.Np * L.Np, 256)), dim3(256), 0, stream, LA, n,
+                        L.Np, (float *)(ws + L.LA32), (float *)(ws + L.LAhi), (float *)(ws + L.LAlo), st)) !=
+        cudaSuccess)
+        return e;
+    return launch_pdl(normalize_split_kernel, dim3(grid_for(L.Mp * L.Mp, 256)), dim3(256), 0, stream, LB, m, L.Mp,
+                      (float *)(ws + L.LB32), (float *)(ws + L.LBhi), (float *)(ws + L.LBlo), st);
 }
 
 }  // namespace bakron
