@@ -437,6 +437,15 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
     const int64_t row0 = (int64_t)I * T, col0 = (int64_t)J * T;
     const int mr = (int)min64(T, p.m - row0), nc = (int)min64(T, p.n - col0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // Warm L2 with the tile's two factor diagonal blocks (read by the products
+    // and the sweeps; each leaf launch uses blocks no earlier launch touched).
+    // A prefetch is only a hint, so it may run before the dependency wait.
+    for (int idx = tid; idx < 2 * T * (T / 32); idx += kThreadsW) {
+        const int which = idx / (T * (T / 32)), r = (idx / (T / 32)) % T, seg = idx % (T / 32);
+        const float *ptr = which == 0 ? p.LA32 + (col0 + r) * p.Np + col0 + 32 * seg
+                                      : p.LB32 + (row0 + r) * p.Mp + row0 + 32 * seg;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+    }
     pdl_wait();  // every global input (Wt, factors, steps) comes from earlier kernels
 
     for (int idx = tid; idx < T * RS3 / 4; idx += kThreadsW) {
@@ -510,7 +519,6 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
                 v.w = 4 * c + 3 < b ? v.w : 0.f;
                 la[c] = v;
             }
-            const float *Dcol = sDt + (q * S3 + b) * RS3 + pp * S3;
             const float *LBp = sLB + pp * S3 * WS3;
             const float *Wp = sW + pp * S3 * WS3;
             // newest-term coefficient LtA[b, b-1] (0 for b = 0)
@@ -518,54 +526,75 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
             // Software pipeline over the anti-diagonal steps.  At the start of step
             // d every entry on diagonals <= d-1 is final and every entry on
             // diagonal d is still zero in smem, so the dot products of this lane's
-            // NEXT entry (row a+1) loaded now automatically leave out exactly the
+            // NEXT entry (row a+1) read now automatically leave out exactly the
             // two terms that become final during step d; those are added at step
             // d+1 from R[a+1][b-1] (written by lane b-1) and this lane's own D.
+            // The lane's own column of D lives in registers (dcol[k] holds rows
+            // 4k..4k+3), so each step streams only one row of R and one row of
+            // LtB from smem, and only the chunks the lane needs.
+            float4 dcol[S3 / 4];
+#pragma unroll
+            for (int c = 0; c < S3 / 4; ++c) dcol[c] = make_float4(0.f, 0.f, 0.f, 0.f);
             float pu = 0.f, ps = 0.f;  // partial sums for the current entry
             float d_prev = 0.f;        // D[a-1][b]
+            const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int d = 0; d < 2 * S3 - 1; ++d) {
                 const int a = d - b;
-                const int an = min(max(a + 1, 0), S3 - 1);  // next entry's row (clamped)
-                // (1) bulk loads for the next entry, before any store of this step
-                const float *Rn = sR + (pp * S3 + an) * RS3 + q * S3;
-                const float *Bn = LBp + an * WS3;
-                float4 rv[8], bv[8], dv[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    rv[c] = *(const float4 *)(Rn + 4 * c);
-                    bv[c] = *(const float4 *)(Bn + 4 * c);
-                    dv[c] = *(const float4 *)(Dcol + 4 * c);
-                }
-                // (2) newest terms and the decision for the current entry (a, b)
                 const bool active = a >= 0 && a < S3;
                 const int ac = min(max(a, 0), S3 - 1);
+                const int an = min(max(a + 1, 0), S3 - 1);  // next entry's row (clamped)
+                // (1) critical loads first: they must not queue behind the bulk
                 const float r_new = b > 0 ? sR[(pp * S3 + ac) * RS3 + q * S3 + b - 1] : 0.f;
                 const float lb_new = ac > 0 ? LBp[ac * WS3 + ac - 1] : 0.f;
                 const float w0 = Wp[ac * WS3 + b];
-                const float uu = fmaf(r_new, la_new, pu), sc = fmaf(lb_new, d_prev, ps);
                 const int ta = pp * S3 + a, tb = q * S3 + b;
+                const float s = scale[ac + pp * S3], rs = rcp[ac + pp * S3];
+                // (2) bulk loads for the next entry (before any store of this step);
+                // a chunk is loaded only by lanes that need an index in it
+                const float *Rn = sR + (pp * S3 + an) * RS3 + q * S3;
+                const float *Bn = LBp + an * WS3;
+                float4 rv[S3 / 4], bv[S3 / 4];
+#pragma unroll
+                for (int c = 0; c < S3 / 4; ++c) {
+                    rv[c] = zero4;
+                    bv[c] = zero4;
+                    if (4 * c < b) rv[c] = *(const float4 *)(Rn + 4 * c);
+                    if (4 * c <= a) bv[c] = *(const float4 *)(Bn + 4 * c);
+                }
+                // (3) the current entry
+                const float uu = fmaf(r_new, la_new, pu), sc = fmaf(lb_new, d_prev, ps);
+                float dl = 0.f;
                 if (active && ta < mr && tb < nc) {
                     const float wt = w0 - uu - sc;
-                    const float s = scale[ta];
-                    const float c = decide(wt, s, rcp[ta], fqmin, fqmax);
-                    const float dl = fmaf(-s, c, wt);
+                    const float c = decide(wt, s, rs, fqmin, fqmax);
+                    dl = fmaf(-s, c, wt);
                     sR[ta * RS3 + tb] = sc + dl;
                     sDt[tb * RS3 + ta] = dl;
                     sCode[ta * T + tb] = (int8_t)c;
                     if (p.wt_out) p.wt_out[(row0 + ta) * p.n + col0 + tb] = wt;
-                    d_prev = dl;
-                } else {
-                    d_prev = 0.f;
                 }
-                // (3) partial sums of the next entry
+                // (4) partial sums of the next entry (dcol does not yet hold D[a][b])
                 float u4[4] = {0.f, 0.f, 0.f, 0.f}, s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < S3 / 4; ++c) {
                     u4[c & 3] = dot4(rv[c], la[c], u4[c & 3]);
-                    s4[c & 3] = dot4(bv[c], dv[c], s4[c & 3]);
+                    s4[c & 3] = dot4(bv[c], dcol[c], s4[c & 3]);
                 }
                 pu = (u4[0] + u4[1]) + (u4[2] + u4[3]);
                 ps = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+                // (5) D[a][b] into the register column
+                d_prev = dl;
+                {
+                    // branch-free insert: compare the row against each register slot
+                    const int row = active ? a : -1;
+#pragma unroll
+                    for (int c = 0; c < S3 / 4; ++c) {
+                        dcol[c].x = row == 4 * c + 0 ? dl : dcol[c].x;
+                        dcol[c].y = row == 4 * c + 1 ? dl : dcol[c].y;
+                        dcol[c].z = row == 4 * c + 2 ? dl : dcol[c].z;
+                        dcol[c].w = row == 4 * c + 3 ? dl : dcol[c].w;
+                    }
+                }
                 __syncwarp();
             }
         }
