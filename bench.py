@@ -31,6 +31,8 @@ METRIC = "quantized weights/sec for 4096×4096 INT4 BaKron solve; % tensor-pipe 
 TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 : BF16 tensor peak ratio
 FALLBACK_BF16_TFLOPS = 1590.0
 LEAF_BYTES_PER_WEIGHT = 25  # read Wt 4 + diagonal factor blocks 8; write code 1, V 4, D hi/lo 8
+LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 255), 3: ("leaf_warp_kernel", 7 * 63)}
+DEFAULT_LEAF = 3  # the library's default leaf structure
 
 
 def peaks():
@@ -95,7 +97,11 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
 
 
-def dist_setup(n_gpus):
+def dist_setup(backend="nccl", timeout_s=300):
+    """One process per GPU (torchrun env): returns rank, world size, local rank
+    and the torch.distributed module (None when running alone).  The only
+    collectives are the timing barriers and the max-over-ranks reductions:
+    each rank solves its own matrix."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws <= 1:
         return 0, 1, 0, None
@@ -105,9 +111,28 @@ def dist_setup(n_gpus):
     import torch.distributed as dist
 
     rank, local = int(os.environ["RANK"]), int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    kw = {}
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+        kw["device_id"] = torch.device("cuda", local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
     return rank, ws, local, dist
+
+
+def max_over_ranks(x, dist, device="cpu"):
+    """Max of a per-rank float over all ranks (identity when running alone)."""
+    if dist is None:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(world, m, n, ms_per_step):
+    """Whole-job weights/s: every rank solves one m x n matrix per step."""
+    return world * m * n / (ms_per_step / 1e3)
 
 
 def load_inputs(name, rank, dist):
@@ -122,7 +147,7 @@ def load_inputs(name, rank, dist):
     return W, A, B
 
 
-def cpu_baseline(W, A, B, bits, target_s=15.0):
+def cpu_baseline(W, A, B, bits, target_s=15.0, single_thread=False):
     """Oracle (FP64 anti-diagonal pull, OpenMP over each diagonal) timed on a
     bounded sample: the top r rows, a closed sub-problem (rows < r never depend
     on later rows), with r chosen for about ``target_s`` of work; the time is
@@ -151,10 +176,43 @@ def cpu_baseline(W, A, B, bits, target_s=15.0):
         r = min(m, 2 * r)
     t = run(r) if r != r0 else t0
     t_full = t * work(m) / work(r)
-    return {"value": m * n / t_full, "unit": "weights/s", "cores": threads, "kind": "oracle",
-            "sample": f"top {r} of {m} rows of the {m}x{n} workload (closed sub-problem), {t:.2f} s measured, "
-                      f"scaled x{work(m) / work(r):.2f} by multiply-add count",
-            "sample_seconds": t}
+    out = {"value": m * n / t_full, "unit": "weights/s", "cores": threads, "kind": "oracle",
+           "sample": f"top {r} of {m} rows of the {m}x{n} workload (closed sub-problem), {t:.2f} s measured, "
+                     f"scaled x{work(m) / work(r):.2f} by multiply-add count",
+           "sample_seconds": t, "nproc": os.cpu_count()}
+    if single_thread and threads > 1:
+        r1 = min(m, 64)
+        t1 = time.perf_counter()
+        oracle.solve(W[:r1], LtA, np.ascontiguousarray(LtB[:r1, :r1]), s[:r1], qmin, qmax, mode="pull", nthreads=1)
+        t1 = time.perf_counter() - t1
+        out["single_thread_value"] = m * n / (t1 * work(m) / work(r1))
+        out["single_thread_sample"] = f"top {r1} rows, 1 thread, {t1:.2f} s measured"
+    return out
+
+
+def band_levels(launches):
+    """Band-product time and tensor-pipe fraction per recursion level (node
+    width l in tile diagonals), medians over the profiled steps."""
+    by = {}
+    for step in launches:
+        acc = {}
+        for r in step:
+            if r["kind"] in ("stage1", "stage2"):
+                a = acc.setdefault(r["l"], [0.0, 0.0, 0])
+                a[0] += r["ms"]
+                a[1] += r["flops"]
+                a[2] += 1
+        for l, a in acc.items():
+            by.setdefault(l, []).append(a)
+    bf16, _, _ = peaks()
+    peak = bf16 * TF32_PER_BF16
+    out = []
+    for l in sorted(by, reverse=True):
+        ms = statistics.median(a[0] for a in by[l])
+        fl = by[l][0][1]
+        tf = 3.0 * fl / (ms / 1e3) / 1e12 if ms > 0 else 0.0
+        out.append({"l": l, "launches": by[l][0][2], "ms": ms, "flops": fl, "tflops": tf, "frac": tf / peak})
+    return out
 
 
 def run_reference(args):
@@ -213,7 +271,7 @@ def main():
     import two_sided_gptq_b200 as bk
     import workloads
 
-    rank, world, local, dist = dist_setup(args.gpus)
+    rank, world, local, dist = dist_setup("nccl")
     w = workloads.WORKLOADS[args.workload]
     W, A, B = load_inputs(args.workload, rank, dist)
     dev = torch.device("cuda", local)
@@ -259,21 +317,19 @@ def main():
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
-    elapsed = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     status = bk.get_status(ws)
     ms_per_step = elapsed / args.steps
-    value = world * m * n / (ms_per_step / 1e3)
+    value = aggregate_rate(world, m, n, ms_per_step)
 
     # per-kernel-class device times (separate profiled steps, events on the launch stream)
-    prof = []
+    prof, launches = [], []
     for _ in range(max(1, args.profile_steps)):
         bk.solve(Wd, LA, LB, bits=w.bits, ws=ws, out=out, check_status=False, stream=stream, profile=True)
         prof.append(bk.last_profile())
+        launches.append(bk.last_profile_launches())
     pr = {k: statistics.median(p[k] for p in prof) for k in prof[0]}
+    levels = band_levels(launches)
     plan = bk.plan_stats(m, n)
     bf16, hbm, src = peaks()
     tf32_peak = bf16 * TF32_PER_BF16
@@ -300,18 +356,14 @@ def main():
         bk.solve_host(Wh, LAh, LBh, bits=w.bits, V=Vh, codes=ch, scales=sh, ws=wsh, stream=stream, synchronize=False)
     h1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = h0.elapsed_time(h1) / e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(h0.elapsed_time(h1) / e2e_steps, dist, dev)
     assert np.array_equal(ch.numpy(), codes.cpu().numpy()), "host-buffer solve disagrees with device solve"
 
     line = None
     if rank == 0:
         cb = None
         if world == 1 and not args.no_cpu_baseline:
-            cb = cpu_baseline(W, A, B, w.bits)
+            cb = cpu_baseline(W, A, B, w.bits, single_thread=True)
         line = {
             "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -324,13 +376,18 @@ def main():
                 "flops_per_step": 3.0 * plan["update_flops"],
                 "flops_note": "3 TF32 MMAs per multiply-add (3xTF32) x algorithmic tile-product FLOPs of the schedule",
                 "band_ms_per_step": gemm_ms},
-            "leaf": {"kernel": "leaf_pull_kernel", "ms_per_step": pr["leaf_ms"], "launches_per_step": pr["leaf_launches"],
+            "band_levels": levels,
+            "leaf": {"kernel": LEAF_KERNELS[DEFAULT_LEAF][0], "ms_per_step": pr["leaf_ms"],
+                     "launches_per_step": pr["leaf_launches"],
                      "achieved_gbs": leaf_bytes / (pr["leaf_ms"] / 1e3) / 1e9, "hbm_peak_gbs": hbm,
-                     "bytes_per_step": leaf_bytes, "bound": "latency (2T-1 dependent steps per tile diagonal)"},
+                     "bytes_per_step": leaf_bytes, "bound": "latency (dependent rounding steps)",
+                     "sequential_steps_per_leaf": LEAF_KERNELS[DEFAULT_LEAF][1],
+                     "ns_per_sequential_step": pr["leaf_ms"] * 1e6 / (pr["leaf_launches"] * LEAF_KERNELS[DEFAULT_LEAF][1]),
+                     "share_of_profiled_step": pr["leaf_ms"] / pr["total_ms"]},
             "profile_ms": pr,
             "factor_ms": factor_ms,
             "cpu_baseline": cb,
-            "e2e": {"value": world * m * n / (e2e_ms / 1e3), "unit": "weights/s",
+            "e2e": {"value": aggregate_rate(world, m, n, e2e_ms), "unit": "weights/s",
                     "h2d_bytes_per_step": 4 * (m * n + n * n + m * m),
                     "d2h_bytes_per_step": 4 * m * n + m * n + 4 * m},
             "gpu_launches": launches_per_step * args.steps,

@@ -104,6 +104,19 @@ typedef struct {
 } bakron_profile_t;
 bakron_status_t bakron_get_profile(bakron_profile_t *out);
 
+/* One launch of the latest profiled bakron_solve on the calling host thread,
+ * in launch order: kind 0 prep (the four preparation kernels together), 1 leaf
+ * sweep of tile diagonal k, 2 / 3 stage 1 / stage 2 band product of the
+ * recursion node over tile diagonals [k, k+l) split at k+h; ms its
+ * CUDA-event interval; flops the algorithmic FLOPs of a band product (2 T^3
+ * per 128 x 128 x 128 tile product; 0 for other kinds). */
+typedef struct {
+    int32_t kind, k, h, l;
+    double ms, flops;
+} bakron_profile_launch_t;
+/* Copies min(count, cap) records to `out` (may be NULL) and returns count. */
+int64_t bakron_get_profile_launches(bakron_profile_launch_t *out, int64_t cap);
+
 /* ---------------------------------------------------------------- factor */
 /* Bytes of workspace bakron_factor needs for factors of sizes n and m. */
 size_t bakron_factor_workspace_size(int64_t n, int64_t m);

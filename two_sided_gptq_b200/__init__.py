@@ -16,9 +16,10 @@ from __future__ import annotations
 import ctypes
 
 from . import _native
-from ._native import BakronError, Config, PlanStats, Profile, Quantizer, Status, check
+from ._native import BakronError, Config, PlanStats, Profile, ProfileLaunch, Quantizer, Status, check
 
-__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile", "workspace", "get_status",
+__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile", "last_profile_launches",
+           "workspace", "get_status",
            "BakronError", "Status", "version", "library_path"]
 
 
@@ -183,6 +184,18 @@ def last_profile() -> dict:
     pr = Profile()
     check(_lib().bakron_get_profile(ctypes.byref(pr)), "bakron_get_profile")
     return {f: getattr(pr, f) for f, _ in Profile._fields_}
+
+
+def last_profile_launches() -> list:
+    """Every launch of the latest ``solve(..., profile=True)`` on this thread, in
+    launch order: dicts with kind ("prep", "leaf", "stage1", "stage2"), the
+    recursion node (k, h, l) in tile diagonals, ms and algorithmic FLOPs."""
+    lib = _lib()
+    n = lib.bakron_get_profile_launches(None, 0)
+    buf = (ProfileLaunch * max(1, n))()
+    lib.bakron_get_profile_launches(buf, n)
+    kinds = ("prep", "leaf", "stage1", "stage2")
+    return [{"kind": kinds[r.kind], "k": r.k, "h": r.h, "l": r.l, "ms": r.ms, "flops": r.flops} for r in buf[:n]]
 
 
 def plan_stats(m: int, n: int) -> dict:

@@ -57,6 +57,11 @@ class PlanStats(ctypes.Structure):
 
 # name -> (restype, argtypes); every function declared in include/bakron.h
 _vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+class ProfileLaunch(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("k", ctypes.c_int32), ("h", ctypes.c_int32), ("l", ctypes.c_int32),
+                ("ms", ctypes.c_double), ("flops", ctypes.c_double)]
+
+
 SIGNATURES = {
     "bakron_factor_workspace_size": (_sz, [_i64, _i64]),
     "bakron_factor": (ctypes.c_int, [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
@@ -74,6 +79,7 @@ SIGNATURES = {
     "bakron_plan_stats": (ctypes.c_int, [_i64, _i64, ctypes.POINTER(Config), ctypes.POINTER(PlanStats)]),
     "bakron_version": (ctypes.c_char_p, []),
     "bakron_get_profile": (ctypes.c_int, [ctypes.POINTER(Profile)]),
+    "bakron_get_profile_launches": (_i64, [ctypes.POINTER(ProfileLaunch), _i64]),
     "bakron_solve_noalloc": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, ctypes.POINTER(Quantizer), _vp, _vp, _vp,
                                             ctypes.POINTER(Config), _vp, ctypes.POINTER(ctypes.c_int32)]),
 }

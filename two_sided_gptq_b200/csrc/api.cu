@@ -42,6 +42,7 @@ struct Profiler {
     cudaStream_t stream = nullptr;
     std::vector<cudaEvent_t> pool;
     std::vector<int> kinds;
+    std::vector<NodeParams> nodes;
     size_t used = 0;
     cudaEvent_t next()
     {
@@ -52,10 +53,11 @@ struct Profiler {
         }
         return pool[used++];
     }
-    void begin(int kind)
+    void begin(int kind, NodeParams np = NodeParams{0, 0, 0, 0, 0})
     {
         if (!on) return;
         kinds.push_back(kind);
+        nodes.push_back(np);
         cudaEvent_t e = next();
         if (e) cudaEventRecord(e, stream);
     }
@@ -68,6 +70,22 @@ struct Profiler {
 };
 thread_local Profiler t_prof;
 thread_local bakron_profile_t t_last_profile = {};
+thread_local std::vector<bakron_profile_launch_t> t_last_launches;
+
+// Algorithmic FLOPs of one stage of one recursion node: 2 T^3 per tile
+// product over the node's items.
+double node_stage_flops(const NodeParams &np, int stage)
+{
+    const double t3 = 2.0 * kTile * (double)kTile * kTile;
+    double f = 0.0;
+    const int cols = stage == 1 ? np.l : np.l - np.h;
+    for (int I = 0; I < np.Mt; ++I)
+        for (int x = 0; x < cols; ++x) {
+            Item it = stage == 1 ? stage1_item(np, x, I) : stage2_item(np, x, I);
+            if (it.valid) f += t3 * (it.k1 - it.k0);
+        }
+    return f;
+}
 
 bakron_status_t read_config(const bakron_config_t *c, Config &out)
 {
@@ -133,7 +151,7 @@ struct SolveCtx {
 cudaError_t run_band(const SolveCtx &c, int stage, const NodeParams &np)
 {
     const GemmArgs &g = stage == 1 ? c.s1 : c.s2;
-    t_prof.begin(stage + 1);
+    t_prof.begin(stage + 1, np);
     cudaError_t e = c.gemm == 1 ? launch_band_simt(stage, np, g, c.stream)
                                 : launch_band_tc(stage, np, g, stage == 1 ? c.m1 : c.m2, c.stream);
     t_prof.end();
@@ -143,7 +161,7 @@ cudaError_t run_band(const SolveCtx &c, int stage, const NodeParams &np)
 cudaError_t run_schedule(const SolveCtx &c, int k, int l)
 {
     if (l <= 1) {
-        t_prof.begin(1);
+        t_prof.begin(1, NodeParams{k, 0, 1, c.leaf.Mt, c.leaf.Nt});
         cudaError_t e = launch_leaf(c.leaf, k, c.leaf_variant, c.stream);
         t_prof.end();
         return e;
@@ -187,6 +205,7 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
     t_prof.stream = stream;
     t_prof.used = 0;
     t_prof.kinds.clear();
+    t_prof.nodes.clear();
     t_prof.begin(0);
     if (launch_prep(W, m, n, LA, LB, qmax, q->row_scale, scales, L, w, stream) != cudaSuccess)
         return BAKRON_ERR_CUDA;
@@ -228,11 +247,22 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
         bakron_profile_t pr = {};
         double *ms[4] = {&pr.prep_ms, &pr.leaf_ms, &pr.stage1_ms, &pr.stage2_ms};
         int64_t *cnt[4] = {&pr.prep_launches, &pr.leaf_launches, &pr.stage1_launches, &pr.stage2_launches};
+        t_last_launches.clear();
         for (size_t i = 0; i < t_prof.kinds.size() && 2 * i + 1 < t_prof.used; ++i) {
             float dt = 0.f;
             cudaEventElapsedTime(&dt, t_prof.pool[2 * i], t_prof.pool[2 * i + 1]);
-            *ms[t_prof.kinds[i]] += dt;
-            *cnt[t_prof.kinds[i]] += 1;
+            const int kind = t_prof.kinds[i];
+            *ms[kind] += dt;
+            *cnt[kind] += 1;
+            const NodeParams &np = t_prof.nodes[i];
+            bakron_profile_launch_t r;
+            r.kind = kind;
+            r.k = np.k;
+            r.h = np.h;
+            r.l = np.l;
+            r.ms = dt;
+            r.flops = kind >= 2 ? node_stage_flops(np, kind - 1) : 0.0;
+            t_last_launches.push_back(r);
         }
         pr.prep_launches *= 4;  // scales, padded copy, two factor normalisations
         float tot = 0.f;
@@ -252,17 +282,8 @@ void count_schedule(int k, int l, int Mt, int Nt, bakron_plan_stats_t *o)
     const int h = l / 2;
     count_schedule(k, h, Mt, Nt, o);
     NodeParams np{k, h, l, Mt, Nt};
-    const double t3 = 2.0 * kTile * (double)kTile * kTile;  // FLOPs of one T x T x T tile product
-    for (int I = 0; I < Mt; ++I)
-        for (int x = 0; x < l; ++x) {
-            Item it = stage1_item(np, x, I);
-            if (it.valid) o->stage1_flops += t3 * (it.k1 - it.k0);
-        }
-    for (int I = 0; I < Mt; ++I)
-        for (int x = 0; x < l - h; ++x) {
-            Item it = stage2_item(np, x, I);
-            if (it.valid) o->stage2_flops += t3 * (it.k1 - it.k0);
-        }
+    o->stage1_flops += node_stage_flops(np, 1);
+    o->stage2_flops += node_stage_flops(np, 2);
     o->nodes++;
     count_schedule(k + h, l - h, Mt, Nt, o);
 }
@@ -438,6 +459,14 @@ bakron_status_t bakron_get_status(void *ws_dev, size_t ws_bytes, bakron_stream_t
     if (cudaMemcpy(&h, ws_dev, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return BAKRON_ERR_CUDA;
     if (h.code != 0 && cudaMemset(ws_dev, 0, sizeof(h)) != cudaSuccess) return BAKRON_ERR_CUDA;
     return (bakron_status_t)h.code;
+}
+
+int64_t bakron_get_profile_launches(bakron_profile_launch_t *out, int64_t cap)
+{
+    const int64_t n = (int64_t)t_last_launches.size();
+    if (out)
+        for (int64_t i = 0; i < n && i < cap; ++i) out[i] = t_last_launches[(size_t)i];
+    return n;
 }
 
 bakron_status_t bakron_get_profile(bakron_profile_t *out)
