@@ -60,6 +60,19 @@ __device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc)
     return fmaf(a.w, b.w, acc);
 }
 
+// Two FP32 fused multiply-adds in one packed instruction (sm_100), each
+// rounded to nearest like fmaf.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
 // Rounding decision clamp(rint(wt / s)) with the IEEE fp32 quotient.  Fast
 // path: q = wt * (1/s) is within 2 ulp of the IEEE quotient; whenever q is
 // not within 0.002 of a half-integer (and |q| <= 2^12, beyond which every
@@ -364,21 +377,29 @@ __global__ void __launch_bounds__(kThreads, 1) leaf_single_kernel(LeafArgs p, in
 }
 
 // ------------------------------------------------------------------------
-// Warp-per-sub-tile variant: 4 x 4 sub-tiles of 32, processed in sub-tile
-// diagonal order e = 0..6.  Before phase e, the cross-sub-tile terms of every
-// sub-tile (p, q) with p + q = e are applied left-looking with all 16 warps:
+// Warp-pair-per-sub-tile variant: 4 x 4 sub-tiles of 32, processed in
+// sub-tile diagonal order e = 0..6.  Before phase e, the cross-sub-tile terms
+// of every sub-tile (p, q) with p + q = e are applied left-looking with all 8
+// warps:
 //     S[p,q] = sum_{p'<p} LtB[p,p'] D[p',q],
 //     Wt[p,q] -= sum_{q'<q} R[p,q'] LtA[q,q']^T + S[p,q] LtA[q,q]^T,
 // where R[p,q'] = sum_{p'<=p} LtB[p,p'] D[p',q'] is complete for q' < q.  Then
-// warp p sweeps sub-tile (p, q) alone (lane = column, 63 warp-synchronous
-// steps), and finally R[p,q] = S[p,q] + (the sweep's in-sub-tile R).
-// sR and sDt start at zero, so entries not yet rounded contribute nothing to
-// the sweep's dot products and no masking is needed.
+// warps 2p and 2p+1 sweep sub-tile (p, q) (63 entry anti-diagonal steps, one
+// pair barrier each) and finally R[p,q] = S[p,q] + (the sweep's in-sub-tile R).
+// In the sweep, entry (a, b) needs
+//     Wt_ab = W0_ab - sum_{c<b} R_ac LtA[b,c] - sum_{r<a} LtB[a,r] D_rb:
+// warp A (lane = column b) rounds the entries and keeps the row-side sum,
+// whose operands are its own LtA row (registers) and rows of R (smem); warp B
+// (lane = row rho) keeps the column-side sum, whose operands are its own LtB
+// row (registers) and columns of D (smem).  Both sums are formed a step ahead
+// without their newest term, which warp A adds from the values the previous
+// step produced.  sR and sDt start at zero.
 namespace {
 constexpr int S3 = 32;             // sub-tile side
 constexpr int RS3 = T + 4;         // row stride of sR / sDt: 33 float4 per row
 constexpr int WS3 = S3 + 4;        // row stride of the per-row-block slots
-constexpr size_t kSmemWarp = ((size_t)2 * T * RS3 + 3 * 4 * S3 * WS3 + 2 * T) * sizeof(float) + (size_t)T * T;
+constexpr size_t kSmemWarp =
+    ((size_t)2 * (T + 1) * RS3 + 3 * 4 * S3 * WS3 + 2 * T + 2 * 4 * 2 * S3) * sizeof(float) + (size_t)T * T + 32;
 static_assert(kSmemWarp <= 232448, "leaf shared memory");
 }  // namespace
 
@@ -419,19 +440,29 @@ __device__ __forceinline__ void mma_block(float (&acc)[NT][4], const float *A, i
     }
 }
 
-constexpr int kThreadsW = 256;  // warp variant: 4 sweeping warps, 2 product warps per row block
+constexpr int kThreadsW = 384;  // warp variant: 3 warps per row block of sub-tiles
+
+// Byte of an integer-valued float in [-128, 127] (two's complement) without a
+// conversion instruction: adding 1.5 * 2^23 puts the integer in the low
+// mantissa bits.
+__device__ __forceinline__ int8_t code_byte(float c)
+{
+    return (int8_t)(__float_as_int(c + 12582912.0f) & 0xFF);
+}
 
 __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int K, int I_lo)
 {
     extern __shared__ __align__(16) float smem_f[];
-    float *sR = smem_f;                 // T x RS3: R (full for finished sub-tiles), 0 elsewhere
-    float *sDt = sR + T * RS3;          // T x RS3: D transposed, 0 where not rounded yet
-    float *sW = sDt + T * RS3;          // 4 slots of S3 x WS3: Wt of the sub-tile being swept per row block
-    float *sS = sW + 4 * S3 * WS3;      // 4 slots: S[p,q]
-    float *sLB = sS + 4 * S3 * WS3;     // 4 slots: LtB[p,p]
-    float *scale = sLB + 4 * S3 * WS3;  // T
-    float *rcp = scale + T;             // T
-    int8_t *sCode = (int8_t *)(rcp + T); // T x T codes
+    float *sR = smem_f;                  // T x RS3 (+1 spare row): R, 0 where not rounded yet
+    float *sDt = sR + (T + 1) * RS3;     // T x RS3 (+1 spare row): D transposed, 0 where not rounded yet
+    float *sW = sDt + (T + 1) * RS3;     // 4 slots of S3 x WS3: W0 of the sub-tile being swept, then Wt
+    float *sS = sW + 4 * S3 * WS3;       // 4 slots: S[p,q]
+    float *sLB = sS + 4 * S3 * WS3;      // 4 slots: LtB[p,p]
+    float *scale = sLB + 4 * S3 * WS3;   // T
+    float *rcp = scale + T;              // T
+    float *sPS = rcp + T;                // 4 x 2 x S3: column-side partial sums by column
+    float *sPU = sPS + 4 * 2 * S3;       // 4 x 2 x S3: row-side partial sums by column
+    int8_t *sCode = (int8_t *)(sPU + 4 * 2 * S3);  // T x T codes (+32 spare bytes)
 
     const int I = I_lo + blockIdx.x, J = K - I;
     const int64_t row0 = (int64_t)I * T, col0 = (int64_t)J * T;
@@ -448,7 +479,7 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
     }
     pdl_wait();  // every global input (Wt, factors, steps) comes from earlier kernels
 
-    for (int idx = tid; idx < T * RS3 / 4; idx += kThreadsW) {
+    for (int idx = tid; idx < (T + 1) * RS3 / 4; idx += kThreadsW) {
         ((float4 *)sR)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
         ((float4 *)sDt)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
@@ -463,15 +494,15 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
     const float *LBt = p.LB32 + row0 * p.Mp + row0;  // LtB diagonal block of the tile (global)
     const int lda_g = (int)p.Np, ldb_g = (int)p.Mp;
     const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
-    const int wp = warp >> 1;                          // products: warp -> (row block, 16 x 32 half)
-    const int i0 = (warp & 1) * 16, j0 = 0;
+    const int wp = warp / 3, role = warp - 3 * wp;  // row block of sub-tiles; 0 entries, 1 row side, 2 column side
+    const int i0 = (role & 1) * 16, j0 = 0;         // products: roles 0 and 1 take a 16 x 32 half each
 
     for (int e = 0; e < 7; ++e) {
         const int p_lo = max(0, e - 3), p_hi = min(3, e);
         const bool mine = wp >= p_lo && wp <= p_hi;  // this warp's row block has a sub-tile in phase e
         const int qv = e - wp;
         // S[p,q] = LtB[p, 0:p] D[0:p, q]
-        if (mine) {
+        if (mine && role < 2) {
             float acc[4][4] = {};
             if (wp > 0)
                 mma_block<4>(acc, LBt + (wp * S3) * ldb_g, ldb_g, sDt + (qv * S3) * RS3, RS3, wp * S3, i0, j0);
@@ -487,8 +518,8 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
             }
         }
         __syncthreads();
-        // Wt[p,q] = Wt_global - (R[p, 0:q] LtA[q, 0:q]^T + S[p,q] LtA[q,q]^T)
-        if (mine) {
+        // W0[p,q] = Wt_global - (R[p, 0:q] LtA[q, 0:q]^T + S[p,q] LtA[q,q]^T)
+        if (mine && role < 2) {
             float acc[4][4] = {};
             const float *LAq = LAt + (qv * S3) * lda_g;
             if (qv > 0) mma_block<4>(acc, sR + (wp * S3) * RS3, RS3, LAq, lda_g, qv * S3, i0, j0);
@@ -506,103 +537,151 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
             }
         }
         __syncthreads();
-        // sweep: warp p takes sub-tile (p, e - p), lane = column
-        if (warp <= 3 && warp >= p_lo && warp <= p_hi) {
-            const int pp = warp, q = e - pp, b = lane;
-            float4 la[S3 / 4];  // LtA[q,q] row b, strictly lower part
-#pragma unroll
-            for (int c = 0; c < S3 / 4; ++c) {
-                float4 v = *(const float4 *)(LAt + (q * S3 + b) * lda_g + q * S3 + 4 * c);
-                v.x = 4 * c + 0 < b ? v.x : 0.f;
-                v.y = 4 * c + 1 < b ? v.y : 0.f;
-                v.z = 4 * c + 2 < b ? v.z : 0.f;
-                v.w = 4 * c + 3 < b ? v.w : 0.f;
-                la[c] = v;
-            }
+        // sweep: warps 3p, 3p+1, 3p+2 take sub-tile (p, e - p) together, one
+        // barrier of the three per entry anti-diagonal step
+        if (mine) {
+            const int pp = wp, q = e - pp;
             const float *LBp = sLB + pp * S3 * WS3;
-            const float *Wp = sW + pp * S3 * WS3;
-            // newest-term coefficient LtA[b, b-1] (0 for b = 0)
-            const float la_new = b > 0 ? LAt[(q * S3 + b) * lda_g + q * S3 + b - 1] : 0.f;
-            // Software pipeline over the anti-diagonal steps.  At the start of step
-            // d every entry on diagonals <= d-1 is final and every entry on
-            // diagonal d is still zero in smem, so the dot products of this lane's
-            // NEXT entry (row a+1) read now automatically leave out exactly the
-            // two terms that become final during step d; those are added at step
-            // d+1 from R[a+1][b-1] (written by lane b-1) and this lane's own D.
-            // The lane's own column of D lives in registers (dcol[k] holds rows
-            // 4k..4k+3), so each step streams only one row of R and one row of
-            // LtB from smem, and only the chunks the lane needs.
-            float4 dcol[S3 / 4];
-#pragma unroll
-            for (int c = 0; c < S3 / 4; ++c) dcol[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-            float pu = 0.f, ps = 0.f;  // partial sums for the current entry
-            float d_prev = 0.f;        // D[a-1][b]
-            const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int d = 0; d < 2 * S3 - 1; ++d) {
-                const int a = d - b;
-                const bool active = a >= 0 && a < S3;
-                const int ac = min(max(a, 0), S3 - 1);
-                const int an = min(max(a + 1, 0), S3 - 1);  // next entry's row (clamped)
-                // (1) critical loads first: they must not queue behind the bulk
-                const float r_new = b > 0 ? sR[(pp * S3 + ac) * RS3 + q * S3 + b - 1] : 0.f;
-                const float lb_new = ac > 0 ? LBp[ac * WS3 + ac - 1] : 0.f;
-                const float w0 = Wp[ac * WS3 + b];
-                const int ta = pp * S3 + a, tb = q * S3 + b;
-                const float s = scale[ac + pp * S3], rs = rcp[ac + pp * S3];
-                // (2) bulk loads for the next entry (before any store of this step);
-                // a chunk is loaded only by lanes that need an index in it
-                const float *Rn = sR + (pp * S3 + an) * RS3 + q * S3;
-                const float *Bn = LBp + an * WS3;
-                float4 rv[S3 / 4], bv[S3 / 4];
-#pragma unroll
-                for (int c = 0; c < S3 / 4; ++c) {
-                    rv[c] = zero4;
-                    bv[c] = zero4;
-                    if (4 * c < b) rv[c] = *(const float4 *)(Rn + 4 * c);
-                    if (4 * c <= a) bv[c] = *(const float4 *)(Bn + 4 * c);
-                }
-                // (3) the current entry
-                const float uu = fmaf(r_new, la_new, pu), sc = fmaf(lb_new, d_prev, ps);
-                float dl = 0.f;
-                if (active && ta < mr && tb < nc) {
-                    const float wt = w0 - uu - sc;
-                    const float c = decide(wt, s, rs, fqmin, fqmax);
-                    dl = fmaf(-s, c, wt);
-                    sR[ta * RS3 + tb] = sc + dl;
-                    sDt[tb * RS3 + ta] = dl;
-                    sCode[ta * T + tb] = (int8_t)c;
-                    if (p.wt_out) p.wt_out[(row0 + ta) * p.n + col0 + tb] = wt;
-                }
-                // (4) partial sums of the next entry (dcol does not yet hold D[a][b])
-                float u4[4] = {0.f, 0.f, 0.f, 0.f}, s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int c = 0; c < S3 / 4; ++c) {
-                    u4[c & 3] = dot4(rv[c], la[c], u4[c & 3]);
-                    s4[c & 3] = dot4(bv[c], dcol[c], s4[c & 3]);
-                }
-                pu = (u4[0] + u4[1]) + (u4[2] + u4[3]);
-                ps = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-                // (5) D[a][b] into the register column
-                d_prev = dl;
-                {
-                    // branch-free insert: compare the row against each register slot
-                    const int row = active ? a : -1;
-#pragma unroll
-                    for (int c = 0; c < S3 / 4; ++c) {
-                        dcol[c].x = row == 4 * c + 0 ? dl : dcol[c].x;
-                        dcol[c].y = row == 4 * c + 1 ? dl : dcol[c].y;
-                        dcol[c].z = row == 4 * c + 2 ? dl : dcol[c].z;
-                        dcol[c].w = row == 4 * c + 3 ? dl : dcol[c].w;
+            float *ps_buf = sPS + pp * 2 * S3;  // [2][S3]: column-side sums, by column
+            float *pu_buf = sPU + pp * 2 * S3;  // [2][S3]: row-side sums, by column
+            float *Wp = sW + pp * S3 * WS3;
+            const int bar_id = 1 + pp;
+            if (role == 0) {
+                // ---- entry warp (lane = column b): rounds entry (d - b, b) at step d
+                const int b = lane, tb = q * S3 + b;
+                const float la_new = b > 0 ? LAt[(q * S3 + b) * lda_g + q * S3 + b - 1] : 0.f;
+                // row-dependent constants of an entry, loaded a step before it is rounded
+                auto row_consts = [&](int a, float &w0, float &lbn, float &sv, float &rv_) {
+                    const int ac = min(max(a, 0), S3 - 1);
+                    w0 = Wp[ac * WS3 + b];
+                    lbn = ac > 0 ? LBp[ac * WS3 + ac - 1] : 0.f;
+                    sv = scale[pp * S3 + ac];
+                    rv_ = rcp[pp * S3 + ac];
+                };
+                float w0, lb_new, sc_s, sc_r;
+                row_consts(-b, w0, lb_new, sc_s, sc_r);
+                float d_prev = 0.f;
+#pragma unroll 2
+                for (int d = 0; d < 2 * S3 - 1; ++d) {
+                    const int a = d - b;
+                    const int ac = min(max(a, 0), S3 - 1);
+                    // the values the previous step produced (the other warps' sums
+                    // leave out the newest row and column terms, added here)
+                    const float ps_in = d > 0 ? ps_buf[(d & 1) * S3 + b] : 0.f;
+                    const float pu_in = d > 0 ? pu_buf[(d & 1) * S3 + b] : 0.f;
+                    const float r_new = b > 0 ? sR[(pp * S3 + ac) * RS3 + tb - 1] : 0.f;
+                    float w0n, lbn_n, sn, rn;
+                    row_consts(a + 1, w0n, lbn_n, sn, rn);
+                    const float sc = fmaf(lb_new, d_prev, ps_in);
+                    const float wt = w0 - fmaf(r_new, la_new, pu_in) - sc;
+                    // clamp(rint(wt / s)) with the IEEE quotient (see decide); the exact
+                    // division runs only when some lane of the warp is near a midpoint
+                    const float qf = wt * sc_r;
+                    float cq = rintf(qf);
+                    const bool near = fabsf(qf - cq) > 0.498f && fabsf(qf) <= 4096.f;
+                    if (__any_sync(0xffffffffu, near)) {
+                        if (near) cq = rintf(__fdiv_rn(wt, sc_s));
                     }
+                    cq = fminf(fmaxf(cq, fqmin), fqmax);
+                    const int ta = pp * S3 + a;
+                    const bool valid = a >= 0 && a < S3 && ta < mr && tb < nc;
+                    const float dl = valid ? fmaf(-sc_s, cq, wt) : 0.f;
+                    // invalid lanes write to the spare row / bytes instead of branching
+                    const int iR = valid ? ta * RS3 + tb : T * RS3 + lane;
+                    const int iD = valid ? tb * RS3 + ta : T * RS3 + lane;
+                    const int iC = valid ? ta * T + tb : T * T + lane;
+                    const int iW = valid ? a * WS3 + b : ac * WS3 + S3 + (lane & 3);  // spare: row padding
+                    sR[iR] = sc + dl;
+                    sDt[iD] = dl;
+                    sCode[iC] = code_byte(cq);
+                    Wp[iW] = wt;  // pre-rounding value, copied out when requested
+                    d_prev = dl;
+                    w0 = w0n; lb_new = lbn_n; sc_s = sn; sc_r = rn;
+                    group_sync(bar_id, 96);
                 }
-                __syncwarp();
+            } else if (role == 1) {
+                // ---- row-side warp (lane = column b): sum_{c <= b-2} R[a+1][c] LtA[b][c]
+                // for the entry warp's next entry (a+1, b).  Column b-1 of that R
+                // row is written during this step; its coefficient here is zero.
+                const int b = lane;
+                float2 la[S3 / 2];
+#pragma unroll
+                for (int c = 0; c < S3 / 2; ++c) {
+                    float2 v = *(const float2 *)(LAt + (q * S3 + b) * lda_g + q * S3 + 2 * c);
+                    v.x = 2 * c + 0 <= b - 2 ? v.x : 0.f;
+                    v.y = 2 * c + 1 <= b - 2 ? v.y : 0.f;
+                    la[c] = v;
+                }
+                float4 rv[S3 / 4];  // chunks this lane never loads stay zero
+#pragma unroll
+                for (int c = 0; c < S3 / 4; ++c) rv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                for (int d = 0; d < 2 * S3 - 1; ++d) {
+                    const int an = min(max(d - b + 1, 0), S3 - 1);
+                    const float *Rn = sR + (pp * S3 + an) * RS3 + q * S3;
+#pragma unroll
+                    for (int c = 0; c < S3 / 4; ++c)
+                        if (4 * c <= b - 2) rv[c] = *(const float4 *)(Rn + 4 * c);
+                    float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
+                    float2 u2 = make_float2(0.f, 0.f), u3 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int c = 0; c < S3 / 4; c += 2) {
+                        u0 = ffma2(make_float2(rv[c].x, rv[c].y), la[2 * c], u0);
+                        u1 = ffma2(make_float2(rv[c].z, rv[c].w), la[2 * c + 1], u1);
+                        u2 = ffma2(make_float2(rv[c + 1].x, rv[c + 1].y), la[2 * c + 2], u2);
+                        u3 = ffma2(make_float2(rv[c + 1].z, rv[c + 1].w), la[2 * c + 3], u3);
+                    }
+                    pu_buf[((d + 1) & 1) * S3 + b] = ((u0.x + u1.x) + (u2.x + u3.x)) + ((u0.y + u1.y) + (u2.y + u3.y));
+                    group_sync(bar_id, 96);
+                }
+            } else {
+                // ---- column-side warp (lane = row rho): sum_{r <= rho-2} LtB[rho][r] D[r][b]
+                // for the entry warp's entry (rho, b = d+1-rho) at step d+1.  Row
+                // rho-1 of that D column is written during this step; its
+                // coefficient here is zero.
+                const int rho = lane;
+                float2 lbr[S3 / 2];
+#pragma unroll
+                for (int c = 0; c < S3 / 2; ++c) {
+                    float2 v = *(const float2 *)(LBp + rho * WS3 + 2 * c);
+                    v.x = 2 * c + 0 <= rho - 2 ? v.x : 0.f;
+                    v.y = 2 * c + 1 <= rho - 2 ? v.y : 0.f;
+                    lbr[c] = v;
+                }
+                float4 dv[S3 / 4];
+#pragma unroll
+                for (int c = 0; c < S3 / 4; ++c) dv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                for (int d = 0; d < 2 * S3 - 1; ++d) {
+                    const int b = d + 1 - rho;
+                    const int bc = min(max(b, 0), S3 - 1);
+                    const float *Dc = sDt + (q * S3 + bc) * RS3 + pp * S3;
+#pragma unroll
+                    for (int c = 0; c < S3 / 4; ++c)
+                        if (4 * c <= rho - 2) dv[c] = *(const float4 *)(Dc + 4 * c);
+                    float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+                    float2 s2 = make_float2(0.f, 0.f), s3 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int c = 0; c < S3 / 4; c += 2) {
+                        s0 = ffma2(make_float2(dv[c].x, dv[c].y), lbr[2 * c], s0);
+                        s1 = ffma2(make_float2(dv[c].z, dv[c].w), lbr[2 * c + 1], s1);
+                        s2 = ffma2(make_float2(dv[c + 1].x, dv[c + 1].y), lbr[2 * c + 2], s2);
+                        s3 = ffma2(make_float2(dv[c + 1].z, dv[c + 1].w), lbr[2 * c + 3], s3);
+                    }
+                    if (b == bc)
+                        ps_buf[((d + 1) & 1) * S3 + b] = ((s0.x + s1.x) + (s2.x + s3.x)) + ((s0.y + s1.y) + (s2.y + s3.y));
+                    group_sync(bar_id, 96);
+                }
             }
         }
         __syncthreads();
-        // R[p,q] = S[p,q] + in-sub-tile R
+        // R[p,q] = S[p,q] + in-sub-tile R; the pre-rounding values when requested
         for (int idx = tid; idx < (p_hi - p_lo + 1) * S3 * S3; idx += kThreadsW) {
             const int pp = p_lo + idx / (S3 * S3), r = (idx / S3) % S3, c = idx % S3;
             sR[(pp * S3 + r) * RS3 + (e - pp) * S3 + c] += sS[pp * S3 * WS3 + r * WS3 + c];
+            const int ta = pp * S3 + r, tb = (e - pp) * S3 + c;
+            if (p.wt_out && ta < mr && tb < nc)
+                p.wt_out[(row0 + ta) * p.n + col0 + tb] = sW[pp * S3 * WS3 + r * WS3 + c];
         }
         __syncthreads();
     }
