@@ -11,7 +11,11 @@
 //
 // Warp roles (192 threads): warp 0 lane 0 issues TMA into a 3-stage ring;
 // warp 1 owns TMEM and lane 0 issues the MMAs; warps 2..5 read the
-// accumulator back (tcgen05.ld, 32 lanes each) and write the tile.
+// accumulator back (tcgen05.ld, 32 lanes each), write their rows of the
+// finished tile into the then idle stage buffers in the swizzled box layout,
+// and hand each 32 x 32 box to TMA: a tile store for stage 1 (X^T hi and lo),
+// a tile add-reduction of -D into Wt for stage 2 (each Wt tile has one writer
+// per launch, so the single rounding of Wt + (-D) equals a read-modify-write).
 // Every mbarrier wait is bounded by a %globaltimer deadline; on expiry the
 // kernel records BAKRON_ERR_DEVICE_TIMEOUT, drains what it issued and exits.
 #include <cuda.h>
@@ -26,6 +30,7 @@ constexpr int T = kTile;
 constexpr int KB = 32;                    // fp32 columns per stage (128 bytes)
 constexpr int kStages = 3;
 constexpr int kTileBytes = T * KB * 4;    // 16 KB per operand part
+constexpr int kBoxBytes = 32 * KB * 4;    // 4 KB: one 32 x 32 output box
 constexpr int kStageBytes = 4 * kTileBytes;
 constexpr int kThreads = 192;
 constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
@@ -97,6 +102,34 @@ __device__ __forceinline__ void umma_tf32(uint32_t tmem_d, uint64_t adesc, uint6
 __device__ __forceinline__ void umma_commit(uint32_t bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+// Tile store (stage 1) and tile add-reduction (stage 2) from shared memory
+// through the tensor map, tracked as one bulk async-group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, uint32_t src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
+                 ::"l"((uint64_t)map), "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_add_2d(const CUtensorMap *map, int x, int y, uint32_t src)
+{
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];"
+                 ::"l"((uint64_t)map), "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+// Commit the bulk stores and wait until they have read their shared-memory
+// source (the global writes complete with the grid).
+__device__ __forceinline__ void bulk_commit_and_wait_read()
+{
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// L2 prefetch of one box through a tensor map (a hint; no completion).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, int y)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"((uint64_t)map), "r"(x),
+                 "r"(y)
                  : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -173,6 +206,16 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
+    if (threadIdx.x == 0) {
+        // The A operand is a normalised factor, written by the preparation
+        // kernels long before: warm L2 with its first boxes while the previous
+        // kernel finishes (a prefetch is only a hint).
+        const int nk_pre = min((it.k1 - it.k0) * (T / KB), 8);
+        for (int kb = 0; kb < nk_pre; ++kb) {
+            tma_prefetch_2d(&maps.a_hi, it.k0 * T + kb * KB, it.ra * T);
+            tma_prefetch_2d(&maps.a_lo, it.k0 * T + kb * KB, it.ra * T);
+        }
+    }
     pdl_wait();  // operands and the output tile were written by earlier kernels
 
     // The contraction runs over nchunk chunks of one tile (T = 128 columns) each.
@@ -289,38 +332,48 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce_bar(buf)) : "memory");
         }
         pdl_trigger();
-        if (good) {
-            const int64_t orow = (int64_t)it.ra * T + quad * 32 + lane;
-            const int64_t ocol = (int64_t)it.rb * T;
+        // Each epilogue warp stages its 32 rows one column block (32 columns)
+        // at a time and hands each 32 x 32 box to TMA at once, so staging and
+        // storing overlap.  Row r of a box is 128 bytes whose 16-byte chunk c
+        // sits at chunk position c ^ (r & 7) (128-byte swizzle).
+        uint8_t *wbuf = smem + quad * (2 * T / 32) * kBoxBytes;  // this warp's boxes
+        const int y = it.ra * T + quad * 32;
+        const bool store = good && !*(volatile int *)&abort_sh;
 #pragma unroll
-            for (int c0 = 0; c0 < T; c0 += 32) {
-                if (STAGE == 1) {
-                    float4 *hi = (float4 *)(g.out_hi + orow * g.ldo + ocol + c0);
-                    float4 *lo = (float4 *)(g.out_lo + orow * g.ldo + ocol + c0);
+        for (int cb = 0; cb < T / 32; ++cb) {
+            if (store) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
+                for (int c = 0; c < 8; ++c) {
+                    const int col = cb * 32 + 4 * c;
+                    const uint32_t off = (uint32_t)(lane * 128 + ((c ^ (lane & 7)) << 4));
+                    if (STAGE == 1) {
                         float4 h, l;
-                        split_tf32(acc[c0 + 4 * q + 0], h.x, l.x);
-                        split_tf32(acc[c0 + 4 * q + 1], h.y, l.y);
-                        split_tf32(acc[c0 + 4 * q + 2], h.z, l.z);
-                        split_tf32(acc[c0 + 4 * q + 3], h.w, l.w);
-                        hi[q] = h;
-                        lo[q] = l;
+                        split_tf32(acc[col + 0], h.x, l.x);
+                        split_tf32(acc[col + 1], h.y, l.y);
+                        split_tf32(acc[col + 2], h.z, l.z);
+                        split_tf32(acc[col + 3], h.w, l.w);
+                        *(float4 *)(wbuf + (2 * cb) * kBoxBytes + off) = h;
+                        *(float4 *)(wbuf + (2 * cb + 1) * kBoxBytes + off) = l;
+                    } else {
+                        *(float4 *)(wbuf + cb * kBoxBytes + off) =
+                            make_float4(-acc[col + 0], -acc[col + 1], -acc[col + 2], -acc[col + 3]);
                     }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            }
+            __syncwarp();
+            if (store && lane == 0) {
+                const int x = it.rb * T + cb * 32;
+                if (STAGE == 1) {
+                    tma_store_2d(&maps.o0, x, y, smem_u32(wbuf + (2 * cb) * kBoxBytes));
+                    tma_store_2d(&maps.o1, x, y, smem_u32(wbuf + (2 * cb + 1) * kBoxBytes));
                 } else {
-                    float4 *o = (float4 *)(g.out_acc + orow * g.ldo + ocol + c0);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float4 w = o[q];
-                        w.x -= acc[c0 + 4 * q + 0];
-                        w.y -= acc[c0 + 4 * q + 1];
-                        w.z -= acc[c0 + 4 * q + 2];
-                        w.w -= acc[c0 + 4 * q + 3];
-                        o[q] = w;
-                    }
+                    tma_add_2d(&maps.o0, x, y, smem_u32(wbuf + cb * kBoxBytes));
                 }
             }
         }
+        if (store && lane == 0) bulk_commit_and_wait_read();
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
@@ -352,14 +405,15 @@ EncodeTiledFn get_encode()
     return fn;
 }
 
-// rows x cols fp32 row-major matrix with row stride ld (elements); box 32 x 128.
-bool make_map(CUtensorMap *map, const float *base, int64_t rows, int64_t cols, int64_t ld)
+// rows x cols fp32 row-major matrix with row stride ld (elements); boxes of
+// box_rows rows x 32 columns.
+bool make_map(CUtensorMap *map, const float *base, int64_t rows, int64_t cols, int64_t ld, int box_rows = T)
 {
     EncodeTiledFn enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
-    cuuint32_t box[2] = {(cuuint32_t)KB, (cuuint32_t)T};
+    cuuint32_t box[2] = {(cuuint32_t)KB, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, (void *)base, dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -381,8 +435,15 @@ bool make_tc_maps(int stage, int Mt, int Nt, const GemmArgs &g, TcMaps *maps)
     // B = X^T (Np x Mp).  In both, an operand's column count equals its row stride.
     const int64_t Mp = (int64_t)Mt * T, Np = (int64_t)Nt * T;
     const int64_t a_rows = stage == 1 ? Np : Mp, b_rows = stage == 1 ? Mp : Np;
-    return make_map(&maps->a_hi, g.Ahi, a_rows, g.lda, g.lda) && make_map(&maps->a_lo, g.Alo, a_rows, g.lda, g.lda) &&
-           make_map(&maps->b_hi, g.Bhi, b_rows, g.ldb, g.ldb) && make_map(&maps->b_lo, g.Blo, b_rows, g.ldb, g.ldb);
+    // outputs: stage 1 X^T (Np x Mp), stage 2 Wt (Mp x Np); row stride ldo
+    const int64_t o_rows = stage == 1 ? Np : Mp;
+    const bool outs = stage == 1 ? make_map(&maps->o0, g.out_hi, o_rows, g.ldo, g.ldo, 32) &&
+                                       make_map(&maps->o1, g.out_lo, o_rows, g.ldo, g.ldo, 32)
+                                 : make_map(&maps->o0, g.out_acc, o_rows, g.ldo, g.ldo, 32) &&
+                                       make_map(&maps->o1, g.out_acc, o_rows, g.ldo, g.ldo, 32);
+    return outs && make_map(&maps->a_hi, g.Ahi, a_rows, g.lda, g.lda) &&
+           make_map(&maps->a_lo, g.Alo, a_rows, g.lda, g.lda) && make_map(&maps->b_hi, g.Bhi, b_rows, g.ldb, g.ldb) &&
+           make_map(&maps->b_lo, g.Blo, b_rows, g.ldb, g.ldb);
 }
 
 cudaError_t launch_band_tc(int stage, const NodeParams &np, const GemmArgs &g, const TcMaps &maps,

@@ -64,16 +64,35 @@ __host__ __device__ constexpr size_t align_up(size_t x, size_t a = kAlign) { ret
 // TF32 split used by the 3xTF32 band products: x ~= hi + lo with hi = rna_tf32(x)
 // and lo = rna_tf32(x - hi); both have their 13 low mantissa bits clear, so the
 // tensor core consumes them exactly.
+// Round to TF32 (10 explicit mantissa bits), nearest with ties away from zero,
+// the rounding of cvt.rna.tf32.f32: add half a TF32 ulp to the magnitude bits
+// and clear the 13 dropped bits (a carry into the exponent is the correct
+// result).  Two integer instructions instead of a conversion.
 __device__ __forceinline__ float to_tf32(float x)
 {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 __device__ __forceinline__ void split_tf32(float x, float &hi, float &lo)
 {
     hi = to_tf32(x);
     lo = to_tf32(x - hi);
+}
+
+// Correctly rounded fp32 quotient a / b without a divide, from rb = RN(1/b)
+// (Markstein's correction step; P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Develop. 34,
+// 1990): q = RN(a rb) lies within an ulp of a / b, the remainder a - b q is
+// exact as one fused multiply-add, and RN(q + (a - b q) rb) = RN(a / b) when rb
+// is the correctly rounded reciprocal and the operands, the quotient and the
+// remainder are normal numbers.  For steps b in [2^-60, 2^60] (callers route
+// other steps to the IEEE division) the remainder stays normal whenever
+// |a| >= 2^-100, and for smaller |a| the quotient is below 2^-40, so
+// rint(quotient) -- the rounding decision -- is exact for every a.
+__device__ __forceinline__ float div_rn_recip(float a, float b, float rb)
+{
+    const float q = a * rb;
+    const float r = fmaf(-b, q, a);
+    return fmaf(r, rb, q);
 }
 
 // Layout of the solve workspace (all offsets multiples of kAlign).

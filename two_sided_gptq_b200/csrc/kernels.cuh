@@ -44,7 +44,8 @@ cudaError_t launch_band_simt(int stage, const NodeParams &np, const GemmArgs &g,
 // operand parts depend only on the workspace, so they are encoded once per
 // solve.
 struct TcMaps {
-    CUtensorMap a_hi, a_lo, b_hi, b_lo;
+    CUtensorMap a_hi, a_lo, b_hi, b_lo;  // operands, boxes of 128 rows x 32 fp32
+    CUtensorMap o0, o1;                  // outputs: stage 1 X^T hi / lo; stage 2 Wt (o0 only)
 };
 cudaError_t band_tc_configure();
 bool make_tc_maps(int stage, int Mt, int Nt, const GemmArgs &g, TcMaps *maps);

@@ -22,6 +22,8 @@
 //   (1,0) -= S10 LtA[0,0]^T
 //   (1,1) -= (R10 + S10) LtA[1,0]^T + S11 LtA[1,1]^T
 // computed with mma.sync m16n8k8 TF32 in 3xTF32 form (lo*hi + hi*lo + hi*hi).
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -243,13 +245,18 @@ __device__ void apply_product(const float (&acc)[2][4], float *out, int ldo, boo
     }
 }
 
-__device__ void load_scales(const LeafArgs &p, float *scale, float *rcp, int64_t row0, int mr)
+// Steps and their correctly rounded reciprocals; returns true for a thread
+// whose step lies outside [2^-60, 2^60], where the decisions take the IEEE
+// division instead of the reciprocal-based one (div_rn_recip).
+__device__ bool load_scales(const LeafArgs &p, float *scale, float *rcp, int64_t row0, int mr)
 {
     if (threadIdx.x < T) {
         const float s = threadIdx.x < mr ? p.scales[row0 + threadIdx.x] : 1.f;
         scale[threadIdx.x] = s;
         rcp[threadIdx.x] = __frcp_rn(s);
+        return !(s >= 0x1p-60f && s <= 0x1p60f);
     }
+    return false;
 }
 
 // Two-level variant: 2 x 2 sub-tiles of 64.
@@ -487,8 +494,9 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
         const int blk = idx / (S3 * S3), r = (idx / S3) % S3, c = idx % S3;
         sLB[blk * S3 * WS3 + r * WS3 + c] = p.LB32[(row0 + blk * S3 + r) * p.Mp + row0 + blk * S3 + c];
     }
-    load_scales(p, scale, rcp, row0, mr);
-    __syncthreads();
+    // steps outside the range of the reciprocal-based division switch the
+    // whole tile to the IEEE division (a tile-uniform choice)
+    const bool exact_div = __syncthreads_or(load_scales(p, scale, rcp, row0, mr)) != 0;
 
     const float *LAt = p.LA32 + col0 * p.Np + col0;  // LtA diagonal block of the tile (global)
     const float *LBt = p.LB32 + row0 * p.Mp + row0;  // LtB diagonal block of the tile (global)
@@ -558,47 +566,48 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
                     sv = scale[pp * S3 + ac];
                     rv_ = rcp[pp * S3 + ac];
                 };
-                float w0, lb_new, sc_s, sc_r;
-                row_consts(-b, w0, lb_new, sc_s, sc_r);
-                float d_prev = 0.f;
+                auto sweep = [&](auto ieee_tag) {
+                    constexpr bool kIeee = decltype(ieee_tag)::value;
+                    float w0, lb_new, sc_s, sc_r;
+                    row_consts(-b, w0, lb_new, sc_s, sc_r);
+                    float d_prev = 0.f;
 #pragma unroll 2
-                for (int d = 0; d < 2 * S3 - 1; ++d) {
-                    const int a = d - b;
-                    const int ac = min(max(a, 0), S3 - 1);
-                    // the values the previous step produced (the other warps' sums
-                    // leave out the newest row and column terms, added here)
-                    const float ps_in = d > 0 ? ps_buf[(d & 1) * S3 + b] : 0.f;
-                    const float pu_in = d > 0 ? pu_buf[(d & 1) * S3 + b] : 0.f;
-                    const float r_new = b > 0 ? sR[(pp * S3 + ac) * RS3 + tb - 1] : 0.f;
-                    float w0n, lbn_n, sn, rn;
-                    row_consts(a + 1, w0n, lbn_n, sn, rn);
-                    const float sc = fmaf(lb_new, d_prev, ps_in);
-                    const float wt = w0 - fmaf(r_new, la_new, pu_in) - sc;
-                    // clamp(rint(wt / s)) with the IEEE quotient (see decide); the exact
-                    // division runs only when some lane of the warp is near a midpoint
-                    const float qf = wt * sc_r;
-                    float cq = rintf(qf);
-                    const bool near = fabsf(qf - cq) > 0.498f && fabsf(qf) <= 4096.f;
-                    if (__any_sync(0xffffffffu, near)) {
-                        if (near) cq = rintf(__fdiv_rn(wt, sc_s));
+                    for (int d = 0; d < 2 * S3 - 1; ++d) {
+                        const int a = d - b;
+                        const int ac = min(max(a, 0), S3 - 1);
+                        // the values the previous step produced (the other warps' sums
+                        // leave out the newest row and column terms, added here)
+                        const float ps_in = d > 0 ? ps_buf[(d & 1) * S3 + b] : 0.f;
+                        const float pu_in = d > 0 ? pu_buf[(d & 1) * S3 + b] : 0.f;
+                        const float r_new = b > 0 ? sR[(pp * S3 + ac) * RS3 + tb - 1] : 0.f;
+                        float w0n, lbn_n, sn, rn;
+                        row_consts(a + 1, w0n, lbn_n, sn, rn);
+                        const float sc = fmaf(lb_new, d_prev, ps_in);
+                        const float wt = w0 - fmaf(r_new, la_new, pu_in) - sc;
+                        // clamp(rint(wt / s)) with the correctly rounded fp32 quotient
+                        const float qf = kIeee ? __fdiv_rn(wt, sc_s) : div_rn_recip(wt, sc_s, sc_r);
+                        const float cq = fminf(fmaxf(rintf(qf), fqmin), fqmax);
+                        const int ta = pp * S3 + a;
+                        const bool valid = a >= 0 && a < S3 && ta < mr && tb < nc;
+                        const float dl = valid ? fmaf(-sc_s, cq, wt) : 0.f;
+                        // invalid lanes write to spare slots instead of branching
+                        const int iR = valid ? ta * RS3 + tb : T * RS3 + lane;
+                        const int iD = valid ? tb * RS3 + ta : T * RS3 + lane;
+                        const int iC = valid ? ta * T + tb : T * T + lane;
+                        const int iW = valid ? a * WS3 + b : ac * WS3 + S3 + (lane & 3);  // row padding
+                        sR[iR] = sc + dl;
+                        sDt[iD] = dl;
+                        sCode[iC] = code_byte(cq);
+                        Wp[iW] = wt;  // pre-rounding value, copied out when requested
+                        d_prev = dl;
+                        w0 = w0n; lb_new = lbn_n; sc_s = sn; sc_r = rn;
+                        group_sync(bar_id, 96);
                     }
-                    cq = fminf(fmaxf(cq, fqmin), fqmax);
-                    const int ta = pp * S3 + a;
-                    const bool valid = a >= 0 && a < S3 && ta < mr && tb < nc;
-                    const float dl = valid ? fmaf(-sc_s, cq, wt) : 0.f;
-                    // invalid lanes write to the spare row / bytes instead of branching
-                    const int iR = valid ? ta * RS3 + tb : T * RS3 + lane;
-                    const int iD = valid ? tb * RS3 + ta : T * RS3 + lane;
-                    const int iC = valid ? ta * T + tb : T * T + lane;
-                    const int iW = valid ? a * WS3 + b : ac * WS3 + S3 + (lane & 3);  // spare: row padding
-                    sR[iR] = sc + dl;
-                    sDt[iD] = dl;
-                    sCode[iC] = code_byte(cq);
-                    Wp[iW] = wt;  // pre-rounding value, copied out when requested
-                    d_prev = dl;
-                    w0 = w0n; lb_new = lbn_n; sc_s = sn; sc_r = rn;
-                    group_sync(bar_id, 96);
-                }
+                };
+                if (exact_div)
+                    sweep(std::true_type{});
+                else
+                    sweep(std::false_type{});
             } else if (role == 1) {
                 // ---- row-side warp (lane = column b): sum_{c <= b-2} R[a+1][c] LtA[b][c]
                 // for the entry warp's next entry (a+1, b).  Column b-1 of that R
