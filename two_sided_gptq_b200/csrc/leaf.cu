@@ -384,29 +384,35 @@ __global__ void __launch_bounds__(kThreads, 1) leaf_single_kernel(LeafArgs p, in
 }
 
 // ------------------------------------------------------------------------
-// Warp-pair-per-sub-tile variant: 4 x 4 sub-tiles of 32, processed in
-// sub-tile diagonal order e = 0..6.  Before phase e, the cross-sub-tile terms
-// of every sub-tile (p, q) with p + q = e are applied left-looking with all 8
-// warps:
-//     S[p,q] = sum_{p'<p} LtB[p,p'] D[p',q],
-//     Wt[p,q] -= sum_{q'<q} R[p,q'] LtA[q,q']^T + S[p,q] LtA[q,q]^T,
-// where R[p,q'] = sum_{p'<=p} LtB[p,p'] D[p',q'] is complete for q' < q.  Then
-// warps 2p and 2p+1 sweep sub-tile (p, q) (63 entry anti-diagonal steps, one
-// pair barrier each) and finally R[p,q] = S[p,q] + (the sweep's in-sub-tile R).
-// In the sweep, entry (a, b) needs
-//     Wt_ab = W0_ab - sum_{c<b} R_ac LtA[b,c] - sum_{r<a} LtB[a,r] D_rb:
-// warp A (lane = column b) rounds the entries and keeps the row-side sum,
-// whose operands are its own LtA row (registers) and rows of R (smem); warp B
-// (lane = row rho) keeps the column-side sum, whose operands are its own LtB
-// row (registers) and columns of D (smem).  Both sums are formed a step ahead
-// without their newest term, which warp A adds from the values the previous
-// step produced.  sR and sDt start at zero.
+// Warp variant (the default): 4 x 4 sub-tiles of 32, processed in sub-tile
+// diagonal order e = 0..6, three warps per row block of sub-tiles.  Phase e,
+// for every sub-tile (p, q) with p + q = e:
+//     S[p,q]  = sum_{p'<p} LtB[p,p'] D[p',q]              (written into R[p,q]),
+//     W0[p,q] = Wt[p,q] - sum_{q'<q} R[p,q'] LtA[q,q']^T - S[p,q],
+// where R[p,q'] = sum_{p'<=p} LtB[p,p'] D[p',q'] is complete for q' < q; then
+// the three warps of row block p sweep the sub-tile (63 entry anti-diagonal
+// steps, one 96-thread barrier each).  Entry (a, b) of the sub-tile needs
+//     Wt_ab = W0_ab - sum_{c<b} R_ac LtA[b,c] - sum_{r<a} LtB[a,r] D_rb,
+// with R holding S plus the sub-tile's own terms, so the S terms of the
+// row-side sum come in through R:
+//   * the entry warp (lane = column b) rounds the entries and writes
+//     R_ab = S_ab + sum_{r<=a} LtB[a,r] D_rb;
+//   * the row-side warp (lane = column b) forms sum_{c<=b-2} R_ac LtA[b,c]
+//     from its LtA row (registers) and rows of R (smem);
+//   * the column-side warp (lane = row rho) forms sum_{r<=rho-2} LtB[rho,r] D_rb
+//     from its LtB row (registers) and columns of D (smem);
+// both sums a step ahead without their newest term, which the entry warp adds
+// from the values the previous step produced.  The Wt blocks and LtA strips of
+// the next phase are staged into shared memory by asynchronous copies while the
+// current phase sweeps.  sR and sDt start at zero.
 namespace {
 constexpr int S3 = 32;             // sub-tile side
 constexpr int RS3 = T + 4;         // row stride of sR / sDt: 33 float4 per row
 constexpr int WS3 = S3 + 4;        // row stride of the per-row-block slots
+constexpr int kLAStage = S3 * (3 * S3 * 2 + 4 * 3);  // largest phase: strips for q = 3, 2, 1
 constexpr size_t kSmemWarp =
-    ((size_t)2 * (T + 1) * RS3 + 3 * 4 * S3 * WS3 + 2 * T + 2 * 4 * 2 * S3) * sizeof(float) + (size_t)T * T + 32;
+    ((size_t)2 * (T + 1) * RS3 + 2 * 4 * S3 * WS3 + kLAStage + 4 * S3 + 2 * T + 2 * 4 * 2 * S3) * sizeof(float) +
+    (size_t)T * T + 32;
 static_assert(kSmemWarp <= 232448, "leaf shared memory");
 }  // namespace
 
@@ -457,15 +463,23 @@ __device__ __forceinline__ int8_t code_byte(float c)
     return (int8_t)(__float_as_int(c + 12582912.0f) & 0xFF);
 }
 
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+
 __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int K, int I_lo)
 {
     extern __shared__ __align__(16) float smem_f[];
-    float *sR = smem_f;                  // T x RS3 (+1 spare row): R, 0 where not rounded yet
+    float *sR = smem_f;                  // T x RS3 (+1 spare row): R, S before the sweep, 0 before that
     float *sDt = sR + (T + 1) * RS3;     // T x RS3 (+1 spare row): D transposed, 0 where not rounded yet
     float *sW = sDt + (T + 1) * RS3;     // 4 slots of S3 x WS3: W0 of the sub-tile being swept, then Wt
-    float *sS = sW + 4 * S3 * WS3;       // 4 slots: S[p,q]
-    float *sLB = sS + 4 * S3 * WS3;      // 4 slots: LtB[p,p]
-    float *scale = sLB + 4 * S3 * WS3;   // T
+    float *sWt = sW + 4 * S3 * WS3;      // 4 slots: Wt of the next sub-tile (staged during the sweep)
+    float *sLA = sWt + 4 * S3 * WS3;     // LtA[q, 0:q] strips of the next phase (staged during the sweep)
+    float *sLBd = sLA + kLAStage;        // 4 x S3: LtB sub-diagonal LtB[r][r-1] per row block
+    float *scale = sLBd + 4 * S3;        // T
     float *rcp = scale + T;              // T
     float *sPS = rcp + T;                // 4 x 2 x S3: column-side partial sums by column
     float *sPU = sPS + 4 * 2 * S3;       // 4 x 2 x S3: row-side partial sums by column
@@ -475,101 +489,160 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
     const int64_t row0 = (int64_t)I * T, col0 = (int64_t)J * T;
     const int mr = (int)min64(T, p.m - row0), nc = (int)min64(T, p.n - col0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float *LAt = p.LA32 + col0 * p.Np + col0;  // LtA diagonal block of the tile (global)
+    const float *LBt = p.LB32 + row0 * p.Mp + row0;  // LtB diagonal block of the tile (global)
+    const int lda_g = (int)p.Np, ldb_g = (int)p.Mp;
     // Warm L2 with the tile's two factor diagonal blocks (read by the products
     // and the sweeps; each leaf launch uses blocks no earlier launch touched).
     // A prefetch is only a hint, so it may run before the dependency wait.
     for (int idx = tid; idx < 2 * T * (T / 32); idx += kThreadsW) {
         const int which = idx / (T * (T / 32)), r = (idx / (T / 32)) % T, seg = idx % (T / 32);
-        const float *ptr = which == 0 ? p.LA32 + (col0 + r) * p.Np + col0 + 32 * seg
-                                      : p.LB32 + (row0 + r) * p.Mp + row0 + 32 * seg;
+        const float *ptr = which == 0 ? LAt + r * lda_g + 32 * seg : LBt + r * ldb_g + 32 * seg;
         asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
     }
     pdl_wait();  // every global input (Wt, factors, steps) comes from earlier kernels
+
+    // Stage, for the sub-tiles (p, q = e - p) of phase e, the tile's Wt block and
+    // the strip LtA[q, 0:q] (32 rows x 32 q columns, row stride 32 q + 4), strips
+    // laid out back to back in row-block order.  Every thread issues a share of
+    // 16-byte asynchronous copies and commits them as one group.
+    auto stage_phase = [&](int e) {
+        if (e > 6) return;
+        int off = 0;
+        for (int pp = max(0, e - 3); pp <= min(3, e); ++pp) {
+            const int q = e - pp;
+            if (q > 0) {
+                const int ld = S3 * q + 4, c4 = 8 * q;
+                for (int c = tid; c < S3 * c4; c += kThreadsW) {
+                    const int j = c / c4, k4 = c - j * c4;
+                    cp_async16(sLA + off + j * ld + 4 * k4, LAt + (q * S3 + j) * lda_g + 4 * k4);
+                }
+                off += S3 * ld;
+            }
+            for (int c = tid; c < S3 * 8; c += kThreadsW) {
+                const int i = c >> 3, k4 = c & 7;
+                cp_async16(sWt + pp * S3 * WS3 + i * WS3 + 4 * k4,
+                           p.Wt + (row0 + pp * S3 + i) * p.Np + col0 + q * S3 + 4 * k4);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // offset of row block pp's strip in phase e
+    auto la_offset = [](int e, int pp) {
+        int off = 0;
+        for (int p2 = max(0, e - 3); p2 < pp; ++p2)
+            if (e - p2 > 0) off += S3 * (S3 * (e - p2) + 4);
+        return off;
+    };
+    stage_phase(0);
 
     for (int idx = tid; idx < (T + 1) * RS3 / 4; idx += kThreadsW) {
         ((float4 *)sR)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
         ((float4 *)sDt)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int idx = tid; idx < 4 * S3 * S3; idx += kThreadsW) {  // LtB diagonal sub-blocks (prep output)
-        const int blk = idx / (S3 * S3), r = (idx / S3) % S3, c = idx % S3;
-        sLB[blk * S3 * WS3 + r * WS3 + c] = p.LB32[(row0 + blk * S3 + r) * p.Mp + row0 + blk * S3 + c];
+    if (tid < T) {
+        const int blk = tid / S3, r = tid % S3;
+        sLBd[tid] = r > 0 ? LBt[(blk * S3 + r) * ldb_g + blk * S3 + r - 1] : 0.f;
+    }
+    const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
+    const int wp = warp / 3, role = warp - 3 * wp;  // row block of sub-tiles; 0 entries, 1 row side, 2 column side
+    const int i0 = (role & 1) * 16, j0 = 0;         // products: roles 0 and 1 take a 16 x 32 half each
+    // column-side warp: its LtB[p,p] row rho (columns <= rho-2), fixed for the kernel
+    float2 lbr[S3 / 2];
+    if (role == 2) {
+#pragma unroll
+        for (int c = 0; c < S3 / 2; ++c) {
+            float2 v = *(const float2 *)(LBt + (wp * S3 + lane) * ldb_g + wp * S3 + 2 * c);
+            v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
+            v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
+            lbr[c] = v;
+        }
     }
     // steps outside the range of the reciprocal-based division switch the
     // whole tile to the IEEE division (a tile-uniform choice)
     const bool exact_div = __syncthreads_or(load_scales(p, scale, rcp, row0, mr)) != 0;
 
-    const float *LAt = p.LA32 + col0 * p.Np + col0;  // LtA diagonal block of the tile (global)
-    const float *LBt = p.LB32 + row0 * p.Mp + row0;  // LtB diagonal block of the tile (global)
-    const int lda_g = (int)p.Np, ldb_g = (int)p.Mp;
-    const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
-    const int wp = warp / 3, role = warp - 3 * wp;  // row block of sub-tiles; 0 entries, 1 row side, 2 column side
-    const int i0 = (role & 1) * 16, j0 = 0;         // products: roles 0 and 1 take a 16 x 32 half each
-
     for (int e = 0; e < 7; ++e) {
         const int p_lo = max(0, e - 3), p_hi = min(3, e);
         const bool mine = wp >= p_lo && wp <= p_hi;  // this warp's row block has a sub-tile in phase e
         const int qv = e - wp;
-        // S[p,q] = LtB[p, 0:p] D[0:p, q]
-        if (mine && role < 2) {
+        // S[p,q] = LtB[p, 0:p] D[0:p, q], written into R's (p,q) block (zero so far)
+        if (mine && role < 2 && wp > 0) {
             float acc[4][4] = {};
-            if (wp > 0)
-                mma_block<4>(acc, LBt + (wp * S3) * ldb_g, ldb_g, sDt + (qv * S3) * RS3, RS3, wp * S3, i0, j0);
+            mma_block<4>(acc, LBt + (wp * S3) * ldb_g, ldb_g, sDt + (qv * S3) * RS3, RS3, wp * S3, i0, j0);
             const int g = lane >> 2, t = lane & 3;
-            float *o = sS + wp * S3 * WS3;
+            float *o = sR + (wp * S3) * RS3 + qv * S3;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const int j = j0 + nt * 8 + 2 * t;
-                o[(i0 + g) * WS3 + j] = acc[nt][0];
-                o[(i0 + g) * WS3 + j + 1] = acc[nt][1];
-                o[(i0 + g + 8) * WS3 + j] = acc[nt][2];
-                o[(i0 + g + 8) * WS3 + j + 1] = acc[nt][3];
+                o[(i0 + g) * RS3 + j] = acc[nt][0];
+                o[(i0 + g) * RS3 + j + 1] = acc[nt][1];
+                o[(i0 + g + 8) * RS3 + j] = acc[nt][2];
+                o[(i0 + g + 8) * RS3 + j + 1] = acc[nt][3];
             }
         }
+        // row-side warp: LtA[q,q] row b (columns <= b-2); entry warp: LtA[b][b-1]
+        float2 la[S3 / 2];
+        float la_new = 0.f;
+        if (mine && role == 1) {
+#pragma unroll
+            for (int c = 0; c < S3 / 2; ++c) {
+                float2 v = *(const float2 *)(LAt + (qv * S3 + lane) * lda_g + qv * S3 + 2 * c);
+                v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
+                v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
+                la[c] = v;
+            }
+        }
+        if (mine && role == 0 && lane > 0) la_new = LAt[(qv * S3 + lane) * lda_g + qv * S3 + lane - 1];
+        asm volatile("cp.async.wait_all;" ::: "memory");  // this phase's staged Wt and LtA strips
         __syncthreads();
-        // W0[p,q] = Wt_global - (R[p, 0:q] LtA[q, 0:q]^T + S[p,q] LtA[q,q]^T)
+        // W0[p,q] = Wt[p,q] - R[p, 0:q] LtA[q, 0:q]^T - S[p,q]; the sweep adds the
+        // S terms of the row-side sums through R (R[p,q] starts as S[p,q])
         if (mine && role < 2) {
             float acc[4][4] = {};
-            const float *LAq = LAt + (qv * S3) * lda_g;
-            if (qv > 0) mma_block<4>(acc, sR + (wp * S3) * RS3, RS3, LAq, lda_g, qv * S3, i0, j0);
-            mma_block<4>(acc, sS + wp * S3 * WS3, WS3, LAq + qv * S3, lda_g, S3, i0, j0);
+            if (qv > 0)
+                mma_block<4>(acc, sR + (wp * S3) * RS3, RS3, sLA + la_offset(e, wp), S3 * qv + 4, qv * S3, i0, j0);
             const int g = lane >> 2, t = lane & 3;
             float *o = sW + wp * S3 * WS3;
-            const float *wg = p.Wt + (row0 + wp * S3) * p.Np + col0 + qv * S3;
+            const float *wt = sWt + wp * S3 * WS3;
+            const float *sq = sR + (wp * S3) * RS3 + qv * S3;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const int j = j0 + nt * 8 + 2 * t;
-                o[(i0 + g) * WS3 + j] = wg[(i0 + g) * p.Np + j] - acc[nt][0];
-                o[(i0 + g) * WS3 + j + 1] = wg[(i0 + g) * p.Np + j + 1] - acc[nt][1];
-                o[(i0 + g + 8) * WS3 + j] = wg[(i0 + g + 8) * p.Np + j] - acc[nt][2];
-                o[(i0 + g + 8) * WS3 + j + 1] = wg[(i0 + g + 8) * p.Np + j + 1] - acc[nt][3];
+                o[(i0 + g) * WS3 + j] = wt[(i0 + g) * WS3 + j] - acc[nt][0] - sq[(i0 + g) * RS3 + j];
+                o[(i0 + g) * WS3 + j + 1] = wt[(i0 + g) * WS3 + j + 1] - acc[nt][1] - sq[(i0 + g) * RS3 + j + 1];
+                o[(i0 + g + 8) * WS3 + j] = wt[(i0 + g + 8) * WS3 + j] - acc[nt][2] - sq[(i0 + g + 8) * RS3 + j];
+                o[(i0 + g + 8) * WS3 + j + 1] =
+                    wt[(i0 + g + 8) * WS3 + j + 1] - acc[nt][3] - sq[(i0 + g + 8) * RS3 + j + 1];
             }
         }
         __syncthreads();
+        stage_phase(e + 1);  // lands while this phase sweeps
         // sweep: warps 3p, 3p+1, 3p+2 take sub-tile (p, e - p) together, one
         // barrier of the three per entry anti-diagonal step
         if (mine) {
-            const int pp = wp, q = e - pp;
-            const float *LBp = sLB + pp * S3 * WS3;
+            const int pp = wp, q = qv;
             float *ps_buf = sPS + pp * 2 * S3;  // [2][S3]: column-side sums, by column
             float *pu_buf = sPU + pp * 2 * S3;  // [2][S3]: row-side sums, by column
             float *Wp = sW + pp * S3 * WS3;
+            const float *LBd = sLBd + pp * S3;
             const int bar_id = 1 + pp;
             if (role == 0) {
                 // ---- entry warp (lane = column b): rounds entry (d - b, b) at step d
                 const int b = lane, tb = q * S3 + b;
-                const float la_new = b > 0 ? LAt[(q * S3 + b) * lda_g + q * S3 + b - 1] : 0.f;
-                // row-dependent constants of an entry, loaded a step before it is rounded
-                auto row_consts = [&](int a, float &w0, float &lbn, float &sv, float &rv_) {
+                // row-dependent values of an entry, loaded a step before it is rounded
+                auto row_consts = [&](int a, float &w0, float &lbn, float &sv, float &rv_, float &s0) {
                     const int ac = min(max(a, 0), S3 - 1);
                     w0 = Wp[ac * WS3 + b];
-                    lbn = ac > 0 ? LBp[ac * WS3 + ac - 1] : 0.f;
+                    lbn = LBd[ac];
                     sv = scale[pp * S3 + ac];
                     rv_ = rcp[pp * S3 + ac];
+                    s0 = sR[(pp * S3 + ac) * RS3 + tb];  // S[a][b] until this entry overwrites it
                 };
                 auto sweep = [&](auto ieee_tag) {
                     constexpr bool kIeee = decltype(ieee_tag)::value;
-                    float w0, lb_new, sc_s, sc_r;
-                    row_consts(-b, w0, lb_new, sc_s, sc_r);
+                    float w0, lb_new, sc_s, sc_r, s_ab;
+                    row_consts(-b, w0, lb_new, sc_s, sc_r, s_ab);
                     float d_prev = 0.f;
 #pragma unroll 2
                     for (int d = 0; d < 2 * S3 - 1; ++d) {
@@ -580,8 +653,8 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
                         const float ps_in = d > 0 ? ps_buf[(d & 1) * S3 + b] : 0.f;
                         const float pu_in = d > 0 ? pu_buf[(d & 1) * S3 + b] : 0.f;
                         const float r_new = b > 0 ? sR[(pp * S3 + ac) * RS3 + tb - 1] : 0.f;
-                        float w0n, lbn_n, sn, rn;
-                        row_consts(a + 1, w0n, lbn_n, sn, rn);
+                        float w0n, lbn_n, sn, rn, s_n;
+                        row_consts(a + 1, w0n, lbn_n, sn, rn, s_n);
                         const float sc = fmaf(lb_new, d_prev, ps_in);
                         const float wt = w0 - fmaf(r_new, la_new, pu_in) - sc;
                         // clamp(rint(wt / s)) with the correctly rounded fp32 quotient
@@ -595,12 +668,12 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
                         const int iD = valid ? tb * RS3 + ta : T * RS3 + lane;
                         const int iC = valid ? ta * T + tb : T * T + lane;
                         const int iW = valid ? a * WS3 + b : ac * WS3 + S3 + (lane & 3);  // row padding
-                        sR[iR] = sc + dl;
+                        sR[iR] = s_ab + sc + dl;
                         sDt[iD] = dl;
                         sCode[iC] = code_byte(cq);
                         Wp[iW] = wt;  // pre-rounding value, copied out when requested
                         d_prev = dl;
-                        w0 = w0n; lb_new = lbn_n; sc_s = sn; sc_r = rn;
+                        w0 = w0n; lb_new = lbn_n; sc_s = sn; sc_r = rn; s_ab = s_n;
                         group_sync(bar_id, 96);
                     }
                 };
@@ -613,14 +686,6 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
                 // for the entry warp's next entry (a+1, b).  Column b-1 of that R
                 // row is written during this step; its coefficient here is zero.
                 const int b = lane;
-                float2 la[S3 / 2];
-#pragma unroll
-                for (int c = 0; c < S3 / 2; ++c) {
-                    float2 v = *(const float2 *)(LAt + (q * S3 + b) * lda_g + q * S3 + 2 * c);
-                    v.x = 2 * c + 0 <= b - 2 ? v.x : 0.f;
-                    v.y = 2 * c + 1 <= b - 2 ? v.y : 0.f;
-                    la[c] = v;
-                }
                 float4 rv[S3 / 4];  // chunks this lane never loads stay zero
 #pragma unroll
                 for (int c = 0; c < S3 / 4; ++c) rv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -649,14 +714,6 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
                 // rho-1 of that D column is written during this step; its
                 // coefficient here is zero.
                 const int rho = lane;
-                float2 lbr[S3 / 2];
-#pragma unroll
-                for (int c = 0; c < S3 / 2; ++c) {
-                    float2 v = *(const float2 *)(LBp + rho * WS3 + 2 * c);
-                    v.x = 2 * c + 0 <= rho - 2 ? v.x : 0.f;
-                    v.y = 2 * c + 1 <= rho - 2 ? v.y : 0.f;
-                    lbr[c] = v;
-                }
                 float4 dv[S3 / 4];
 #pragma unroll
                 for (int c = 0; c < S3 / 4; ++c) dv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -684,15 +741,13 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
             }
         }
         __syncthreads();
-        // R[p,q] = S[p,q] + in-sub-tile R; the pre-rounding values when requested
-        for (int idx = tid; idx < (p_hi - p_lo + 1) * S3 * S3; idx += kThreadsW) {
-            const int pp = p_lo + idx / (S3 * S3), r = (idx / S3) % S3, c = idx % S3;
-            sR[(pp * S3 + r) * RS3 + (e - pp) * S3 + c] += sS[pp * S3 * WS3 + r * WS3 + c];
-            const int ta = pp * S3 + r, tb = (e - pp) * S3 + c;
-            if (p.wt_out && ta < mr && tb < nc)
-                p.wt_out[(row0 + ta) * p.n + col0 + tb] = sW[pp * S3 * WS3 + r * WS3 + c];
+        if (p.wt_out) {  // the pre-rounding values of this phase's sub-tiles
+            for (int idx = tid; idx < (p_hi - p_lo + 1) * S3 * S3; idx += kThreadsW) {
+                const int pp = p_lo + idx / (S3 * S3), r = (idx / S3) % S3, c = idx % S3;
+                const int ta = pp * S3 + r, tb = (e - pp) * S3 + c;
+                if (ta < mr && tb < nc) p.wt_out[(row0 + ta) * p.n + col0 + tb] = sW[pp * S3 * WS3 + r * WS3 + c];
+            }
         }
-        __syncthreads();
     }
     pdl_trigger();
     for (int idx = tid; idx < T * T; idx += kThreadsW) {  // V = s * code, residual split
