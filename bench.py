@@ -31,8 +31,23 @@ METRIC = "quantized weights/sec for 4096×4096 INT4 BaKron solve; % tensor-pipe 
 TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 : BF16 tensor peak ratio
 FALLBACK_BF16_TFLOPS = 1590.0
 LEAF_BYTES_PER_WEIGHT = 25  # read Wt 4 + diagonal factor blocks 8; write code 1, V 4, D hi/lo 8
-LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 255), 3: ("leaf_warp_kernel", 7 * 63)}
-DEFAULT_LEAF = 3  # the library's default leaf structure
+LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 255), 3: ("leaf_warp_kernel", 7 * 63),
+                4: ("leaf_wide_kernel", 3 * 127)}
+# DRAM traffic of the band products from an ncu capture of one solve's 124
+# band launches (profiles/band_tc_4096_dram.md); reported only while the
+# kernel sources hash to the value the capture was taken with.
+BAND_TRAFFIC = {"sources_sha256": None, "bytes_per_launch": None, "profile": "profiles/band_tc_4096_dram.md"}
+BAND_SOURCES = ("two_sided_gptq_b200/csrc/band_tc.cu", "two_sided_gptq_b200/csrc/common.cuh",
+                "two_sided_gptq_b200/csrc/kernels.cuh")
+
+
+def band_sources_sha256():
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in BAND_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()
 
 
 def peaks():
@@ -296,8 +311,11 @@ def main():
     out = (V, codes, scales)
     stream = torch.cuda.current_stream()
 
+    # the schedule's leaf structure, picked by measurement on this problem
+    leaf, leaf_tune_ms = bk.tune_leaf(Wd, LA, LB, bits=w.bits, ws=ws, out=out, stream=stream)
+
     def step():
-        bk.solve(Wd, LA, LB, bits=w.bits, ws=ws, out=out, check_status=False, stream=stream)
+        bk.solve(Wd, LA, LB, bits=w.bits, ws=ws, out=out, check_status=False, stream=stream, leaf=leaf)
 
     for _ in range(args.warmup):
         step()
@@ -325,7 +343,8 @@ def main():
     # per-kernel-class device times (separate profiled steps, events on the launch stream)
     prof, launches = [], []
     for _ in range(max(1, args.profile_steps)):
-        bk.solve(Wd, LA, LB, bits=w.bits, ws=ws, out=out, check_status=False, stream=stream, profile=True)
+        bk.solve(Wd, LA, LB, bits=w.bits, ws=ws, out=out, check_status=False, stream=stream, profile=True,
+                 leaf=leaf)
         prof.append(bk.last_profile())
         launches.append(bk.last_profile_launches())
     pr = {k: statistics.median(p[k] for p in prof) for k in prof[0]}
@@ -334,7 +353,8 @@ def main():
     bf16, hbm, src = peaks()
     tf32_peak = bf16 * TF32_PER_BF16
     gemm_ms = pr["stage1_ms"] + pr["stage2_ms"]
-    achieved = 3.0 * plan["update_flops"] / (gemm_ms / 1e3) / 1e12
+    # a one-tile-diagonal problem (m, n <= 128) has no band products
+    achieved = 3.0 * plan["update_flops"] / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
     leaf_bytes = LEAF_BYTES_PER_WEIGHT * m * n
     launches_per_step = 4 + int(plan["leaves"]) + 2 * int(plan["nodes"])
 
@@ -347,13 +367,14 @@ def main():
     sh = torch.empty((m,), dtype=torch.float32).pin_memory()
     wsh = bk.workspace(bk.solve_host_workspace_size(m, n), dev)
     for _ in range(2):
-        bk.solve_host(Wh, LAh, LBh, bits=w.bits, V=Vh, codes=ch, scales=sh, ws=wsh, stream=stream)
+        bk.solve_host(Wh, LAh, LBh, bits=w.bits, V=Vh, codes=ch, scales=sh, ws=wsh, stream=stream, leaf=leaf)
     torch.cuda.synchronize()
     h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_steps = max(3, args.steps // 2)
     h0.record(stream)
     for _ in range(e2e_steps):
-        bk.solve_host(Wh, LAh, LBh, bits=w.bits, V=Vh, codes=ch, scales=sh, ws=wsh, stream=stream, synchronize=False)
+        bk.solve_host(Wh, LAh, LBh, bits=w.bits, V=Vh, codes=ch, scales=sh, ws=wsh, stream=stream, synchronize=False,
+                      leaf=leaf)
     h1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(h0.elapsed_time(h1) / e2e_steps, dist, dev)
@@ -371,18 +392,21 @@ def main():
             "roofline": {
                 "bound": "tensor", "kernel": "band_tc_kernel (stage 1 + stage 2 band products)",
                 "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s", "frac": achieved / tf32_peak,
-                "traffic": None,
+                "traffic": (BAND_TRAFFIC["bytes_per_launch"]
+                            if BAND_TRAFFIC["sources_sha256"] == band_sources_sha256() else None),
+                "traffic_source": BAND_TRAFFIC["profile"],
                 "peak_source": f"{src} bf16 {bf16:.1f} TFLOP/s x {TF32_PER_BF16:.4f} (nominal TF32:BF16), burst",
                 "flops_per_step": 3.0 * plan["update_flops"],
                 "flops_note": "3 TF32 MMAs per multiply-add (3xTF32) x algorithmic tile-product FLOPs of the schedule",
                 "band_ms_per_step": gemm_ms},
             "band_levels": levels,
-            "leaf": {"kernel": LEAF_KERNELS[DEFAULT_LEAF][0], "ms_per_step": pr["leaf_ms"],
+            "leaf": {"kernel": LEAF_KERNELS[leaf][0], "structure": leaf, "tune_ms": dict(zip((1, 2, 3, 4), leaf_tune_ms)),
+                     "ms_per_step": pr["leaf_ms"],
                      "launches_per_step": pr["leaf_launches"],
                      "achieved_gbs": leaf_bytes / (pr["leaf_ms"] / 1e3) / 1e9, "hbm_peak_gbs": hbm,
                      "bytes_per_step": leaf_bytes, "bound": "latency (dependent rounding steps)",
-                     "sequential_steps_per_leaf": LEAF_KERNELS[DEFAULT_LEAF][1],
-                     "ns_per_sequential_step": pr["leaf_ms"] * 1e6 / (pr["leaf_launches"] * LEAF_KERNELS[DEFAULT_LEAF][1]),
+                     "sequential_steps_per_leaf": LEAF_KERNELS[leaf][1],
+                     "ns_per_sequential_step": pr["leaf_ms"] * 1e6 / (pr["leaf_launches"] * LEAF_KERNELS[leaf][1]),
                      "share_of_profiled_step": pr["leaf_ms"] / pr["total_ms"]},
             "profile_ms": pr,
             "factor_ms": factor_ms,

@@ -93,7 +93,9 @@ typedef struct {
     int32_t leaf;     /* leaf sweep structure: 0 = default (3); 1 = each tile as
                          2 x 2 sub-tiles of 64 swept by the whole CTA; 2 = one
                          anti-diagonal sweep over the whole 128 x 128 tile; 3 =
-                         4 x 4 sub-tiles of 32, each swept by one warp. */
+                         4 x 4 sub-tiles of 32, each swept by three warps; 4 =
+                         2 x 2 sub-tiles of 64, each swept by six warps
+                         (bakron_tune_leaf picks one by measurement). */
 } bakron_config_t;
 
 /* Per-kernel-class device time of the latest profiled bakron_solve on the
@@ -155,6 +157,22 @@ bakron_status_t bakron_solve(const float *W_dev, int64_t m, int64_t n, const flo
                              const float *LB_dev, const bakron_quantizer_t *q, float *V_dev,
                              int8_t *codes_dev, float *scales_dev, void *ws_dev, size_t ws_bytes,
                              const bakron_config_t *cfg, bakron_stream_t stream);
+
+/* Leaf structure picked by measurement (the schedule's leaf size: 4 x 4
+ * sub-tiles of 32, 2 x 2 of 64, or the whole 128 x 128 tile per sweep).  Runs
+ * bakron_solve on the caller's problem once per structure after one warm-up
+ * solve, timing each with CUDA events on `stream` (the call synchronises
+ * `stream`), and writes the fastest structure (a bakron_config_t.leaf value,
+ * 1..4) to *leaf_out and the four times in ms to ms_out[0..3] (leaf 1..4;
+ * ms_out may be NULL).  Arguments as for bakron_solve; cfg->leaf is ignored
+ * and cfg->profile must be 0.  V, codes and scales hold the last solve's
+ * results (all structures give the same codes up to rounding ties).  Device
+ * errors are read with bakron_get_status as after bakron_solve. */
+bakron_status_t bakron_tune_leaf(const float *W_dev, int64_t m, int64_t n, const float *LA_dev,
+                                 const float *LB_dev, const bakron_quantizer_t *q, float *V_dev,
+                                 int8_t *codes_dev, float *scales_dev, void *ws_dev, size_t ws_bytes,
+                                 const bakron_config_t *cfg, bakron_stream_t stream, int32_t *leaf_out,
+                                 double *ms_out);
 
 /* Bytes of device workspace bakron_solve_host needs (solve workspace plus
  * device staging for W, LA, LB, V, codes and scales). */

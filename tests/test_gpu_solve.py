@@ -110,7 +110,7 @@ def test_leaf_variants(case):
         W, A, B = workloads.random_problem(m, n, seed=m + 7 * n)
         LA, LB = oracle_factors(A, B)
         label = f"{m}x{n}"
-    for leaf in (1, 2, 3):
+    for leaf in (1, 2, 3, 4):
         check_solve(W, LA, LB, 4, leaf=leaf, label=f"{label}/leaf{leaf}")
 
 
@@ -130,3 +130,18 @@ def test_full_size_workloads(name):
     check_solve(W, LA, LB, workloads.WORKLOADS[name].bits, label=name)
     if name != "large2":
         _cache.pop("large" if name == "large4" else name, None)
+
+
+def test_tune_leaf_picks_a_measured_structure():
+    """bakron_tune_leaf times every leaf structure on the problem and returns
+    the fastest; its outputs meet the parity contract."""
+    import torch
+
+    import two_sided_gptq_b200 as bk
+
+    W, A, B, LA, LB = named("mid")
+    Wd, LAd, LBd = (torch.from_numpy(x).cuda() for x in (W, LA.astype(np.float32), LB.astype(np.float32)))
+    leaf, ms = bk.tune_leaf(Wd, LAd, LBd, bits=4)
+    assert leaf in (1, 2, 3, 4) and all(t > 0 for t in ms)
+    assert ms[leaf - 1] == min(ms)
+    check_solve(W, LA, LB, 4, leaf=leaf, label=f"mid/tuned-leaf{leaf}")

@@ -18,7 +18,7 @@ import ctypes
 from . import _native
 from ._native import BakronError, Config, PlanStats, Profile, ProfileLaunch, Quantizer, Status, check
 
-__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile", "last_profile_launches",
+__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile", "last_profile_launches", "tune_leaf",
            "workspace", "get_status",
            "BakronError", "Status", "version", "library_path"]
 
@@ -107,7 +107,9 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
 
     ``gemm=0`` uses the tcgen05 3xTF32 band products, ``gemm=1`` the FP32
     CUDA-core ones; ``leaf`` selects the leaf sweep structure (0 default,
-    1 two-level CTA-wide, 2 single-level, 3 warp per 32 x 32 sub-tile).  ``out`` may supply ``(V, codes, scales)`` buffers and
+    1 two-level CTA-wide, 2 single-level, 3 three warps per 32 x 32
+    sub-tile, 4 six warps per 64 x 64 sub-tile; :func:`tune_leaf` picks one by
+    measurement).  ``out`` may supply ``(V, codes, scales)`` buffers and
     ``ws`` a workspace; ``check_status=False`` skips the synchronising status
     read (for timing).
     """
@@ -135,12 +137,39 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     return V, codes, scales
 
 
+def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, timeout_ms=0):
+    """Leaf structure chosen by measurement (``bakron_tune_leaf``): one timed
+    solve per structure on this problem.  Returns ``(leaf, [ms_leaf1, ...,
+    ms_leaf4])``; pass ``leaf`` to :func:`solve`."""
+    torch = _torch()
+    lib = _lib()
+    _dev_f32(W, "W"), _dev_f32(LA, "LA"), _dev_f32(LB, "LB")
+    m, n = W.shape
+    cfg = _config(gemm, timeout_ms)
+    if out is None:
+        out = (torch.empty((m, n), dtype=torch.float32, device=W.device),
+               torch.empty((m, n), dtype=torch.int8, device=W.device),
+               torch.empty((m,), dtype=torch.float32, device=W.device))
+    V, codes, scales = out
+    if ws is None:
+        ws = workspace(lib.bakron_solve_workspace_size(m, n, ctypes.byref(cfg)), W.device)
+    q = Quantizer(int(bits), 0, 0, None)
+    leaf = ctypes.c_int32(0)
+    ms = (ctypes.c_double * 4)()
+    st = _stream(stream)
+    check(lib.bakron_tune_leaf(_ptr(W), m, n, _ptr(LA), _ptr(LB), ctypes.byref(q), _ptr(V), _ptr(codes),
+                               _ptr(scales), _ptr(ws), ws.numel(), ctypes.byref(cfg), st, ctypes.byref(leaf), ms),
+          "bakron_tune_leaf")
+    check(lib.bakron_get_status(_ptr(ws), ws.numel(), st), "bakron_tune_leaf (device)")
+    return int(leaf.value), [float(x) for x in ms]
+
+
 def solve_host_workspace_size(m: int, n: int, gemm: int = 0) -> int:
     return int(_lib().bakron_solve_host_workspace_size(m, n, ctypes.byref(_config(gemm))))
 
 
 def solve_host(W, LA, LB, bits=4, *, V=None, codes=None, scales=None, gemm=0, ws=None, stream=None,
-               synchronize=True):
+               synchronize=True, leaf=0):
     """BaKron solve on HOST buffers (torch CPU tensors, ideally pinned): the
     library stages them through ``ws`` on the device and copies the results
     back.  Returns ``(V, codes, scales)`` host tensors."""
@@ -153,7 +182,7 @@ def solve_host(W, LA, LB, bits=4, *, V=None, codes=None, scales=None, gemm=0, ws
     V = torch.empty((m, n), dtype=torch.float32, pin_memory=True) if V is None else V
     codes = torch.empty((m, n), dtype=torch.int8, pin_memory=True) if codes is None else codes
     scales = torch.empty((m,), dtype=torch.float32, pin_memory=True) if scales is None else scales
-    cfg = _config(gemm)
+    cfg = _config(gemm, leaf=leaf)
     if ws is None:
         ws = workspace(lib.bakron_solve_host_workspace_size(m, n, ctypes.byref(cfg)))
     q = Quantizer(int(bits), 0, 0, 0)

@@ -80,6 +80,9 @@ SIGNATURES = {
     "bakron_version": (ctypes.c_char_p, []),
     "bakron_get_profile": (ctypes.c_int, [ctypes.POINTER(Profile)]),
     "bakron_get_profile_launches": (_i64, [ctypes.POINTER(ProfileLaunch), _i64]),
+    "bakron_tune_leaf": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, ctypes.POINTER(Quantizer), _vp, _vp, _vp, _vp, _sz,
+                                        ctypes.POINTER(Config), _vp, ctypes.POINTER(ctypes.c_int32),
+                                        ctypes.POINTER(ctypes.c_double)]),
     "bakron_solve_noalloc": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, ctypes.POINTER(Quantizer), _vp, _vp, _vp,
                                             ctypes.POINTER(Config), _vp, ctypes.POINTER(ctypes.c_int32)]),
 }

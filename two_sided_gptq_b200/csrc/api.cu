@@ -99,7 +99,7 @@ bakron_status_t read_config(const bakron_config_t *c, Config &out)
     if (c->timeout_ms > 0) out.timeout_ms = c->timeout_ms;
     out.wt_out = c->wt_out;
     out.profile = c->profile ? 1 : 0;
-    if (c->leaf < 0 || c->leaf > 3) return BAKRON_ERR_INVALID_ARG;
+    if (c->leaf < 0 || c->leaf > 4) return BAKRON_ERR_INVALID_ARG;
     if (c->leaf != 0) out.leaf = c->leaf - 1;  // 0 keeps the default
     return BAKRON_OK;
 }
@@ -326,6 +326,50 @@ bakron_status_t bakron_solve(const float *W_dev, int64_t m, int64_t n, const flo
 {
     return solve_device(W_dev, m, n, LA_dev, LB_dev, q, V_dev, codes_dev, scales_dev, ws_dev, ws_bytes,
                         cfg, (cudaStream_t)stream, true);
+}
+
+bakron_status_t bakron_tune_leaf(const float *W_dev, int64_t m, int64_t n, const float *LA_dev,
+                                 const float *LB_dev, const bakron_quantizer_t *q, float *V_dev,
+                                 int8_t *codes_dev, float *scales_dev, void *ws_dev, size_t ws_bytes,
+                                 const bakron_config_t *cfg, bakron_stream_t stream, int32_t *leaf_out,
+                                 double *ms_out)
+{
+    if (!leaf_out) return BAKRON_ERR_INVALID_ARG;
+    bakron_config_t c = {};
+    if (cfg) c = *cfg;
+    if (c.profile) return BAKRON_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaEvent_t ev[2];
+    if (cudaEventCreate(&ev[0]) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (cudaEventCreate(&ev[1]) != cudaSuccess) {
+        cudaEventDestroy(ev[0]);
+        return BAKRON_ERR_CUDA;
+    }
+    bakron_status_t s = BAKRON_OK;
+    double best = 0.0;
+    int best_leaf = 0;
+    for (int leaf = 0; leaf <= 4 && s == BAKRON_OK; ++leaf) {
+        c.leaf = leaf == 0 ? 3 : leaf;  // round 0 is the warm-up
+        if (cudaEventRecord(ev[0], st) != cudaSuccess) { s = BAKRON_ERR_CUDA; break; }
+        s = bakron_solve(W_dev, m, n, LA_dev, LB_dev, q, V_dev, codes_dev, scales_dev, ws_dev, ws_bytes, &c, stream);
+        if (s != BAKRON_OK) break;
+        if (cudaEventRecord(ev[1], st) != cudaSuccess || cudaEventSynchronize(ev[1]) != cudaSuccess) {
+            s = BAKRON_ERR_CUDA;
+            break;
+        }
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, ev[0], ev[1]) != cudaSuccess) { s = BAKRON_ERR_CUDA; break; }
+        if (leaf == 0) continue;
+        if (ms_out) ms_out[leaf - 1] = ms;
+        if (best_leaf == 0 || ms < best) {
+            best = ms;
+            best_leaf = leaf;
+        }
+    }
+    cudaEventDestroy(ev[0]);
+    cudaEventDestroy(ev[1]);
+    if (s == BAKRON_OK) *leaf_out = best_leaf;
+    return s;
 }
 
 // Host-buffer variant: staging buffers follow the solve workspace.

@@ -764,12 +764,291 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
     }
 }
 
+// ------------------------------------------------------------------------
+// Wide variant: 2 x 2 sub-tiles of 64 in three sub-tile-diagonal phases (fewer
+// dependent steps than the 4 x 4 split: 3 x 127 instead of 7 x 63, and three
+// product phases instead of seven), six warps per row block of sub-tiles: two
+// entry warps (columns 0-31 / 32-63 of the sub-tile), two row-side warps (same
+// columns) and two column-side warps (rows 0-31 / 32-63), one 192-thread
+// barrier per step.  Phase e, sub-tile (p, q = e - p):
+//     S[p,q]  = LtB[1,0] D[0,q] for p = 1 (written into R's (1,q) block),
+//     W0[p,q] = Wt[p,q] - R[p,0] LtA[1,0]^T (q = 1) - S[p,q],
+// then the sweep as in the warp variant.  Wt blocks are staged by cp.async
+// into three slots (phase 0 uses slot 0; phase 1 slots 1, 2; phase 2 slot 0
+// again, staged during phase 1), LtA[1,0] once at the start.
+namespace {
+constexpr int SW = 64;                 // sub-tile side
+constexpr int LDW = SW + 4;            // row stride of slots and the LtA block
+constexpr int kThreadsWide = 384;
+constexpr size_t kSmemWide = ((size_t)2 * (T + 1) * RS3 + 4 * SW * LDW + 2 * T + T + 2 * 2 * 2 * SW) * sizeof(float) +
+                             (size_t)T * T + 32;
+static_assert(kSmemWide <= 232448, "wide leaf shared memory");
+}  // namespace
+
+__global__ void __launch_bounds__(kThreadsWide, 1) leaf_wide_kernel(LeafArgs p, int K, int I_lo)
+{
+    extern __shared__ __align__(16) float smem_f[];
+    float *sR = smem_f;                  // T x RS3 (+1 spare row): R, S before the sweep, 0 before that
+    float *sDt = sR + (T + 1) * RS3;     // T x RS3 (+1 spare row): D transposed
+    float *sSlot = sDt + (T + 1) * RS3;  // 3 slots of SW x LDW: Wt, then W0, then the pre-rounding values
+    float *sLA = sSlot + 3 * SW * LDW;   // LtA[1,0] block of the tile (SW x LDW)
+    float *scale = sLA + SW * LDW;       // T
+    float *rcp = scale + T;              // T
+    float *sLBd = rcp + T;               // T: LtB[r][r-1] inside each diagonal sub-block (0 on its first row)
+    float *sPS = sLBd + T;               // 2 x 2 x SW: column-side partial sums by column
+    float *sPU = sPS + 2 * 2 * SW;       // 2 x 2 x SW: row-side partial sums by column
+    int8_t *sCode = (int8_t *)(sPU + 2 * 2 * SW);  // T x T codes (+32 spare bytes)
+
+    const int I = I_lo + blockIdx.x, J = K - I;
+    const int64_t row0 = (int64_t)I * T, col0 = (int64_t)J * T;
+    const int mr = (int)min64(T, p.m - row0), nc = (int)min64(T, p.n - col0);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float *LAt = p.LA32 + col0 * p.Np + col0;
+    const float *LBt = p.LB32 + row0 * p.Mp + row0;
+    const int lda_g = (int)p.Np, ldb_g = (int)p.Mp;
+    for (int idx = tid; idx < 2 * T * (T / 32); idx += kThreadsWide) {
+        const int which = idx / (T * (T / 32)), r = (idx / (T / 32)) % T, seg = idx % (T / 32);
+        const float *ptr = which == 0 ? LAt + r * lda_g + 32 * seg : LBt + r * ldb_g + 32 * seg;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+    }
+    pdl_wait();
+
+    // Wt block of sub-tile (pp, q) into a slot
+    auto stage_wt = [&](int pp, int q, int slot) {
+        for (int c = tid; c < SW * (SW / 4); c += kThreadsWide) {
+            const int i = c / (SW / 4), k4 = c % (SW / 4);
+            cp_async16(sSlot + slot * SW * LDW + i * LDW + 4 * k4,
+                       p.Wt + (row0 + pp * SW + i) * p.Np + col0 + q * SW + 4 * k4);
+        }
+    };
+    stage_wt(0, 0, 0);
+    for (int c = tid; c < SW * (SW / 4); c += kThreadsWide) {  // LtA[1,0]
+        const int j = c / (SW / 4), k4 = c % (SW / 4);
+        cp_async16(sLA + j * LDW + 4 * k4, LAt + (SW + j) * lda_g + 4 * k4);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+
+    for (int idx = tid; idx < (T + 1) * RS3 / 4; idx += kThreadsWide) {
+        ((float4 *)sR)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+        ((float4 *)sDt)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (tid < T) {
+        const int blk = tid / SW, r = tid % SW;
+        sLBd[tid] = r > 0 ? LBt[(blk * SW + r) * ldb_g + blk * SW + r - 1] : 0.f;
+    }
+    const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
+    const int wp = warp / 6, wr = warp % 6, role = wr >> 1, half = wr & 1;
+    const bool exact_div = __syncthreads_or(load_scales(p, scale, rcp, row0, mr)) != 0;
+
+    for (int e = 0; e < 3; ++e) {
+        const int p_lo = max(0, e - 1), p_hi = min(1, e);
+        const bool mine = wp >= p_lo && wp <= p_hi;
+        const int qv = e - wp;
+        const int slot = e == 1 ? 1 + wp : 0;
+        // S[1,q] = LtB[1,0] D[0,q] into R's (1,q) block: four warps, 16 rows each
+        if (mine && wp == 1 && wr < 4) {
+            float acc[8][4] = {};
+            mma_block<8>(acc, LBt + SW * ldb_g, ldb_g, sDt + (qv * SW) * RS3, RS3, SW, wr * 16, 0);
+            const int g = lane >> 2, t = lane & 3;
+            float *o = sR + SW * RS3 + qv * SW;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const int j = nt * 8 + 2 * t;
+                o[(wr * 16 + g) * RS3 + j] = acc[nt][0];
+                o[(wr * 16 + g) * RS3 + j + 1] = acc[nt][1];
+                o[(wr * 16 + g + 8) * RS3 + j] = acc[nt][2];
+                o[(wr * 16 + g + 8) * RS3 + j + 1] = acc[nt][3];
+            }
+        }
+        // the sums' coefficient rows, columns <= (own index) - 2: row-side warps
+        // LtA[q,q] row b, column-side warps LtB[p,p] row rho (one register array
+        // serves either role); entry warps: LtA[b][b-1]
+        float2 coef[SW / 2];
+        float la_new = 0.f;
+        if (mine && role >= 1) {
+            const int x = half * 32 + lane;
+            const float *row = role == 1 ? LAt + (qv * SW + x) * lda_g + qv * SW : LBt + (wp * SW + x) * ldb_g + wp * SW;
+#pragma unroll
+            for (int c = 0; c < SW / 2; ++c) {
+                float2 v = make_float2(0.f, 0.f);
+                if (2 * c <= x - 2) v = *(const float2 *)(row + 2 * c);
+                v.y = 2 * c + 1 <= x - 2 ? v.y : 0.f;
+                coef[c] = v;
+            }
+        }
+        if (mine && role == 0) {
+            const int b = half * 32 + lane;
+            if (b > 0) la_new = LAt[(qv * SW + b) * lda_g + qv * SW + b - 1];
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncthreads();
+        // W0[p,q] = Wt[p,q] - R[p,0] LtA[1,0]^T (q = 1) - S[p,q], in place in the slot
+        if (mine && wr < 4) {
+            float acc[8][4] = {};
+            if (qv == 1) mma_block<8>(acc, sR + (wp * SW) * RS3, RS3, sLA, LDW, SW, wr * 16, 0);
+            const int g = lane >> 2, t = lane & 3;
+            float *o = sSlot + slot * SW * LDW;
+            const float *sq = sR + (wp * SW) * RS3 + qv * SW;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const int j = nt * 8 + 2 * t, i = wr * 16 + g;
+                o[i * LDW + j] -= acc[nt][0] + sq[i * RS3 + j];
+                o[i * LDW + j + 1] -= acc[nt][1] + sq[i * RS3 + j + 1];
+                o[(i + 8) * LDW + j] -= acc[nt][2] + sq[(i + 8) * RS3 + j];
+                o[(i + 8) * LDW + j + 1] -= acc[nt][3] + sq[(i + 8) * RS3 + j + 1];
+            }
+        }
+        __syncthreads();
+        if (e == 0) {  // phase 1's blocks, while phase 0 sweeps
+            stage_wt(0, 1, 1);
+            stage_wt(1, 0, 2);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        } else if (e == 1) {  // phase 2's block into the slot phase 0 used
+            stage_wt(1, 1, 0);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        }
+        if (mine) {
+            const int pp = wp, q = qv;
+            float *ps_buf = sPS + pp * 2 * SW;
+            float *pu_buf = sPU + pp * 2 * SW;
+            float *Wp = sSlot + slot * SW * LDW;
+            const float *LBd = sLBd + pp * SW;
+            const int bar_id = 1 + pp;
+            if (role == 0) {
+                const int b = half * 32 + lane, tb = q * SW + b;
+                auto row_consts = [&](int a, float &w0, float &lbn, float &sv, float &rv_, float &s0) {
+                    const int ac = min(max(a, 0), SW - 1);
+                    w0 = Wp[ac * LDW + b];
+                    lbn = LBd[ac];
+                    sv = scale[pp * SW + ac];
+                    rv_ = rcp[pp * SW + ac];
+                    s0 = sR[(pp * SW + ac) * RS3 + tb];
+                };
+                auto sweep = [&](auto ieee_tag) {
+                    constexpr bool kIeee = decltype(ieee_tag)::value;
+                    float w0, lb_new, sc_s, sc_r, s_ab;
+                    row_consts(-b, w0, lb_new, sc_s, sc_r, s_ab);
+                    float d_prev = 0.f;
+#pragma unroll 2
+                    for (int d = 0; d < 2 * SW - 1; ++d) {
+                        const int a = d - b;
+                        const int ac = min(max(a, 0), SW - 1);
+                        const float ps_in = d > 0 ? ps_buf[(d & 1) * SW + b] : 0.f;
+                        const float pu_in = d > 0 ? pu_buf[(d & 1) * SW + b] : 0.f;
+                        const float r_new = b > 0 ? sR[(pp * SW + ac) * RS3 + tb - 1] : 0.f;
+                        float w0n, lbn_n, sn, rn, s_n;
+                        row_consts(a + 1, w0n, lbn_n, sn, rn, s_n);
+                        const float sc = fmaf(lb_new, d_prev, ps_in);
+                        const float wt = w0 - fmaf(r_new, la_new, pu_in) - sc;
+                        const float qf = kIeee ? __fdiv_rn(wt, sc_s) : div_rn_recip(wt, sc_s, sc_r);
+                        const float cq = fminf(fmaxf(rintf(qf), fqmin), fqmax);
+                        const int ta = pp * SW + a;
+                        const bool valid = a >= 0 && a < SW && ta < mr && tb < nc;
+                        const float dl = valid ? fmaf(-sc_s, cq, wt) : 0.f;
+                        const int iR = valid ? ta * RS3 + tb : T * RS3 + lane;
+                        const int iD = valid ? tb * RS3 + ta : T * RS3 + lane;
+                        const int iC = valid ? ta * T + tb : T * T + lane;
+                        const int iW = valid ? a * LDW + b : ac * LDW + SW + (lane & 3);
+                        sR[iR] = s_ab + sc + dl;
+                        sDt[iD] = dl;
+                        sCode[iC] = code_byte(cq);
+                        Wp[iW] = wt;
+                        d_prev = dl;
+                        w0 = w0n; lb_new = lbn_n; sc_s = sn; sc_r = rn; s_ab = s_n;
+                        group_sync(bar_id, 192);
+                    }
+                };
+                if (exact_div)
+                    sweep(std::true_type{});
+                else
+                    sweep(std::false_type{});
+            } else if (role == 1) {
+                // row-side sums sum_{c <= b-2} R[a+1][c] LtA[b][c]
+                const int b = half * 32 + lane;
+                float4 rv[SW / 4];
+#pragma unroll
+                for (int c = 0; c < SW / 4; ++c) rv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                for (int d = 0; d < 2 * SW - 1; ++d) {
+                    const int an = min(max(d - b + 1, 0), SW - 1);
+                    const float *Rn = sR + (pp * SW + an) * RS3 + q * SW;
+#pragma unroll
+                    for (int c = 0; c < SW / 4; ++c)
+                        if (4 * c <= b - 2) rv[c] = *(const float4 *)(Rn + 4 * c);
+                    float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
+                    float2 u2 = make_float2(0.f, 0.f), u3 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int c = 0; c < SW / 4; c += 2) {
+                        u0 = ffma2(make_float2(rv[c].x, rv[c].y), coef[2 * c], u0);
+                        u1 = ffma2(make_float2(rv[c].z, rv[c].w), coef[2 * c + 1], u1);
+                        u2 = ffma2(make_float2(rv[c + 1].x, rv[c + 1].y), coef[2 * c + 2], u2);
+                        u3 = ffma2(make_float2(rv[c + 1].z, rv[c + 1].w), coef[2 * c + 3], u3);
+                    }
+                    pu_buf[((d + 1) & 1) * SW + b] = ((u0.x + u1.x) + (u2.x + u3.x)) + ((u0.y + u1.y) + (u2.y + u3.y));
+                    group_sync(bar_id, 192);
+                }
+            } else {
+                // column-side sums sum_{r <= rho-2} LtB[rho][r] D[r][b], b = d+1-rho
+                const int rho = half * 32 + lane;
+                float4 dv[SW / 4];
+#pragma unroll
+                for (int c = 0; c < SW / 4; ++c) dv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                for (int d = 0; d < 2 * SW - 1; ++d) {
+                    const int b = d + 1 - rho;
+                    const int bc = min(max(b, 0), SW - 1);
+                    const float *Dc = sDt + (q * SW + bc) * RS3 + pp * SW;
+#pragma unroll
+                    for (int c = 0; c < SW / 4; ++c)
+                        if (4 * c <= rho - 2) dv[c] = *(const float4 *)(Dc + 4 * c);
+                    float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+                    float2 s2 = make_float2(0.f, 0.f), s3 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int c = 0; c < SW / 4; c += 2) {
+                        s0 = ffma2(make_float2(dv[c].x, dv[c].y), coef[2 * c], s0);
+                        s1 = ffma2(make_float2(dv[c].z, dv[c].w), coef[2 * c + 1], s1);
+                        s2 = ffma2(make_float2(dv[c + 1].x, dv[c + 1].y), coef[2 * c + 2], s2);
+                        s3 = ffma2(make_float2(dv[c + 1].z, dv[c + 1].w), coef[2 * c + 3], s3);
+                    }
+                    if (b == bc)
+                        ps_buf[((d + 1) & 1) * SW + b] = ((s0.x + s1.x) + (s2.x + s3.x)) + ((s0.y + s1.y) + (s2.y + s3.y));
+                    group_sync(bar_id, 192);
+                }
+            }
+        }
+        __syncthreads();
+        if (p.wt_out) {
+            for (int idx = tid; idx < (p_hi - p_lo + 1) * SW * SW; idx += kThreadsWide) {
+                const int pp = p_lo + idx / (SW * SW), r = (idx / SW) % SW, c = idx % SW;
+                const int sl = e == 1 ? 1 + pp : 0;
+                const int ta = pp * SW + r, tb = (e - pp) * SW + c;
+                if (ta < mr && tb < nc) p.wt_out[(row0 + ta) * p.n + col0 + tb] = sSlot[sl * SW * LDW + r * LDW + c];
+            }
+        }
+    }
+    pdl_trigger();
+    for (int idx = tid; idx < T * T; idx += kThreadsWide) {
+        const int r = idx / T, c = idx % T;
+        if (r >= mr || c >= nc) continue;
+        const int64_t gi = row0 + r, gj = col0 + c;
+        const int8_t code = sCode[r * T + c];
+        p.codes[gi * p.n + gj] = code;
+        p.V[gi * p.n + gj] = scale[r] * (float)code;
+        float hi, lo;
+        split_tf32(sDt[c * RS3 + r], hi, lo);
+        p.Dhi[gi * p.Np + gj] = hi;
+        p.Dlo[gi * p.Np + gj] = lo;
+    }
+}
+
 cudaError_t leaf_configure()
 {
     cudaError_t e = cudaFuncSetAttribute(leaf_nested_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemNested);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(leaf_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemWarp);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(leaf_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemWide);
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(leaf_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemSingle);
 }
@@ -778,6 +1057,8 @@ cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stre
 {
     int I_lo = max(0, K - (p.Nt - 1)), I_hi = min(p.Mt - 1, K);
     if (I_hi < I_lo) return cudaSuccess;
+    if (variant == 3)
+        return launch_pdl(leaf_wide_kernel, dim3(I_hi - I_lo + 1), dim3(kThreadsWide), kSmemWide, stream, p, K, I_lo);
     if (variant == 2)
         return launch_pdl(leaf_warp_kernel, dim3(I_hi - I_lo + 1), dim3(kThreadsW), kSmemWarp, stream, p, K, I_lo);
     if (variant == 1)
