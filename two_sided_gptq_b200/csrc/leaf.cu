@@ -411,7 +411,7 @@ constexpr int RS3 = T + 4;         // row stride of sR / sDt: 33 float4 per row
 constexpr int WS3 = S3 + 4;        // row stride of the per-row-block slots
 constexpr int kLAStage = S3 * (3 * S3 * 2 + 4 * 3);  // largest phase: strips for q = 3, 2, 1
 constexpr size_t kSmemWarp =
-    ((size_t)2 * (T + 1) * RS3 + 2 * 4 * S3 * WS3 + kLAStage + 4 * S3 + 2 * T + 2 * 4 * 2 * S3) * sizeof(float) +
+    ((size_t)2 * (T + 1) * RS3 + 4 * S3 * WS3 + 2 * kLAStage + 4 * S3 + 2 * T + 2 * 4 * 2 * S3) * sizeof(float) +
     (size_t)T * T + 32;
 static_assert(kSmemWarp <= 232448, "leaf shared memory");
 }  // namespace
@@ -475,10 +475,10 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
     extern __shared__ __align__(16) float smem_f[];
     float *sR = smem_f;                  // T x RS3 (+1 spare row): R, S before the sweep, 0 before that
     float *sDt = sR + (T + 1) * RS3;     // T x RS3 (+1 spare row): D transposed, 0 where not rounded yet
-    float *sW = sDt + (T + 1) * RS3;     // 4 slots of S3 x WS3: W0 of the sub-tile being swept, then Wt
-    float *sWt = sW + 4 * S3 * WS3;      // 4 slots: Wt of the next sub-tile (staged during the sweep)
-    float *sLA = sWt + 4 * S3 * WS3;     // LtA[q, 0:q] strips of the next phase (staged during the sweep)
-    float *sLBd = sLA + kLAStage;        // 4 x S3: LtB sub-diagonal LtB[r][r-1] per row block
+    float *sW = sDt + (T + 1) * RS3;     // 4 slots of S3 x WS3: S, then W0 of the sub-tile being swept, then Wt
+    float *sLA = sW + 4 * S3 * WS3;      // LtA[q, 0:q] strips of the next phase (staged during the sweep)
+    float *sLBs = sLA + kLAStage;        // LtB[p, 0:p] strips of the next phase (staged during the sweep)
+    float *sLBd = sLBs + kLAStage;       // 4 x S3: LtB sub-diagonal LtB[r][r-1] per row block
     float *scale = sLBd + 4 * S3;        // T
     float *rcp = scale + T;              // T
     float *sPS = rcp + T;                // 4 x 2 x S3: column-side partial sums by column
@@ -502,13 +502,15 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
     }
     pdl_wait();  // every global input (Wt, factors, steps) comes from earlier kernels
 
-    // Stage, for the sub-tiles (p, q = e - p) of phase e, the tile's Wt block and
-    // the strip LtA[q, 0:q] (32 rows x 32 q columns, row stride 32 q + 4), strips
-    // laid out back to back in row-block order.  Every thread issues a share of
-    // 16-byte asynchronous copies and commits them as one group.
+    // Stage, for the sub-tiles (p, q = e - p) of phase e: the tile's Wt block
+    // into R's (p,q) block (untouched until then), the strip LtA[q, 0:q] (32
+    // rows x 32 q columns, row stride 32 q + 4) and the strip LtB[p, 0:p] (32
+    // rows x 32 p columns, row stride 32 p + 4), strips laid out back to back
+    // in row-block order.  Every thread issues a share of 16-byte asynchronous
+    // copies and commits them as one group.
     auto stage_phase = [&](int e) {
         if (e > 6) return;
-        int off = 0;
+        int off = 0, offb = 0;
         for (int pp = max(0, e - 3); pp <= min(3, e); ++pp) {
             const int q = e - pp;
             if (q > 0) {
@@ -519,27 +521,41 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
                 }
                 off += S3 * ld;
             }
+            if (pp > 0) {
+                const int ld = S3 * pp + 4, c4 = 8 * pp;
+                for (int c = tid; c < S3 * c4; c += kThreadsW) {
+                    const int i = c / c4, k4 = c - i * c4;
+                    cp_async16(sLBs + offb + i * ld + 4 * k4, LBt + (pp * S3 + i) * ldb_g + 4 * k4);
+                }
+                offb += S3 * ld;
+            }
             for (int c = tid; c < S3 * 8; c += kThreadsW) {
                 const int i = c >> 3, k4 = c & 7;
-                cp_async16(sWt + pp * S3 * WS3 + i * WS3 + 4 * k4,
+                cp_async16(sR + (pp * S3 + i) * RS3 + q * S3 + 4 * k4,
                            p.Wt + (row0 + pp * S3 + i) * p.Np + col0 + q * S3 + 4 * k4);
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    // offset of row block pp's strip in phase e
+    // offsets of row block pp's LtA and LtB strips in phase e
     auto la_offset = [](int e, int pp) {
         int off = 0;
         for (int p2 = max(0, e - 3); p2 < pp; ++p2)
             if (e - p2 > 0) off += S3 * (S3 * (e - p2) + 4);
         return off;
     };
-    stage_phase(0);
-
+    auto lb_offset = [](int e, int pp) {
+        int off = 0;
+        for (int p2 = max(0, e - 3); p2 < pp; ++p2)
+            if (p2 > 0) off += S3 * (S3 * p2 + 4);
+        return off;
+    };
     for (int idx = tid; idx < (T + 1) * RS3 / 4; idx += kThreadsW) {
         ((float4 *)sR)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
         ((float4 *)sDt)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    __syncthreads();  // R is zero before the first staged block lands in it
+    stage_phase(0);
     if (tid < T) {
         const int blk = tid / S3, r = tid % S3;
         sLBd[tid] = r > 0 ? LBt[(blk * S3 + r) * ldb_g + blk * S3 + r - 1] : 0.f;
@@ -566,19 +582,21 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
         const int p_lo = max(0, e - 3), p_hi = min(3, e);
         const bool mine = wp >= p_lo && wp <= p_hi;  // this warp's row block has a sub-tile in phase e
         const int qv = e - wp;
-        // S[p,q] = LtB[p, 0:p] D[0:p, q], written into R's (p,q) block (zero so far)
+        asm volatile("cp.async.wait_all;" ::: "memory");  // this phase's staged Wt blocks and strips
+        __syncthreads();
+        // S[p,q] = LtB[p, 0:p] D[0:p, q] into the row block's slot
         if (mine && role < 2 && wp > 0) {
             float acc[4][4] = {};
-            mma_block<4>(acc, LBt + (wp * S3) * ldb_g, ldb_g, sDt + (qv * S3) * RS3, RS3, wp * S3, i0, j0);
+            mma_block<4>(acc, sLBs + lb_offset(e, wp), S3 * wp + 4, sDt + (qv * S3) * RS3, RS3, wp * S3, i0, j0);
             const int g = lane >> 2, t = lane & 3;
-            float *o = sR + (wp * S3) * RS3 + qv * S3;
+            float *o = sW + wp * S3 * WS3;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const int j = j0 + nt * 8 + 2 * t;
-                o[(i0 + g) * RS3 + j] = acc[nt][0];
-                o[(i0 + g) * RS3 + j + 1] = acc[nt][1];
-                o[(i0 + g + 8) * RS3 + j] = acc[nt][2];
-                o[(i0 + g + 8) * RS3 + j + 1] = acc[nt][3];
+                o[(i0 + g) * WS3 + j] = acc[nt][0];
+                o[(i0 + g) * WS3 + j + 1] = acc[nt][1];
+                o[(i0 + g + 8) * WS3 + j] = acc[nt][2];
+                o[(i0 + g + 8) * WS3 + j + 1] = acc[nt][3];
             }
         }
         // row-side warp: LtA[q,q] row b (columns <= b-2); entry warp: LtA[b][b-1]
@@ -594,27 +612,27 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
             }
         }
         if (mine && role == 0 && lane > 0) la_new = LAt[(qv * S3 + lane) * lda_g + qv * S3 + lane - 1];
-        asm volatile("cp.async.wait_all;" ::: "memory");  // this phase's staged Wt and LtA strips
         __syncthreads();
-        // W0[p,q] = Wt[p,q] - R[p, 0:q] LtA[q, 0:q]^T - S[p,q]; the sweep adds the
-        // S terms of the row-side sums through R (R[p,q] starts as S[p,q])
+        // W0[p,q] = Wt[p,q] - R[p, 0:q] LtA[q, 0:q]^T - S[p,q] into the slot; R's
+        // (p,q) block (holding the staged Wt) becomes S: the sweep adds the S terms
+        // of the row-side sums through R
         if (mine && role < 2) {
             float acc[4][4] = {};
             if (qv > 0)
                 mma_block<4>(acc, sR + (wp * S3) * RS3, RS3, sLA + la_offset(e, wp), S3 * qv + 4, qv * S3, i0, j0);
             const int g = lane >> 2, t = lane & 3;
             float *o = sW + wp * S3 * WS3;
-            const float *wt = sWt + wp * S3 * WS3;
-            const float *sq = sR + (wp * S3) * RS3 + qv * S3;
+            float *rq = sR + (wp * S3) * RS3 + qv * S3;
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int j = j0 + nt * 8 + 2 * t;
-                o[(i0 + g) * WS3 + j] = wt[(i0 + g) * WS3 + j] - acc[nt][0] - sq[(i0 + g) * RS3 + j];
-                o[(i0 + g) * WS3 + j + 1] = wt[(i0 + g) * WS3 + j + 1] - acc[nt][1] - sq[(i0 + g) * RS3 + j + 1];
-                o[(i0 + g + 8) * WS3 + j] = wt[(i0 + g + 8) * WS3 + j] - acc[nt][2] - sq[(i0 + g + 8) * RS3 + j];
-                o[(i0 + g + 8) * WS3 + j + 1] =
-                    wt[(i0 + g + 8) * WS3 + j + 1] - acc[nt][3] - sq[(i0 + g + 8) * RS3 + j + 1];
-            }
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int i = i0 + g + 8 * (h >> 1), j = j0 + nt * 8 + 2 * t + (h & 1);
+                    const float sv = wp > 0 ? o[i * WS3 + j] : 0.f;
+                    const float wt = rq[i * RS3 + j];
+                    o[i * WS3 + j] = wt - acc[nt][h] - sv;
+                    rq[i * RS3 + j] = sv;
+                }
         }
         __syncthreads();
         stage_phase(e + 1);  // lands while this phase sweeps
