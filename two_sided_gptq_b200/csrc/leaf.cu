@@ -500,6 +500,13 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
         const float *ptr = which == 0 ? LAt + r * lda_g + 32 * seg : LBt + r * ldb_g + 32 * seg;
         asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
     }
+    // Zeroing R and D touches no global memory, so it overlaps the previous
+    // kernel's tail.
+    for (int idx = tid; idx < (T + 1) * RS3 / 4; idx += kThreadsW) {
+        ((float4 *)sR)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+        ((float4 *)sDt)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();  // R is zero before the first staged block lands in it
     pdl_wait();  // every global input (Wt, factors, steps) comes from earlier kernels
 
     // Stage, for the sub-tiles (p, q = e - p) of phase e: the tile's Wt block
@@ -550,11 +557,6 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
             if (p2 > 0) off += S3 * (S3 * p2 + 4);
         return off;
     };
-    for (int idx = tid; idx < (T + 1) * RS3 / 4; idx += kThreadsW) {
-        ((float4 *)sR)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
-        ((float4 *)sDt)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    __syncthreads();  // R is zero before the first staged block lands in it
     stage_phase(0);
     if (tid < T) {
         const int blk = tid / S3, r = tid % S3;
