@@ -59,17 +59,26 @@ typedef enum {
 /* Fixed per-row integer grid (the base quantizer; the method is modular in
  * it, per the arXiv abstract).  Row i has step s_i and codes in [qmin, qmax];
  * the rounding decision is clamp(rint(Wt_ij / s_i)) in fp32, ties to even.
- *   bits      2..8.
- *   qmin,qmax both 0 selects the symmetric range qmax = 2^(bits-1)-1,
- *             qmin = -qmax; otherwise -128 <= qmin < qmax <= 127.
- *   row_scale NULL: s_i = max_j |W_ij| / qmax (fp32, IEEE division; a row of
- *             zeros gets s_i = 1).  Non-NULL: device pointer to m positive
- *             finite steps, used as given. */
+ *   bits        2..8.
+ *   qmin,qmax   both 0 selects the symmetric range qmax = 2^(bits-1)-1,
+ *               qmin = -qmax; otherwise -128 <= qmin < qmax <= 127.
+ *   row_scale   NULL: steps computed on the device (below).  Non-NULL: device
+ *               pointer to m positive finite steps, used as given.
+ *   shrink_grid 0: s_i = max_j |W_ij| / qmax (fp32, IEEE division; a row of
+ *               zeros gets s_i = 1).  G in [2, 1024]: s_i is searched for the
+ *               least round-to-nearest error of row i ("per-row scaling factor
+ *               (shrink) up to factor 2, MSE search", the review's list of free
+ *               parameters): over c_k = 1 - fp32(k/2) / fp32(G-1), k = 0..G-1,
+ *               the step fp32(fp32(c_k * absmax_i) / qmax) whose error
+ *               sum_j (W_ij - s q_ij)^2, q_ij = clamp(rint(fp32(W_ij / s))),
+ *               summed in FP64, is smallest (the first k on equal errors).
+ *               Ignored when row_scale is given. */
 typedef struct {
     int32_t bits;
     int32_t qmin;
     int32_t qmax;
     const float *row_scale;
+    int32_t shrink_grid;
 } bakron_quantizer_t;
 
 /* Solver configuration (NULL = defaults; zero fields take defaults).

@@ -117,6 +117,48 @@ def scales(W: np.ndarray, qmax: int) -> np.ndarray:
     return s
 
 
+def shrink_candidates(grid: int) -> np.ndarray:
+    """The searched shrink factors ``c_k = 1 - (1/2) k / (grid - 1)``, k = 0..grid-1,
+    from 1 down to 1/2 ("per-row scaling factor (shrink) up to factor 2, MSE
+    search" in the review's free-parameter list), each rounded to fp32 as
+    ``1 - fp32(k/2) / fp32(grid - 1)``."""
+    k = np.arange(grid, dtype=np.float32)
+    return (np.float32(1.0) - (np.float32(0.5) * k) / np.float32(grid - 1)).astype(np.float32)
+
+
+def row_mse(W: np.ndarray, s: np.ndarray, qmin: int, qmax: int) -> np.ndarray:
+    """Round-to-nearest error of each row on its grid: ``sum_j (W_ij - s_i q_ij)^2``
+    with ``q = clamp(rint(fp32(W_ij / s_i)))``; the sum is taken in FP64."""
+    q = decide(W, s, qmin, qmax).astype(np.float64)
+    d = np.asarray(W, dtype=np.float32).astype(np.float64) - np.asarray(s, np.float32).astype(np.float64)[:, None] * q
+    return np.sum(d * d, axis=1)
+
+
+def scales_mse(W: np.ndarray, qmin: int, qmax: int, grid: int) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row step searched for the least round-to-nearest error: over the
+    candidates ``s_k = fp32(fp32(c_k * absmax) / qmax)`` (``c_k`` from
+    :func:`shrink_candidates`) the one with the smallest :func:`row_mse`, the
+    first (largest step) on equal errors; a zero row keeps ``s = 1``.  Returns
+    the steps and, per row, the relative gap between the best and the
+    second-best error (where two candidates' errors differ by less than the
+    FP64 summation order can, either is a valid answer)."""
+    W32 = np.asarray(W, dtype=np.float32)
+    amax = np.max(np.abs(W32), axis=1) if W32.shape[1] else np.zeros(W32.shape[0], np.float32)
+    cands = shrink_candidates(grid)
+    errs = np.empty((W32.shape[0], grid))
+    steps = np.empty((W32.shape[0], grid), np.float32)
+    for k, c in enumerate(cands):
+        sk = ((c * amax).astype(np.float32) / np.float32(qmax)).astype(np.float32)
+        sk[amax == 0] = np.float32(1.0)
+        steps[:, k] = sk
+        errs[:, k] = row_mse(W32, sk, qmin, qmax)
+    best = np.argmin(errs, axis=1)  # first index on equal errors
+    rows = np.arange(W32.shape[0])
+    s = steps[rows, best]
+    srt = np.sort(errs, axis=1)
+    gap = (srt[:, 1] - srt[:, 0]) / np.maximum(srt[:, 0], 1e-300) if grid > 1 else np.full(W32.shape[0], np.inf)
+    return s.astype(np.float32), gap
+
 def decide(Wt: np.ndarray, s: np.ndarray, qmin: int, qmax: int) -> np.ndarray:
     """Rounding decision in fp32: ``clamp(rint(float32(Wt) / s))`` (round half to even)."""
     x = np.asarray(Wt, dtype=np.float32) / np.asarray(s, dtype=np.float32)[:, None]

@@ -77,6 +77,10 @@ def test_argument_errors_return_before_any_device_work(lib):
     q_bad = _native.Quantizer(4, 3, -3, None)
     a[5] = ctypes.byref(q_bad)
     assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
+    for grid in (1, -2, 1025):  # the step search takes 2..1024 candidates
+        q_bad = _native.Quantizer(4, 0, 0, None, grid)
+        a[5] = ctypes.byref(q_bad)
+        assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
     cfg = _native.Config(0, 5, 0, 0, None)
     a = list(args())
     a[11] = ctypes.byref(cfg)

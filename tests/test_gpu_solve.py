@@ -145,3 +145,31 @@ def test_tune_leaf_picks_a_measured_structure():
     assert leaf in (1, 2, 3, 4) and all(t > 0 for t in ms)
     assert ms[leaf - 1] == min(ms)
     check_solve(W, LA, LB, 4, leaf=leaf, label=f"mid/tuned-leaf{leaf}")
+
+
+@pytest.mark.parametrize("case", [("mid", 4, 100), ((300, 260), 3, 64), ((129, 257), 2, 20)])
+def test_mse_searched_steps(case):
+    """shrink_grid: the device's searched steps equal the oracle's (a row whose
+    two best candidates' errors lie within 1e-12 of each other may take either:
+    FP64 summation order decides there), and the solve on those steps meets the
+    parity contract."""
+    import torch
+
+    import two_sided_gptq_b200 as bk
+
+    what, bits, grid = case
+    if isinstance(what, str):
+        W, A, B, LA, LB = named(what)
+    else:
+        W, A, B = workloads.random_problem(*what, seed=sum(what) + grid)
+        LA, LB = oracle_factors(A, B)
+    qmin, qmax = oracle.grid(bits)
+    Wd, LAd, LBd = (torch.from_numpy(x).cuda() for x in (W, LA, LB))
+    _, _, s_gpu = bk.solve(Wd, LAd, LBd, bits=bits, shrink_grid=grid)
+    s_gpu = s_gpu.cpu().numpy()
+    s_or, gap = oracle.scales_mse(W, qmin, qmax, grid)
+    diff = s_gpu != s_or
+    print(f"[mse {what}] rows {len(s_or)} differing {int(diff.sum())} shrunk {int((s_or < oracle.scales(W, qmax)).sum())}")
+    assert np.all(gap[diff] < 1e-12), (np.nonzero(diff)[0][:5], gap[diff][:5])
+    assert (s_or < oracle.scales(W, qmax)).any()  # the search does move some steps
+    check_solve(W, LA, LB, bits, row_scale=s_gpu, label=f"{what}/mse{grid}")

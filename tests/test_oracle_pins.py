@@ -387,3 +387,58 @@ def test_planted_mistakes_are_caught(oracle_mod):
     assert not np.array_equal(o.solve(W2, LtB2, LtA2, s2, qmin, qmax)[0], ref2)
     assert np.array_equal(o.solve(W2, LtA2, LtB2, s2, qmin, qmax)[0], ref2)
     del ref
+
+
+# ---------------------------------------------------------------------------
+# Per-row step searched for the least round-to-nearest error ("per-row
+# scaling factor (shrink) up to factor 2, MSE search": review, free parameters)
+# ---------------------------------------------------------------------------
+def test_shrink_candidates_span_one_to_one_half(oracle_mod):
+    oracle = oracle_mod
+    c = oracle.shrink_candidates(100)
+    assert c[0] == np.float32(1.0) and c[-1] == np.float32(0.5)
+    assert np.all(np.diff(c) < 0) and c.dtype == np.float32
+    assert list(oracle.shrink_candidates(2)) == [1.0, 0.5]
+
+
+def test_shrink_search_hand_examples(oracle_mod):
+    oracle = oracle_mod
+    # INT2 (q in {-1, 0, 1}), candidates {1, 1/2}.
+    # [0.7, 0.34, 0.34]: step 0.7 rounds the small entries to 0 (error
+    # 2 * 0.34^2 = 0.2312); step 0.35 keeps 0.7 at the clamp (error 0.35^2) and
+    # rounds 0.34 to 0.35 (error 2 * 0.01^2): 0.1227 < 0.2312, so 0.35.
+    # [0.7, 0.3, 0]: step 0.7 costs 0.3^2 = 0.09; step 0.35 costs
+    # 0.35^2 + 0.05^2 = 0.125, so 0.7.
+    W = np.array([[0.7, 0.34, 0.34], [0.7, 0.3, 0.0]], np.float32)
+    s, gap = oracle.scales_mse(W, -1, 1, 2)
+    assert s[0] == np.float32(np.float32(0.5) * np.float32(0.7)) / np.float32(1)
+    assert s[1] == np.float32(0.7)
+    err = oracle.row_mse(W, s, -1, 1)
+    assert abs(err[0] - (0.35 ** 2 + 2 * 0.01 ** 2)) < 1e-6 and abs(err[1] - 0.09) < 1e-6
+
+
+def test_shrink_search_on_grid_row_keeps_absmax_step(oracle_mod):
+    oracle = oracle_mod
+    # a row that already lies on its absmax grid has zero error at c = 1, the
+    # first candidate, so the search keeps s = absmax / qmax
+    rng = np.random.default_rng(4)
+    qmax = 7
+    s0 = np.float32(0.0123)
+    ints = rng.integers(-qmax, qmax + 1, size=(5, 40)).astype(np.float32)
+    ints[:, 0] = qmax
+    W = (ints * s0).astype(np.float32)
+    s, _ = oracle.scales_mse(W, -qmax, qmax, 50)
+    assert np.array_equal(s, oracle.scales(W, qmax))
+    assert np.all(oracle.row_mse(W, s, -qmax, qmax) < 1e-18)
+
+
+def test_shrink_search_never_worse_than_absmax_and_scales_with_rows(oracle_mod):
+    oracle = oracle_mod
+    rng = np.random.default_rng(5)
+    W = (rng.standard_t(3, size=(20, 64)) * 0.02).astype(np.float32)
+    s, _ = oracle.scales_mse(W, -7, 7, 40)
+    assert np.all(oracle.row_mse(W, s, -7, 7) <= oracle.row_mse(W, oracle.scales(W, 7), -7, 7))
+    assert np.all(s <= oracle.scales(W, 7)) and np.all(s >= oracle.scales(W, 7) * np.float32(0.5))
+    # a power-of-two scaling of a row scales its step exactly
+    s2, _ = oracle.scales_mse((W * np.float32(8)).astype(np.float32), -7, 7, 40)
+    assert np.array_equal(s2, (s * np.float32(8)).astype(np.float32))

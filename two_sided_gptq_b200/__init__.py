@@ -102,11 +102,13 @@ def solve_workspace_size(m: int, n: int, gemm: int = 0) -> int:
 
 
 def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None, out=None, stream=None,
-          wt_out=None, check_status=True, timeout_ms=0, profile=False, leaf=0):
+          wt_out=None, check_status=True, timeout_ms=0, profile=False, leaf=0, shrink_grid=0):
     """BaKron solve on device tensors.  Returns ``(V, codes, scales)``.
 
     ``gemm=0`` uses the tcgen05 3xTF32 band products, ``gemm=1`` the FP32
-    CUDA-core ones; ``leaf`` selects the leaf sweep structure (0 default,
+    CUDA-core ones; ``shrink_grid`` > 1 searches each row's step for the least
+    round-to-nearest error over that many shrink factors in [1/2, 1]; ``leaf``
+    selects the leaf sweep structure (0 default,
     1 two-level CTA-wide, 2 single-level, 3 three warps per 32 x 32
     sub-tile, 4 six warps per 64 x 64 sub-tile; :func:`tune_leaf` picks one by
     measurement).  ``out`` may supply ``(V, codes, scales)`` buffers and
@@ -128,7 +130,7 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
         V, codes, scales = out
     if ws is None:
         ws = workspace(lib.bakron_solve_workspace_size(m, n, ctypes.byref(cfg)), W.device)
-    q = Quantizer(int(bits), int(qmin), int(qmax), _ptr(row_scale))
+    q = Quantizer(int(bits), int(qmin), int(qmax), _ptr(row_scale), int(shrink_grid))
     st = _stream(stream)
     check(lib.bakron_solve(_ptr(W), m, n, _ptr(LA), _ptr(LB), ctypes.byref(q), _ptr(V), _ptr(codes), _ptr(scales),
                            _ptr(ws), ws.numel(), ctypes.byref(cfg), st), "bakron_solve")

@@ -33,7 +33,7 @@ class BakronError(RuntimeError):
 
 class Quantizer(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int32), ("qmin", ctypes.c_int32), ("qmax", ctypes.c_int32),
-                ("row_scale", ctypes.c_void_p)]
+                ("row_scale", ctypes.c_void_p), ("shrink_grid", ctypes.c_int32)]
 
 
 class Config(ctypes.Structure):

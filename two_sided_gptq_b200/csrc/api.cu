@@ -108,6 +108,7 @@ bakron_status_t read_grid(const bakron_quantizer_t *q, int &qmin, int &qmax)
 {
     if (!q) return BAKRON_ERR_INVALID_ARG;
     if (q->bits < 2 || q->bits > 8) return BAKRON_ERR_INVALID_ARG;
+    if (q->shrink_grid != 0 && (q->shrink_grid < 2 || q->shrink_grid > 1024)) return BAKRON_ERR_INVALID_ARG;
     if (q->qmin == 0 && q->qmax == 0) {
         qmax = (1 << (q->bits - 1)) - 1;
         qmin = -qmax;
@@ -207,7 +208,8 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
     t_prof.kinds.clear();
     t_prof.nodes.clear();
     t_prof.begin(0);
-    if (launch_prep(W, m, n, LA, LB, qmax, q->row_scale, scales, L, w, stream) != cudaSuccess)
+    if (launch_prep(W, m, n, LA, LB, qmin, qmax, q->row_scale, q->row_scale ? 0 : q->shrink_grid, scales, L, w,
+                    stream) != cudaSuccess)
         return BAKRON_ERR_CUDA;
     t_prof.end();
 

@@ -30,8 +30,8 @@ struct GemmArgs {
     int timeout_ms;
 };
 
-cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, const float *LB,
-                        int qmax, const float *user_scales, float *scales, const SolveLayout &L,
+cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, const float *LB, int qmin,
+                        int qmax, const float *user_scales, int shrink_grid, float *scales, const SolveLayout &L,
                         char *ws, cudaStream_t stream);
 
 cudaError_t leaf_configure();
