@@ -381,6 +381,41 @@ def main():
     e2e_ms = max_over_ranks(h0.elapsed_time(h1) / e2e_steps, dist, dev)
     assert np.array_equal(ch.numpy(), codes.cpu().numpy()), "host-buffer solve disagrees with device solve"
 
+    # several matrices at once (bakron_solve_batch on separate streams): one
+    # solve keeps few SMs busy during its leaf sweeps, so solves overlap
+    n_batch = 4
+    bstreams = [torch.cuda.Stream(device=dev) for _ in range(n_batch)]
+    bouts = [(torch.empty((m, n), dtype=torch.float32, device=dev), torch.empty((m, n), dtype=torch.int8, device=dev),
+              torch.empty((m,), dtype=torch.float32, device=dev)) for _ in range(n_batch)]
+    bws = [bk.workspace(bk.solve_workspace_size(m, n), dev) for _ in range(n_batch)]
+    probs = [(Wd, LA, LB)] * n_batch
+
+    def batch_step():
+        start = torch.cuda.Event()
+        start.record(stream)
+        for bs in bstreams:
+            bs.wait_event(start)
+        bk.solve_batch(probs, bits=w.bits, streams=bstreams, outs=bouts, workspaces=bws, leaf=leaf,
+                       check_status=False)
+        for bs in bstreams:
+            done = torch.cuda.Event()
+            done.record(bs)
+            stream.wait_event(done)
+
+    for _ in range(2):
+        batch_step()
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b_steps = 3
+    b0.record(stream)
+    for _ in range(b_steps):
+        batch_step()
+    b1.record(stream)
+    torch.cuda.synchronize()
+    batch_ms = max_over_ranks(b0.elapsed_time(b1) / b_steps, dist, dev)
+    assert torch.equal(bouts[-1][1], codes), "batched solve disagrees with the single solve"
+    del bws, bouts
+
     line = None
     if rank == 0:
         cb = None
@@ -415,6 +450,9 @@ def main():
             "e2e": {"value": aggregate_rate(world, m, n, e2e_ms), "unit": "weights/s",
                     "h2d_bytes_per_step": 4 * (m * n + n * n + m * m),
                     "d2h_bytes_per_step": 4 * m * n + m * n + 4 * m},
+            "batch": {"matrices_per_step": n_batch, "streams": n_batch, "ms_per_step": batch_ms,
+                      "value": aggregate_rate(world, m, n, batch_ms / n_batch), "unit": "weights/s",
+                      "note": "bakron_solve_batch of the same workload on separate streams (not the headline)"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "device_status": status.name,

@@ -183,6 +183,26 @@ bakron_status_t bakron_tune_leaf(const float *W_dev, int64_t m, int64_t n, const
                                  const bakron_config_t *cfg, bakron_stream_t stream, int32_t *leaf_out,
                                  double *ms_out);
 
+/* Several independent solves (for instance the weight matrices of a model's
+ * layers), solve i enqueued on streams[i % nstreams].  One solve keeps few SMs
+ * busy while its leaf sweeps run (one CTA per tile of a tile diagonal), so
+ * solves on different streams overlap.  Every item needs its own workspace
+ * (and its own outputs); all items share the grid and the config.  All
+ * arguments are checked before anything is enqueued: the first invalid item's
+ * status is returned and nothing runs.  cfg->profile must be 0. */
+typedef struct {
+    const float *W_dev;
+    int64_t m, n;
+    const float *LA_dev, *LB_dev;
+    float *V_dev;
+    int8_t *codes_dev;
+    float *scales_dev;
+    void *ws_dev;
+    size_t ws_bytes;
+} bakron_batch_item_t;
+bakron_status_t bakron_solve_batch(const bakron_batch_item_t *items, int32_t count, const bakron_quantizer_t *q,
+                                   const bakron_config_t *cfg, const bakron_stream_t *streams, int32_t nstreams);
+
 /* Bytes of device workspace bakron_solve_host needs (solve workspace plus
  * device staging for W, LA, LB, V, codes and scales). */
 size_t bakron_solve_host_workspace_size(int64_t m, int64_t n, const bakron_config_t *cfg);

@@ -155,3 +155,25 @@ def test_plan_stats_4096_cubic_work(lib):
     assert 4096 ** 2 * 8192 < f < 2 * 4096 ** 2 * 8192
     r = flops(8192, 8192) / f
     assert 7.0 < r < 9.0, r
+
+
+def test_solve_batch_argument_errors_before_device_work(lib):
+    """bakron_solve_batch checks every item before it enqueues anything."""
+    from two_sided_gptq_b200 import _native
+
+    q = _native.Quantizer(4, 0, 0, None)
+    fake = 1 << 20
+    st = (ctypes.c_void_p * 1)(None)
+    assert lib.bakron_solve_batch(None, 0, ctypes.byref(q), None, st, 1) == _native.Status.OK  # nothing to do
+    assert lib.bakron_solve_batch(None, -1, ctypes.byref(q), None, st, 1) == _native.Status.ERR_INVALID_ARG
+    items = (_native.BatchItem * 2)()
+    good = _native.BatchItem(fake, 8, 8, fake, fake, fake, fake, fake, fake, 1 << 30)
+    items[0] = good
+    items[1] = _native.BatchItem(fake, 0, 8, fake, fake, fake, fake, fake, fake, 1 << 30)  # m = 0
+    assert lib.bakron_solve_batch(items, 2, ctypes.byref(q), None, st, 1) == _native.Status.ERR_INVALID_ARG
+    items[1] = _native.BatchItem(fake + 4, 8, 8, fake, fake, fake, fake, fake, fake, 1 << 30)  # misaligned W
+    assert lib.bakron_solve_batch(items, 2, ctypes.byref(q), None, st, 1) == _native.Status.ERR_ALIGNMENT
+    items[1] = _native.BatchItem(fake, 8, 8, fake, fake, fake, fake, fake, fake, 16)  # short workspace
+    assert lib.bakron_solve_batch(items, 2, ctypes.byref(q), None, st, 1) == _native.Status.ERR_WORKSPACE
+    assert lib.bakron_solve_batch(items, 2, ctypes.byref(q), None, st, 0) == _native.Status.ERR_INVALID_ARG
+

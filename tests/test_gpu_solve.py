@@ -173,3 +173,23 @@ def test_mse_searched_steps(case):
     assert np.all(gap[diff] < 1e-12), (np.nonzero(diff)[0][:5], gap[diff][:5])
     assert (s_or < oracle.scales(W, qmax)).any()  # the search does move some steps
     check_solve(W, LA, LB, bits, row_scale=s_gpu, label=f"{what}/mse{grid}")
+
+
+def test_solve_batch_equals_single_solves():
+    """bakron_solve_batch: independent solves of different shapes on two
+    streams give the same results as one-at-a-time solves."""
+    import torch
+
+    import two_sided_gptq_b200 as bk
+
+    probs = []
+    for (m, n) in ((300, 260), (129, 257), (256, 512)):
+        W, A, B = workloads.random_problem(m, n, seed=m * 7 + n)
+        LA, LB = oracle_factors(A, B)
+        probs.append(tuple(torch.from_numpy(x).cuda() for x in (W, LA, LB)))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    res = bk.solve_batch(probs, bits=4, streams=streams)
+    torch.cuda.synchronize()
+    for (W, LA, LB), (V, codes, scales) in zip(probs, res):
+        V1, c1, s1 = bk.solve(W, LA, LB, bits=4)
+        assert torch.equal(codes, c1) and torch.equal(scales, s1) and torch.equal(V, V1)

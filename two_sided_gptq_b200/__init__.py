@@ -16,9 +16,9 @@ from __future__ import annotations
 import ctypes
 
 from . import _native
-from ._native import BakronError, Config, PlanStats, Profile, ProfileLaunch, Quantizer, Status, check
+from ._native import BakronError, BatchItem, Config, PlanStats, Profile, ProfileLaunch, Quantizer, Status, check
 
-__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile", "last_profile_launches", "tune_leaf",
+__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile", "last_profile_launches", "tune_leaf", "solve_batch",
            "workspace", "get_status",
            "BakronError", "Status", "version", "library_path"]
 
@@ -164,6 +164,44 @@ def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, time
           "bakron_tune_leaf")
     check(lib.bakron_get_status(_ptr(ws), ws.numel(), st), "bakron_tune_leaf (device)")
     return int(leaf.value), [float(x) for x in ms]
+
+
+def solve_batch(problems, bits=4, *, streams, outs=None, workspaces=None, gemm=0, leaf=0, shrink_grid=0,
+                check_status=True):
+    """Independent solves through ``bakron_solve_batch``: ``problems`` is a list
+    of ``(W, LA, LB)`` device tensors, solve i runs on ``streams[i %
+    len(streams)]`` (torch streams).  ``outs`` / ``workspaces`` may supply the
+    ``(V, codes, scales)`` buffers and workspaces.  Returns the list of
+    ``(V, codes, scales)``."""
+    torch = _torch()
+    lib = _lib()
+    cfg = _config(gemm, leaf=leaf)
+    items = (BatchItem * max(1, len(problems)))()
+    res, wss = [], []
+    for i, (W, LA, LB) in enumerate(problems):
+        _dev_f32(W, "W"), _dev_f32(LA, "LA"), _dev_f32(LB, "LB")
+        m, n = W.shape
+        if outs is None:
+            o = (torch.empty((m, n), dtype=torch.float32, device=W.device),
+                 torch.empty((m, n), dtype=torch.int8, device=W.device),
+                 torch.empty((m,), dtype=torch.float32, device=W.device))
+        else:
+            o = outs[i]
+        ws = workspaces[i] if workspaces is not None else workspace(
+            lib.bakron_solve_workspace_size(m, n, ctypes.byref(cfg)), W.device)
+        items[i] = BatchItem(_ptr(W), m, n, _ptr(LA), _ptr(LB), _ptr(o[0]), _ptr(o[1]), _ptr(o[2]), _ptr(ws),
+                             ws.numel())
+        res.append(o)
+        wss.append(ws)
+    st = (ctypes.c_void_p * len(streams))(*[s.cuda_stream for s in streams])
+    q = Quantizer(int(bits), 0, 0, None, int(shrink_grid))
+    check(lib.bakron_solve_batch(items, len(problems), ctypes.byref(q), ctypes.byref(cfg), st, len(streams)),
+          "bakron_solve_batch")
+    if check_status:
+        for i, ws in enumerate(wss):
+            check(lib.bakron_get_status(_ptr(ws), ws.numel(), _stream(streams[i % len(streams)])),
+                  f"bakron_solve_batch item {i} (device)")
+    return res
 
 
 def solve_host_workspace_size(m: int, n: int, gemm: int = 0) -> int:

@@ -36,6 +36,12 @@ class Quantizer(ctypes.Structure):
                 ("row_scale", ctypes.c_void_p), ("shrink_grid", ctypes.c_int32)]
 
 
+class BatchItem(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("m", ctypes.c_int64), ("n", ctypes.c_int64), ("LA", ctypes.c_void_p),
+                ("LB", ctypes.c_void_p), ("V", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("ws", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t)]
+
+
 class Config(ctypes.Structure):
     _fields_ = [("tile", ctypes.c_int32), ("gemm", ctypes.c_int32), ("use_graph", ctypes.c_int32),
                 ("timeout_ms", ctypes.c_int32), ("wt_out", ctypes.c_void_p), ("profile", ctypes.c_int32),
@@ -80,6 +86,8 @@ SIGNATURES = {
     "bakron_version": (ctypes.c_char_p, []),
     "bakron_get_profile": (ctypes.c_int, [ctypes.POINTER(Profile)]),
     "bakron_get_profile_launches": (_i64, [ctypes.POINTER(ProfileLaunch), _i64]),
+    "bakron_solve_batch": (ctypes.c_int, [ctypes.POINTER(BatchItem), ctypes.c_int32, ctypes.POINTER(Quantizer),
+                                          ctypes.POINTER(Config), ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
     "bakron_tune_leaf": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, ctypes.POINTER(Quantizer), _vp, _vp, _vp, _vp, _sz,
                                         ctypes.POINTER(Config), _vp, ctypes.POINTER(ctypes.c_int32),
                                         ctypes.POINTER(ctypes.c_double)]),

@@ -374,6 +374,38 @@ bakron_status_t bakron_tune_leaf(const float *W_dev, int64_t m, int64_t n, const
     return s;
 }
 
+bakron_status_t bakron_solve_batch(const bakron_batch_item_t *items, int32_t count, const bakron_quantizer_t *q,
+                                   const bakron_config_t *cfg, const bakron_stream_t *streams, int32_t nstreams)
+{
+    if (count < 0 || (count > 0 && (!items || !streams || nstreams < 1))) return BAKRON_ERR_INVALID_ARG;
+    if (cfg && cfg->profile) return BAKRON_ERR_INVALID_ARG;
+    Config conf;
+    bakron_status_t s = read_config(cfg, conf);
+    if (s != BAKRON_OK) return s;
+    int qmin = 0, qmax = 0;
+    if ((s = read_grid(q, qmin, qmax)) != BAKRON_OK) return s;
+    for (int32_t i = 0; i < count; ++i) {  // the checks bakron_solve makes before it enqueues
+        const bakron_batch_item_t &it = items[i];
+        if (it.m < 1 || it.n < 1 || it.m > kMaxSide || it.n > kMaxSide) return BAKRON_ERR_INVALID_ARG;
+        if (!it.W_dev || !it.LA_dev || !it.LB_dev || !it.V_dev || !it.codes_dev || !it.scales_dev)
+            return BAKRON_ERR_INVALID_ARG;
+        if (!it.ws_dev) return BAKRON_ERR_WORKSPACE;
+        if (!aligned16(it.W_dev) || !aligned16(it.LA_dev) || !aligned16(it.LB_dev) || !aligned16(it.V_dev) ||
+            !aligned16(it.codes_dev) || !aligned16(it.scales_dev) || !aligned16(it.ws_dev))
+            return BAKRON_ERR_ALIGNMENT;
+        SolveLayout L;
+        L.compute(it.m, it.n, kTile);
+        if (it.ws_bytes < L.total) return BAKRON_ERR_WORKSPACE;
+    }
+    for (int32_t i = 0; i < count; ++i) {
+        const bakron_batch_item_t &it = items[i];
+        s = bakron_solve(it.W_dev, it.m, it.n, it.LA_dev, it.LB_dev, q, it.V_dev, it.codes_dev, it.scales_dev,
+                         it.ws_dev, it.ws_bytes, cfg, streams[i % nstreams]);
+        if (s != BAKRON_OK) return s;
+    }
+    return BAKRON_OK;
+}
+
 // Host-buffer variant: staging buffers follow the solve workspace.
 namespace {
 struct HostLayout {
