@@ -128,6 +128,20 @@ typedef struct {
 /* Copies min(count, cap) records to `out` (may be NULL) and returns count. */
 int64_t bakron_get_profile_launches(bakron_profile_launch_t *out, int64_t cap);
 
+/* ------------------------------------------------------------------ gram */
+/* The Kronecker factor from calibration samples, the step before
+ * bakron_factor (the pages build A and B as expectations of a a^T over
+ * activation / gradient samples, regularised by a multiple of the mean
+ * diagonal: "Assumptions & free parameters", Gram matrix regularisation):
+ *   A_dev (d x d) <- X^T X / N + damping * mean_i (X^T X / N)_ii * I
+ * for X_dev (N x d, row-major samples).  The product runs on the tensor cores
+ * in 3xTF32 (lower tiles), each FP32 sum / N rounded once; A is written in
+ * full (symmetric).  damping >= 0.  Device errors: BAKRON_ERR_NONFINITE (X).
+ * Workspace: bakron_gram_workspace_size(N, d) bytes (X^T split, the product). */
+size_t bakron_gram_workspace_size(int64_t N, int64_t d);
+bakron_status_t bakron_gram(const float *X_dev, int64_t N, int64_t d, float damping, float *A_dev, void *ws_dev,
+                            size_t ws_bytes, bakron_stream_t stream);
+
 /* ---------------------------------------------------------------- factor */
 /* Bytes of workspace bakron_factor needs for factors of sizes n and m. */
 size_t bakron_factor_workspace_size(int64_t n, int64_t m);

@@ -165,6 +165,15 @@ def decide(Wt: np.ndarray, s: np.ndarray, qmin: int, qmax: int) -> np.ndarray:
     return np.clip(np.rint(x), qmin, qmax).astype(np.int32)
 
 
+def gram(X: np.ndarray, damping: float = 0.0) -> np.ndarray:
+    """Kronecker factor from samples (rows of ``X``): ``X^T X / N`` plus
+    ``damping * mean(diag) * I`` (the pages' Gram-matrix regularisation), in
+    FP64."""
+    X64 = np.asarray(X, dtype=np.float64)
+    A = X64.T @ X64 / X64.shape[0]
+    return A + damping * np.mean(np.diag(A)) * np.eye(A.shape[0])
+
+
 # --------------------------------------------------------------------------
 # Factors.
 # --------------------------------------------------------------------------

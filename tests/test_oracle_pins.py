@@ -442,3 +442,17 @@ def test_shrink_search_never_worse_than_absmax_and_scales_with_rows(oracle_mod):
     # a power-of-two scaling of a row scales its step exactly
     s2, _ = oracle.scales_mse((W * np.float32(8)).astype(np.float32), -7, 7, 40)
     assert np.array_equal(s2, (s * np.float32(8)).astype(np.float32))
+
+
+def test_gram_closed_forms(oracle_mod):
+    oracle = oracle_mod
+    # X = [[1, 2], [3, 4]]: X^T X / 2 = [[5, 7], [7, 10]], mean diagonal 7.5
+    X = np.array([[1.0, 2.0], [3.0, 4.0]])
+    assert np.allclose(oracle.gram(X), [[5.0, 7.0], [7.0, 10.0]], rtol=0, atol=1e-15)
+    assert np.allclose(oracle.gram(X, 0.1), [[5.75, 7.0], [7.0, 10.75]], rtol=0, atol=1e-15)
+    # orthogonal columns give a diagonal factor; sample order does not matter
+    Q, _ = np.linalg.qr(np.random.default_rng(6).standard_normal((50, 6)))
+    X = Q * np.array([1.0, 2.0, 3.0, 4.0, 5.0, 6.0])
+    A = oracle.gram(X)
+    assert np.allclose(A, np.diag(np.array([1, 4, 9, 16, 25, 36]) / 50.0), atol=1e-14)
+    assert np.allclose(oracle.gram(X[::-1]), A, atol=1e-14)

@@ -18,7 +18,7 @@ import ctypes
 from . import _native
 from ._native import BakronError, BatchItem, Config, PlanStats, Profile, ProfileLaunch, Quantizer, Status, check
 
-__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile", "last_profile_launches", "tune_leaf", "solve_batch",
+__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile", "last_profile_launches", "tune_leaf", "solve_batch", "gram",
            "workspace", "get_status",
            "BakronError", "Status", "version", "library_path"]
 
@@ -202,6 +202,23 @@ def solve_batch(problems, bits=4, *, streams, outs=None, workspaces=None, gemm=0
             check(lib.bakron_get_status(_ptr(ws), ws.numel(), _stream(streams[i % len(streams)])),
                   f"bakron_solve_batch item {i} (device)")
     return res
+
+
+def gram(X, damping=0.0, *, ws=None, out=None, stream=None, check_status=True):
+    """Kronecker factor ``X^T X / N + damping * mean(diag) * I`` from samples
+    ``X`` (N x d device tensor) on the tensor cores (``bakron_gram``)."""
+    torch = _torch()
+    lib = _lib()
+    _dev_f32(X, "X")
+    N, d = X.shape
+    A = torch.empty((d, d), dtype=torch.float32, device=X.device) if out is None else out
+    if ws is None:
+        ws = workspace(lib.bakron_gram_workspace_size(N, d), X.device)
+    st = _stream(stream)
+    check(lib.bakron_gram(_ptr(X), N, d, float(damping), _ptr(A), _ptr(ws), ws.numel(), st), "bakron_gram")
+    if check_status:
+        check(lib.bakron_get_status(_ptr(ws), ws.numel(), st), "bakron_gram (device)")
+    return A
 
 
 def solve_host_workspace_size(m: int, n: int, gemm: int = 0) -> int:

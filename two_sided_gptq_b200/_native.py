@@ -86,6 +86,8 @@ SIGNATURES = {
     "bakron_version": (ctypes.c_char_p, []),
     "bakron_get_profile": (ctypes.c_int, [ctypes.POINTER(Profile)]),
     "bakron_get_profile_launches": (_i64, [ctypes.POINTER(ProfileLaunch), _i64]),
+    "bakron_gram_workspace_size": (_sz, [_i64, _i64]),
+    "bakron_gram": (ctypes.c_int, [_vp, _i64, _i64, ctypes.c_float, _vp, _vp, _sz, _vp]),
     "bakron_solve_batch": (ctypes.c_int, [ctypes.POINTER(BatchItem), ctypes.c_int32, ctypes.POINTER(Quantizer),
                                           ctypes.POINTER(Config), ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
     "bakron_tune_leaf": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, ctypes.POINTER(Quantizer), _vp, _vp, _vp, _vp, _sz,

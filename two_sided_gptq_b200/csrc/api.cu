@@ -406,6 +406,59 @@ bakron_status_t bakron_solve_batch(const bakron_batch_item_t *items, int32_t cou
     return BAKRON_OK;
 }
 
+namespace {
+struct GramLayout {
+    int64_t Dt, Nt, Dp, Ns;
+    size_t status, xt_hi, xt_lo, G, total;
+    void compute(int64_t N, int64_t d)
+    {
+        Dt = (d + kTile - 1) / kTile; Nt = (N + kTile - 1) / kTile;
+        Dp = Dt * kTile; Ns = Nt * kTile;
+        size_t o = 0;
+        auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+        status = take(kStatusBytes);
+        xt_hi = take((size_t)Dp * Ns * sizeof(float));
+        xt_lo = take((size_t)Dp * Ns * sizeof(float));
+        G = take((size_t)Dp * Dp * sizeof(float));
+        total = o;
+    }
+};
+}  // namespace
+
+size_t bakron_gram_workspace_size(int64_t N, int64_t d)
+{
+    if (N < 1 || d < 1 || N > kMaxSide || d > kMaxSide) return 0;
+    GramLayout L;
+    L.compute(N, d);
+    return L.total;
+}
+
+bakron_status_t bakron_gram(const float *X_dev, int64_t N, int64_t d, float damping, float *A_dev, void *ws_dev,
+                            size_t ws_bytes, bakron_stream_t stream)
+{
+    if (N < 1 || d < 1 || N > kMaxSide || d > kMaxSide) return BAKRON_ERR_INVALID_ARG;
+    if (!X_dev || !A_dev || !(damping >= 0.f) || !isfinite(damping)) return BAKRON_ERR_INVALID_ARG;
+    if (!ws_dev) return BAKRON_ERR_WORKSPACE;
+    if (!aligned16(X_dev) || !aligned16(A_dev) || !aligned16(ws_dev)) return BAKRON_ERR_ALIGNMENT;
+    GramLayout L;
+    L.compute(N, d);
+    if (ws_bytes < L.total) return BAKRON_ERR_WORKSPACE;
+    if (configure_device() != cudaSuccess) return BAKRON_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    char *w = (char *)ws_dev;
+    DeviceStatus *status = (DeviceStatus *)(w + L.status);
+    if (cudaMemsetAsync(status, 0, kStatusBytes, st) != cudaSuccess) return BAKRON_ERR_CUDA;
+    float *xt_hi = (float *)(w + L.xt_hi), *xt_lo = (float *)(w + L.xt_lo), *G = (float *)(w + L.G);
+    if (launch_gram_prep(X_dev, N, d, L.Dp, L.Ns, xt_hi, xt_lo, status, st) != cudaSuccess) return BAKRON_ERR_CUDA;
+    TcMaps maps;
+    if (!make_gram_maps(xt_hi, xt_lo, G, L.Dp, L.Ns, &maps)) return BAKRON_ERR_CUDA;
+    const NodeParams np{0, 0, 0, (int)L.Dt, (int)L.Nt};
+    GemmArgs g{xt_hi, xt_lo, xt_hi, xt_lo, L.Ns, L.Ns, G, nullptr, nullptr, L.Dp, status, 200};
+    if (launch_gram_tc(np, g, maps, st) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (launch_gram_finish(G, d, L.Dp, N, damping, A_dev, st) != cudaSuccess) return BAKRON_ERR_CUDA;
+    return BAKRON_OK;
+}
+
 // Host-buffer variant: staging buffers follow the solve workspace.
 namespace {
 struct HostLayout {

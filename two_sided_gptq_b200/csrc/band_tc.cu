@@ -159,8 +159,9 @@ template <int STAGE>
 __global__ void __launch_bounds__(kThreads, 1)
 band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
 {
-    const Item it = STAGE == 1 ? stage1_item(np, blockIdx.x, blockIdx.y)
-                               : stage2_item(np, blockIdx.x, blockIdx.y);
+    const Item it = STAGE == 1   ? stage1_item(np, blockIdx.x, blockIdx.y)
+                    : STAGE == 2 ? stage2_item(np, blockIdx.x, blockIdx.y)
+                                 : gram_item(np, blockIdx.x, blockIdx.y);
     if (!it.valid) return;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -354,9 +355,12 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
                         split_tf32(acc[col + 3], h.w, l.w);
                         *(float4 *)(wbuf + (2 * cb) * kBoxBytes + off) = h;
                         *(float4 *)(wbuf + (2 * cb + 1) * kBoxBytes + off) = l;
-                    } else {
+                    } else if (STAGE == 2) {
                         *(float4 *)(wbuf + cb * kBoxBytes + off) =
                             make_float4(-acc[col + 0], -acc[col + 1], -acc[col + 2], -acc[col + 3]);
+                    } else {
+                        *(float4 *)(wbuf + cb * kBoxBytes + off) =
+                            make_float4(acc[col + 0], acc[col + 1], acc[col + 2], acc[col + 3]);
                     }
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -367,8 +371,10 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
                 if (STAGE == 1) {
                     tma_store_2d(&maps.o0, x, y, smem_u32(wbuf + (2 * cb) * kBoxBytes));
                     tma_store_2d(&maps.o1, x, y, smem_u32(wbuf + (2 * cb + 1) * kBoxBytes));
-                } else {
+                } else if (STAGE == 2) {
                     tma_add_2d(&maps.o0, x, y, smem_u32(wbuf + cb * kBoxBytes));
+                } else {
+                    tma_store_2d(&maps.o0, x, y, smem_u32(wbuf + cb * kBoxBytes));
                 }
             }
         }
@@ -426,7 +432,22 @@ cudaError_t band_tc_configure()
 {
     cudaError_t e = cudaFuncSetAttribute(band_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(band_tc_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(band_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+}
+
+// Gram products: A = B = X^T hi / lo (Dp x Ns, K-major), output G (Dp x Dp).
+bool make_gram_maps(const float *xt_hi, const float *xt_lo, float *G, int64_t Dp, int64_t Ns, TcMaps *m)
+{
+    return make_map(&m->a_hi, xt_hi, Dp, Ns, Ns) && make_map(&m->a_lo, xt_lo, Dp, Ns, Ns) &&
+           make_map(&m->b_hi, xt_hi, Dp, Ns, Ns) && make_map(&m->b_lo, xt_lo, Dp, Ns, Ns) &&
+           make_map(&m->o0, G, Dp, Dp, Dp, 32) && make_map(&m->o1, G, Dp, Dp, Dp, 32);
+}
+
+cudaError_t launch_gram_tc(const NodeParams &np, const GemmArgs &g, const TcMaps &maps, cudaStream_t stream)
+{
+    return launch_pdl(band_tc_kernel<3>, dim3(np.Mt, np.Mt), dim3(kThreads), kSmem, stream, maps, np, g);
 }
 
 bool make_tc_maps(int stage, int Mt, int Nt, const GemmArgs &g, TcMaps *maps)

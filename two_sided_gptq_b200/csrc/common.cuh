@@ -161,4 +161,12 @@ __host__ __device__ inline Item stage2_item(const NodeParams &p, int x, int Ip)
     return it;
 }
 
+// Gram matrix tile (I, J), J <= I, of G = X^T X: A = B = X^T (rows = features,
+// K = samples); p.Mt = feature tiles, p.Nt = sample tiles.  Grid: x = J, y = I.
+__host__ __device__ inline Item gram_item(const NodeParams &p, int J, int I)
+{
+    Item it{I, J, 0, p.Nt, J <= I && I < p.Mt};
+    return it;
+}
+
 }  // namespace bakron

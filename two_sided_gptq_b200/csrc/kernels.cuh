@@ -52,6 +52,14 @@ bool make_tc_maps(int stage, int Mt, int Nt, const GemmArgs &g, TcMaps *maps);
 cudaError_t launch_band_tc(int stage, const NodeParams &np, const GemmArgs &g, const TcMaps &maps,
                            cudaStream_t stream);
 
+// Gram matrix G = X^T X on the tensor cores (lower tiles), see band_tc.cu.
+bool make_gram_maps(const float *xt_hi, const float *xt_lo, float *G, int64_t Dp, int64_t Ns, TcMaps *m);
+cudaError_t launch_gram_tc(const NodeParams &np, const GemmArgs &g, const TcMaps &maps, cudaStream_t stream);
+cudaError_t launch_gram_prep(const float *X, int64_t N, int64_t d, int64_t Dp, int64_t Ns, float *xt_hi,
+                             float *xt_lo, DeviceStatus *st, cudaStream_t stream);
+cudaError_t launch_gram_finish(const float *G, int64_t d, int64_t Dp, int64_t N, float damping, float *A,
+                               cudaStream_t stream);
+
 // Proxy loss (FP32 products, FP64 reduction) into *out (device double).
 cudaError_t launch_proxy_loss(const float *W, const float *V, const float *A, const float *B,
                               int64_t m, int64_t n, double *out, cudaStream_t stream);
