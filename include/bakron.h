@@ -105,10 +105,20 @@ typedef struct {
                          4 x 4 sub-tiles of 32, each swept by three warps; 4 =
                          2 x 2 sub-tiles of 64, each swept by six warps
                          (bakron_tune_leaf picks one by measurement). */
+    int32_t b_identity; /* 1: B = I (one-sided GPTQ with Hessian A, the case the
+                           two-sided solve reduces to when B = I).  LB_dev may be
+                           NULL and is not read; rows are independent, so the
+                           solve runs over 128-column blocks (the recursion over
+                           column blocks with a one-sided leaf and update)
+                           instead of tile diagonals.  The leaf and gemm
+                           fields are ignored (the update always runs on the
+                           tensor cores, 3xTF32). */
 } bakron_config_t;
 
 /* Per-kernel-class device time of the latest profiled bakron_solve on the
- * calling host thread (sums of CUDA-event intervals around each launch). */
+ * calling host thread (sums of CUDA-event intervals around each launch).  On
+ * the one-sided path (b_identity = 1) the leaf fields count the column-block
+ * leaves and the stage 1 fields the tensor-core updates; stage 2 stays 0. */
 typedef struct {
     double prep_ms, leaf_ms, stage1_ms, stage2_ms, total_ms;
     int64_t prep_launches, leaf_launches, stage1_launches, stage2_launches;
@@ -120,7 +130,9 @@ bakron_status_t bakron_get_profile(bakron_profile_t *out);
  * sweep of tile diagonal k, 2 / 3 stage 1 / stage 2 band product of the
  * recursion node over tile diagonals [k, k+l) split at k+h; ms its
  * CUDA-event interval; flops the algorithmic FLOPs of a band product (2 T^3
- * per 128 x 128 x 128 tile product; 0 for other kinds). */
+ * per 128 x 128 x 128 tile product; 0 for other kinds).  One-sided path:
+ * kind 1 is the leaf of column block k, kind 2 the update of column blocks
+ * [k+h, k+l) by blocks [k, k+h). */
 typedef struct {
     int32_t kind, k, h, l;
     double ms, flops;

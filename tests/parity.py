@@ -49,7 +49,7 @@ def gpu_solve(W, LA32, LB32, bits, gemm=0, row_scale=None, leaf=0):
     dev = "cuda"
     Wd = torch.from_numpy(np.ascontiguousarray(W)).to(dev)
     LAd = torch.from_numpy(np.ascontiguousarray(LA32)).to(dev)
-    LBd = torch.from_numpy(np.ascontiguousarray(LB32)).to(dev)
+    LBd = None if LB32 is None else torch.from_numpy(np.ascontiguousarray(LB32)).to(dev)  # None: B = I
     wt = torch.empty_like(Wd)
     rs = None if row_scale is None else torch.from_numpy(np.asarray(row_scale, np.float32)).to(dev)
     V, codes, scales = bk.solve(Wd, LAd, LBd, bits=bits, gemm=gemm, wt_out=wt, row_scale=rs, leaf=leaf)
@@ -66,7 +66,8 @@ def check_solve(W, LA32, LB32, bits, gemm=0, row_scale=None, label="", leaf=0):
     s = oracle.scales(W, qmax) if row_scale is None else np.asarray(row_scale, np.float32)
     assert np.array_equal(s_gpu.view(np.uint32), s.view(np.uint32)), f"{label}: steps differ"
     LtA = oracle.normalize(LA32.astype(np.float64))
-    LtB = oracle.normalize(LB32.astype(np.float64))
+    # B = I (the one-sided path): the pull with an identity row factor
+    LtB = np.eye(W.shape[0]) if LB32 is None else oracle.normalize(LB32.astype(np.float64))
     r = oracle.forced_check(W, LtA, LtB, s, qmin, qmax, codes, tie_eps=TIE_EPS)
     m, n = W.shape
     r["label"] = label

@@ -85,6 +85,17 @@ def test_argument_errors_return_before_any_device_work(lib):
     a = list(args())
     a[11] = ctypes.byref(cfg)
     assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
+    # b_identity is 0 or 1; LB may be NULL only on the one-sided path
+    cfg = _native.Config(0, 0, 0, 0, None, 0, 0, 2)
+    a[11] = ctypes.byref(cfg)
+    assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
+    a = list(args())
+    a[4] = None
+    assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
+    cfg = _native.Config(0, 0, 0, 0, None, 0, 0, 1)
+    a[11] = ctypes.byref(cfg)
+    a[0] = fake + 4  # with LB = NULL accepted, validation goes on to the next check
+    assert lib.bakron_solve(*a) == _native.Status.ERR_ALIGNMENT
     assert lib.bakron_factor(fake, -1, fake, 4, fake, fake, fake, 1 << 30, None) == _native.Status.ERR_INVALID_ARG
     assert lib.bakron_factor(fake, 4, fake, 4, fake + 8, fake, fake, 1 << 30, None) == _native.Status.ERR_ALIGNMENT
     assert lib.bakron_factor(fake, 4, fake, 4, fake, fake, fake, 16, None) == _native.Status.ERR_WORKSPACE

@@ -59,8 +59,9 @@ def _dev_f32(x, name):
     return x
 
 
-def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False, leaf=0):
-    return Config(0, int(gemm), 0, int(timeout_ms), _ptr(wt_out), 1 if profile else 0, int(leaf))
+def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False, leaf=0, b_identity=False):
+    return Config(0, int(gemm), 0, int(timeout_ms), _ptr(wt_out), 1 if profile else 0, int(leaf),
+                  1 if b_identity else 0)
 
 
 def workspace(nbytes: int, device=None):
@@ -105,6 +106,9 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
           wt_out=None, check_status=True, timeout_ms=0, profile=False, leaf=0, shrink_grid=0):
     """BaKron solve on device tensors.  Returns ``(V, codes, scales)``.
 
+    ``LB=None`` selects the one-sided path (B = I: GPTQ with Hessian A, over
+    128-column blocks).
+
     ``gemm=0`` uses the tcgen05 3xTF32 band products, ``gemm=1`` the FP32
     CUDA-core ones; ``shrink_grid`` > 1 searches each row's step for the least
     round-to-nearest error over that many shrink factors in [1/2, 1]; ``leaf``
@@ -117,11 +121,14 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     """
     torch = _torch()
     lib = _lib()
-    _dev_f32(W, "W"), _dev_f32(LA, "LA"), _dev_f32(LB, "LB")
+    one_sided = LB is None
+    _dev_f32(W, "W"), _dev_f32(LA, "LA")
+    if not one_sided:
+        _dev_f32(LB, "LB")
     m, n = W.shape
-    if LA.shape != (n, n) or LB.shape != (m, m):
+    if LA.shape != (n, n) or (not one_sided and LB.shape != (m, m)):
         raise ValueError("LA must be n x n and LB m x m")
-    cfg = _config(gemm, timeout_ms, wt_out, profile, leaf)
+    cfg = _config(gemm, timeout_ms, wt_out, profile, leaf, one_sided)
     if out is None:
         V = torch.empty((m, n), dtype=torch.float32, device=W.device)
         codes = torch.empty((m, n), dtype=torch.int8, device=W.device)
@@ -234,12 +241,14 @@ def solve_host(W, LA, LB, bits=4, *, V=None, codes=None, scales=None, gemm=0, ws
     lib = _lib()
     m, n = W.shape
     for t, name in ((W, "W"), (LA, "LA"), (LB, "LB")):
+        if t is None and name == "LB":
+            continue  # B = I: the one-sided path
         if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
             raise TypeError(f"{name} must be a contiguous float32 CPU tensor")
     V = torch.empty((m, n), dtype=torch.float32, pin_memory=True) if V is None else V
     codes = torch.empty((m, n), dtype=torch.int8, pin_memory=True) if codes is None else codes
     scales = torch.empty((m,), dtype=torch.float32, pin_memory=True) if scales is None else scales
-    cfg = _config(gemm, leaf=leaf)
+    cfg = _config(gemm, leaf=leaf, b_identity=int(LB is None))
     if ws is None:
         ws = workspace(lib.bakron_solve_host_workspace_size(m, n, ctypes.byref(cfg)))
     q = Quantizer(int(bits), 0, 0, 0)

@@ -45,7 +45,7 @@ class BatchItem(ctypes.Structure):
 class Config(ctypes.Structure):
     _fields_ = [("tile", ctypes.c_int32), ("gemm", ctypes.c_int32), ("use_graph", ctypes.c_int32),
                 ("timeout_ms", ctypes.c_int32), ("wt_out", ctypes.c_void_p), ("profile", ctypes.c_int32),
-                ("leaf", ctypes.c_int32)]
+                ("leaf", ctypes.c_int32), ("b_identity", ctypes.c_int32)]
 
 
 class Profile(ctypes.Structure):

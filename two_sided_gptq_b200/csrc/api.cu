@@ -31,7 +31,7 @@ constexpr const char *kVersion = "bakron-b200 0.1";
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 struct Config {
-    int tile = kTile, gemm = 0, use_graph = 0, timeout_ms = 200, profile = 0, leaf = 2;
+    int tile = kTile, gemm = 0, use_graph = 0, timeout_ms = 200, profile = 0, leaf = 2, b_identity = 0;
     float *wt_out = nullptr;
 };
 
@@ -87,6 +87,19 @@ double node_stage_flops(const NodeParams &np, int stage)
     return f;
 }
 
+// Algorithmic FLOPs of one node of the one-sided recursion over column blocks.
+double gptq_node_flops(const NodeParams &np)
+{
+    const double t3 = 2.0 * kTile * (double)kTile * kTile;
+    double f = 0.0;
+    for (int I = 0; I < np.Mt; ++I)
+        for (int x = 0; x < np.l - np.h; ++x) {
+            Item it = gptq_item(np, x, I);
+            if (it.valid) f += t3 * (it.k1 - it.k0);
+        }
+    return f;
+}
+
 bakron_status_t read_config(const bakron_config_t *c, Config &out)
 {
     out = Config();
@@ -101,6 +114,8 @@ bakron_status_t read_config(const bakron_config_t *c, Config &out)
     out.profile = c->profile ? 1 : 0;
     if (c->leaf < 0 || c->leaf > 4) return BAKRON_ERR_INVALID_ARG;
     if (c->leaf != 0) out.leaf = c->leaf - 1;  // 0 keeps the default
+    if (c->b_identity < 0 || c->b_identity > 1) return BAKRON_ERR_INVALID_ARG;
+    out.b_identity = c->b_identity;
     return BAKRON_OK;
 }
 
@@ -136,6 +151,7 @@ cudaError_t configure_device()
     std::lock_guard<std::mutex> lk(g_cfg_mu);
     if (dev >= 0 && dev < 64 && g_configured[dev]) return cudaSuccess;
     if ((e = leaf_configure()) != cudaSuccess) return e;
+    if ((e = leaf_gptq_configure()) != cudaSuccess) return e;
     if ((e = band_tc_configure()) != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) g_configured[dev] = true;
     return cudaSuccess;
@@ -176,20 +192,42 @@ cudaError_t run_schedule(const SolveCtx &c, int k, int l)
     return run_schedule(c, k + h, l - h);
 }
 
+// One-sided path: midpoint recursion over the column blocks [k, k+l); a leaf
+// rounds one 128-column block, a node updates its right half from its left.
+cudaError_t run_schedule_gptq(SolveCtx &c, const TcMaps &maps, int k, int l)
+{
+    if (l <= 1) {
+        t_prof.begin(1, NodeParams{k, 0, 1, c.leaf.Mt, c.leaf.Nt});
+        cudaError_t e = launch_leaf_gptq(c.leaf, k, c.stream);
+        t_prof.end();
+        return e;
+    }
+    const int h = l / 2;
+    cudaError_t e = run_schedule_gptq(c, maps, k, h);
+    if (e != cudaSuccess) return e;
+    NodeParams np{k, h, l, c.leaf.Mt, c.leaf.Nt};
+    t_prof.begin(2, np);
+    e = launch_gptq_tc(np, c.s1, maps, c.stream);
+    t_prof.end();
+    if (e != cudaSuccess) return e;
+    return run_schedule_gptq(c, maps, k + h, l - h);
+}
+
 bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *LA, const float *LB,
                              const bakron_quantizer_t *q, float *V, int8_t *codes, float *scales,
                              void *ws, size_t ws_bytes, const bakron_config_t *cfg,
                              cudaStream_t stream, bool user_scales_on_device)
 {
     if (m < 1 || n < 1 || m > kMaxSide || n > kMaxSide) return BAKRON_ERR_INVALID_ARG;
-    if (!W || !LA || !LB || !V || !codes || !scales) return BAKRON_ERR_INVALID_ARG;
-    if (!ws) return BAKRON_ERR_WORKSPACE;
-    if (!aligned16(W) || !aligned16(LA) || !aligned16(LB) || !aligned16(V) || !aligned16(codes) ||
-        !aligned16(scales) || !aligned16(ws))
-        return BAKRON_ERR_ALIGNMENT;
     Config conf;
     bakron_status_t s = read_config(cfg, conf);
     if (s != BAKRON_OK) return s;
+    if (conf.b_identity) LB = nullptr;  // not read on the one-sided path
+    if (!W || !LA || (!LB && !conf.b_identity) || !V || !codes || !scales) return BAKRON_ERR_INVALID_ARG;
+    if (!ws) return BAKRON_ERR_WORKSPACE;
+    if (!aligned16(W) || !aligned16(LA) || (LB && !aligned16(LB)) || !aligned16(V) || !aligned16(codes) ||
+        !aligned16(scales) || !aligned16(ws))
+        return BAKRON_ERR_ALIGNMENT;
     if (conf.wt_out && !aligned16(conf.wt_out)) return BAKRON_ERR_ALIGNMENT;
     int qmin = 0, qmax = 0;
     if ((s = read_grid(q, qmin, qmax)) != BAKRON_OK) return s;
@@ -238,11 +276,21 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
     c.s2 = GemmArgs{(const float *)(w + L.LBhi), (const float *)(w + L.LBlo),
                     (const float *)(w + L.XThi), (const float *)(w + L.XTlo), L.Mp, L.Mp,
                     nullptr, nullptr, (float *)(w + L.Wt), L.Np, st, conf.timeout_ms};
-    if (c.gemm == 0 && (!make_tc_maps(1, c.leaf.Mt, c.leaf.Nt, c.s1, &c.m1) ||
-                        !make_tc_maps(2, c.leaf.Mt, c.leaf.Nt, c.s2, &c.m2)))
-        return BAKRON_ERR_CUDA;
-    const int keys = (int)(L.Mt + L.Nt - 1);
-    if (run_schedule(c, 0, keys) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (conf.b_identity) {
+        // one-sided update: Wt (Mp x Np) -= Delta (Mp x Np) . LtA (Np x Np)^T over column blocks
+        c.s1 = GemmArgs{(const float *)(w + L.Dhi), (const float *)(w + L.Dlo), (const float *)(w + L.LAhi),
+                        (const float *)(w + L.LAlo), L.Np, L.Np, nullptr, nullptr, (float *)(w + L.Wt), L.Np, st,
+                        conf.timeout_ms};
+        TcMaps gm;
+        if (!make_gptq_maps(c.s1, L.Mp, L.Np, &gm)) return BAKRON_ERR_CUDA;
+        if (run_schedule_gptq(c, gm, 0, (int)L.Nt) != cudaSuccess) return BAKRON_ERR_CUDA;
+    } else {
+        if (c.gemm == 0 && (!make_tc_maps(1, c.leaf.Mt, c.leaf.Nt, c.s1, &c.m1) ||
+                            !make_tc_maps(2, c.leaf.Mt, c.leaf.Nt, c.s2, &c.m2)))
+            return BAKRON_ERR_CUDA;
+        const int keys = (int)(L.Mt + L.Nt - 1);
+        if (run_schedule(c, 0, keys) != cudaSuccess) return BAKRON_ERR_CUDA;
+    }
     if (t_prof.on) {
         t_prof.on = false;
         if (cudaStreamSynchronize(stream) != cudaSuccess) return BAKRON_ERR_CUDA;
@@ -263,7 +311,7 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
             r.h = np.h;
             r.l = np.l;
             r.ms = dt;
-            r.flops = kind >= 2 ? node_stage_flops(np, kind - 1) : 0.0;
+            r.flops = kind < 2 ? 0.0 : conf.b_identity ? gptq_node_flops(np) : node_stage_flops(np, kind - 1);
             t_last_launches.push_back(r);
         }
         pr.prep_launches *= 4;  // scales, padded copy, two factor normalisations
@@ -491,7 +539,8 @@ bakron_status_t bakron_solve_host(const float *W_host, int64_t m, int64_t n, con
                                   size_t ws_bytes, const bakron_config_t *cfg,
                                   bakron_stream_t stream)
 {
-    if (!W_host || !LA_host || !LB_host || !V_host || !codes_host || !scales_host || !q)
+    const bool one_sided = cfg && cfg->b_identity == 1;
+    if (!W_host || !LA_host || (!LB_host && !one_sided) || !V_host || !codes_host || !scales_host || !q)
         return BAKRON_ERR_INVALID_ARG;
     size_t sb = bakron_solve_workspace_size(m, n, cfg);
     if (!sb) return BAKRON_ERR_INVALID_ARG;
@@ -506,7 +555,7 @@ bakron_status_t bakron_solve_host(const float *W_host, int64_t m, int64_t n, con
         return cudaMemcpyAsync(w + off, src, bytes, cudaMemcpyHostToDevice, s) == cudaSuccess;
     };
     if (!h2d(H.W, W_host, (size_t)m * n * 4) || !h2d(H.LA, LA_host, (size_t)n * n * 4) ||
-        !h2d(H.LB, LB_host, (size_t)m * m * 4))
+        (!one_sided && !h2d(H.LB, LB_host, (size_t)m * m * 4)))
         return BAKRON_ERR_CUDA;
     bakron_quantizer_t qd = *q;
     if (q->row_scale) {

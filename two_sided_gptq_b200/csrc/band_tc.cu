@@ -159,9 +159,11 @@ template <int STAGE>
 __global__ void __launch_bounds__(kThreads, 1)
 band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
 {
+    // STAGE 1, 2: the band products; 3: Gram tiles; 4: the one-sided update
     const Item it = STAGE == 1   ? stage1_item(np, blockIdx.x, blockIdx.y)
                     : STAGE == 2 ? stage2_item(np, blockIdx.x, blockIdx.y)
-                                 : gram_item(np, blockIdx.x, blockIdx.y);
+                    : STAGE == 3 ? gram_item(np, blockIdx.x, blockIdx.y)
+                                 : gptq_item(np, blockIdx.x, blockIdx.y);
     if (!it.valid) return;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -208,13 +210,17 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
     if (threadIdx.x == 0) {
-        // The A operand is a normalised factor, written by the preparation
-        // kernels long before: warm L2 with its first boxes while the previous
-        // kernel finishes (a prefetch is only a hint).
+        // The factor operand (A in the band products and the Gram, B in the
+        // one-sided update) was written by the preparation kernels long
+        // before: warm L2 with its first boxes while the previous kernel
+        // finishes (a prefetch is only a hint).
+        const CUtensorMap *f_hi = STAGE == 4 ? &maps.b_hi : &maps.a_hi;
+        const CUtensorMap *f_lo = STAGE == 4 ? &maps.b_lo : &maps.a_lo;
+        const int f_row = (STAGE == 4 ? it.rb : it.ra) * T;
         const int nk_pre = min((it.k1 - it.k0) * (T / KB), 8);
         for (int kb = 0; kb < nk_pre; ++kb) {
-            tma_prefetch_2d(&maps.a_hi, it.k0 * T + kb * KB, it.ra * T);
-            tma_prefetch_2d(&maps.a_lo, it.k0 * T + kb * KB, it.ra * T);
+            tma_prefetch_2d(f_hi, it.k0 * T + kb * KB, f_row);
+            tma_prefetch_2d(f_lo, it.k0 * T + kb * KB, f_row);
         }
     }
     pdl_wait();  // operands and the output tile were written by earlier kernels
@@ -355,7 +361,7 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
                         split_tf32(acc[col + 3], h.w, l.w);
                         *(float4 *)(wbuf + (2 * cb) * kBoxBytes + off) = h;
                         *(float4 *)(wbuf + (2 * cb + 1) * kBoxBytes + off) = l;
-                    } else if (STAGE == 2) {
+                    } else if (STAGE == 2 || STAGE == 4) {
                         *(float4 *)(wbuf + cb * kBoxBytes + off) =
                             make_float4(-acc[col + 0], -acc[col + 1], -acc[col + 2], -acc[col + 3]);
                     } else {
@@ -371,7 +377,7 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
                 if (STAGE == 1) {
                     tma_store_2d(&maps.o0, x, y, smem_u32(wbuf + (2 * cb) * kBoxBytes));
                     tma_store_2d(&maps.o1, x, y, smem_u32(wbuf + (2 * cb + 1) * kBoxBytes));
-                } else if (STAGE == 2) {
+                } else if (STAGE == 2 || STAGE == 4) {
                     tma_add_2d(&maps.o0, x, y, smem_u32(wbuf + cb * kBoxBytes));
                 } else {
                     tma_store_2d(&maps.o0, x, y, smem_u32(wbuf + cb * kBoxBytes));
@@ -434,6 +440,8 @@ cudaError_t band_tc_configure()
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(band_tc_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(band_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(band_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
 }
 
@@ -443,6 +451,20 @@ bool make_gram_maps(const float *xt_hi, const float *xt_lo, float *G, int64_t Dp
     return make_map(&m->a_hi, xt_hi, Dp, Ns, Ns) && make_map(&m->a_lo, xt_lo, Dp, Ns, Ns) &&
            make_map(&m->b_hi, xt_hi, Dp, Ns, Ns) && make_map(&m->b_lo, xt_lo, Dp, Ns, Ns) &&
            make_map(&m->o0, G, Dp, Dp, Dp, 32) && make_map(&m->o1, G, Dp, Dp, Dp, 32);
+}
+
+// One-sided update: A = Delta hi / lo (Mp x Np), B = LtA hi / lo (Np x Np),
+// output Wt (Mp x Np, add-reduction of -D).
+bool make_gptq_maps(const GemmArgs &g, int64_t Mp, int64_t Np, TcMaps *m)
+{
+    return make_map(&m->a_hi, g.Ahi, Mp, Np, Np) && make_map(&m->a_lo, g.Alo, Mp, Np, Np) &&
+           make_map(&m->b_hi, g.Bhi, Np, Np, Np) && make_map(&m->b_lo, g.Blo, Np, Np, Np) &&
+           make_map(&m->o0, g.out_acc, Mp, Np, Np, 32) && make_map(&m->o1, g.out_acc, Mp, Np, Np, 32);
+}
+
+cudaError_t launch_gptq_tc(const NodeParams &np, const GemmArgs &g, const TcMaps &maps, cudaStream_t stream)
+{
+    return launch_pdl(band_tc_kernel<4>, dim3(np.l - np.h, np.Mt), dim3(kThreads), kSmem, stream, maps, np, g);
 }
 
 cudaError_t launch_gram_tc(const NodeParams &np, const GemmArgs &g, const TcMaps &maps, cudaStream_t stream)

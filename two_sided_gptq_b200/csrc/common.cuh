@@ -161,6 +161,18 @@ __host__ __device__ inline Item stage2_item(const NodeParams &p, int x, int Ip)
     return it;
 }
 
+// One-sided (B = I) update of node p over 128-column blocks: target tile
+// (I, J') with J' in [k+h, k+l) loses sum_{J in [k, k+h)} Delta[I, J] LtA[J', J]^T.
+// Grid: x = J' - (k+h), y = I.
+__host__ __device__ inline Item gptq_item(const NodeParams &p, int x, int I)
+{
+    Item it{0, 0, 0, 0, false};
+    const int Jp = p.k + p.h + x;
+    if (Jp >= p.Nt || I >= p.Mt) return it;
+    it.ra = I; it.rb = Jp; it.k0 = p.k; it.k1 = min(p.k + p.h, p.Nt); it.valid = it.k0 < it.k1;
+    return it;
+}
+
 // Gram matrix tile (I, J), J <= I, of G = X^T X: A = B = X^T (rows = features,
 // K = samples); p.Mt = feature tiles, p.Nt = sample tiles.  Grid: x = J, y = I.
 __host__ __device__ inline Item gram_item(const NodeParams &p, int J, int I)

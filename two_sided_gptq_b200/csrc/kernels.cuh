@@ -52,6 +52,12 @@ bool make_tc_maps(int stage, int Mt, int Nt, const GemmArgs &g, TcMaps *maps);
 cudaError_t launch_band_tc(int stage, const NodeParams &np, const GemmArgs &g, const TcMaps &maps,
                            cudaStream_t stream);
 
+// One-sided (B = I) path: the leaf over a 128-column block and the update.
+cudaError_t leaf_gptq_configure();
+cudaError_t launch_leaf_gptq(const LeafArgs &p, int Jb, cudaStream_t stream);
+bool make_gptq_maps(const GemmArgs &g, int64_t Mp, int64_t Np, TcMaps *m);
+cudaError_t launch_gptq_tc(const NodeParams &np, const GemmArgs &g, const TcMaps &maps, cudaStream_t stream);
+
 // Gram matrix G = X^T X on the tensor cores (lower tiles), see band_tc.cu.
 bool make_gram_maps(const float *xt_hi, const float *xt_lo, float *G, int64_t Dp, int64_t Ns, TcMaps *m);
 cudaError_t launch_gram_tc(const NodeParams &np, const GemmArgs &g, const TcMaps &maps, cudaStream_t stream);

@@ -218,6 +218,7 @@ cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, c
                         L.Np, (float *)(ws + L.LA32), (float *)(ws + L.LAhi), (float *)(ws + L.LAlo), st)) !=
         cudaSuccess)
         return e;
+    if (!LB) return cudaSuccess;  // the one-sided path (B = I) has no output-side factor
     return launch_pdl(normalize_split_kernel, dim3(grid_for(L.Mp * L.Mp, 256)), dim3(256), 0, stream, LB, m, L.Mp,
                       (float *)(ws + L.LB32), (float *)(ws + L.LBhi), (float *)(ws + L.LBlo), st);
 }
