@@ -416,6 +416,22 @@ def main():
     assert torch.equal(bouts[-1][1], codes), "batched solve disagrees with the single solve"
     del bws, bouts
 
+    # the one-sided path (B = I: GPTQ with Hessian A) on the same W and A
+    o_out = (torch.empty_like(Wd), torch.empty((m, n), dtype=torch.int8, device=dev),
+             torch.empty((m,), dtype=torch.float32, device=dev))
+    for _ in range(2):
+        bk.solve(Wd, LA, None, bits=w.bits, ws=ws, out=o_out, stream=stream)
+    torch.cuda.synchronize()
+    o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    o_steps = 5
+    o0.record(stream)
+    for _ in range(o_steps):
+        bk.solve(Wd, LA, None, bits=w.bits, ws=ws, out=o_out, stream=stream, check_status=False)
+    o1.record(stream)
+    torch.cuda.synchronize()
+    one_ms = max_over_ranks(o0.elapsed_time(o1) / o_steps, dist, dev)
+    del o_out
+
     line = None
     if rank == 0:
         cb = None
@@ -453,6 +469,9 @@ def main():
             "batch": {"matrices_per_step": n_batch, "streams": n_batch, "ms_per_step": batch_ms,
                       "value": aggregate_rate(world, m, n, batch_ms / n_batch), "unit": "weights/s",
                       "note": "bakron_solve_batch of the same workload on separate streams (not the headline)"},
+            "one_sided": {"ms_per_step": one_ms, "value": aggregate_rate(world, m, n, one_ms), "unit": "weights/s",
+                          "note": "B = I path (one-sided GPTQ with Hessian A, column-block recursion) on the same "
+                                  "W and A (not the headline)"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "device_status": status.name,
