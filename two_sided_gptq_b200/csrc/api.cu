@@ -268,7 +268,6 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
     c.leaf.qmin = qmin; c.leaf.qmax = qmax;
     c.leaf.st = st;
     c.leaf.wt_out = conf.wt_out;
-    c.leaf.LAdT = (const float *)(w + L.XThi);  // written by the preparation on the one-sided path only
     // stage 1: X^T (Np x Mp) = LtA (Np x Np) . Delta (Mp x Np)^T over tile columns
     c.s1 = GemmArgs{(const float *)(w + L.LAhi), (const float *)(w + L.LAlo),
                     (const float *)(w + L.Dhi), (const float *)(w + L.Dlo), L.Np, L.Np,
@@ -315,7 +314,7 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
             r.flops = kind < 2 ? 0.0 : conf.b_identity ? gptq_node_flops(np) : node_stage_flops(np, kind - 1);
             t_last_launches.push_back(r);
         }
-        pr.prep_launches *= 4;  // scales, padded copy, two factor normalisations (one-sided: one, plus its diagonal blocks)
+        pr.prep_launches *= conf.b_identity ? 3 : 4;  // scales, padded copy, the factor normalisations
         float tot = 0.f;
         if (t_prof.used >= 2) cudaEventElapsedTime(&tot, t_prof.pool[0], t_prof.pool[t_prof.used - 1]);
         pr.total_ms = tot;

@@ -15,7 +15,6 @@ struct LeafArgs {
     int Mt, Nt, qmin, qmax;
     DeviceStatus *st;
     float *wt_out;  // optional m x n pre-rounding values
-    const float *LAdT;  // one-sided path: Nt blocks of 128 x 128, block J row j = LtA[128J + 0..127, 128J + j]
 };
 
 // Operands of the band products.  Stage 1: A = LtA (Np x Np), B = Delta

@@ -4,26 +4,31 @@
 // solve reduces to one-sided GPTQ when B = I).  The recursion then runs over
 // 128-column blocks; this kernel rounds one block.
 //
-// One warp per 32 rows, lane = row.  The row's 128 block entries live in
-// registers; the block is rounded column by column in two halves of 64 in
-// GPTQ's push form: after rounding column j, every later column j' of the
-// half loses Delta_j LtA[j', j], and after the first half its 64 residuals are
-// pushed into the second half.  The coefficients come from the block's
-// transposed copy (prepared once per solve), so the ones a column pushes are
-// contiguous: one asynchronous 64 KB copy into shared memory, then 16-byte
-// broadcast reads.  Codes, V and the residual's TF32 split are staged in
-// shared memory and written row-coalesced at the end.
+// One warp per 32 rows, lane = row.  The block is rounded in column order in
+// steps of 8 columns, in the pull form
+//     Wt_j = W_j - sum_{j' < j} Delta_j' LtA[j, j'] :
+// for the next 8 columns, the terms of all earlier columns of the block come
+// from one loop over 4-column chunks (16-byte reads of the lane's own residuals
+// and broadcast reads of the 8 factor rows, 8 independent sums), then the 8
+// columns are rounded in order with the terms among themselves applied as
+// each residual appears.  Every code path is a short loop, so the kernel runs
+// from the instruction cache; W and the residuals share one row per lane in
+// shared memory (a column's W is replaced by its residual).  Codes, V and the
+// residual's TF32 split are staged in shared memory and written row-coalesced
+// at the end.
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace bakron {
 
 namespace {
-constexpr int GB = 128;        // column block
-constexpr int GH = 64;         // half block
-constexpr int LDL = GB + 4;    // row stride of the transposed diagonal block in smem (16-byte rows)
-constexpr int LDO = GB + 1;    // row stride of the staged outputs (odd: a lane per row hits its own bank)
-constexpr size_t kSmemGptq = ((size_t)GB * LDL + 2 * 32 * LDO + 32) * sizeof(float) + (size_t)32 * LDO + 32;
+constexpr int GB = 128;      // column block
+constexpr int GS = 8;        // columns per step
+constexpr int LDL = GB + 4;  // row stride of the LtA diagonal block in smem (16-byte rows)
+constexpr int LDX = GB + 4;  // row stride of the W / residual rows (16-byte rows; 8 lanes cover the banks)
+constexpr int LDO = GB + 1;  // row stride of the staged V and codes (odd: a lane per row hits its own bank)
+constexpr size_t kSmemGptq =
+    ((size_t)GB * LDL + (size_t)32 * LDX + (size_t)32 * LDO) * sizeof(float) + (size_t)32 * LDO + 32;
 static_assert(kSmemGptq <= 232448, "one-sided leaf shared memory");
 
 __device__ __forceinline__ void cp_async16_g(float *dst, const float *src)
@@ -33,47 +38,64 @@ __device__ __forceinline__ void cp_async16_g(float *dst, const float *src)
                  : "memory");
 }
 
-// w[C0 + jj] -= d * LtA[C0 + jj, C0 + j] for jj in (j, 64): the coefficients
-// are row C0 + j of the transposed block, read four at a time.  Called with j
-// a constant (inside fully unrolled loops), so every bound folds away.
-template <int C0>
-__device__ __forceinline__ void push_half(float (&w)[GB], const float *crow, float d, int j)
-{
-#pragma unroll
-    for (int g = 0; g < GH / 4; ++g) {
-        if (4 * g + 3 > j) {
-            const float4 c = *(const float4 *)(crow + C0 + 4 * g);
-            const float cc[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                if (4 * g + e > j) w[C0 + 4 * g + e] = fmaf(-d, cc[e], w[C0 + 4 * g + e]);
-        }
-    }
-}
-
 __device__ __forceinline__ int8_t code_byte1(float c)
 {
     return (int8_t)(__float_as_int(c + 12582912.0f) & 0xFF);
 }
 
-// Round the 64 columns [c0, c0 + 64) of the lane's row: push form inside the
-// half; residual, V and code of each column go to the staging rows (columns
-// at or beyond n are zero padding: their value, code and residual are 0).
-template <bool IEEE, int C0>
-__device__ __forceinline__ void gptq_half(float (&w)[GB], const float *sLA, float s, float rs, float fqmin,
-                                          float fqmax, float *dD, float *dV, int8_t *dC, int ncols, float *wt_row)
+// Round the block's columns in steps of GS; x = the lane's row (W, replaced
+// column by column by the residual), sLA = the factor's diagonal block.
+template <bool IEEE>
+__device__ __forceinline__ void gptq_block(float *x, const float *sLA, float s, float rs, float fqmin, float fqmax,
+                                           float *dV, int8_t *dC, int ncols, float *wt_row)
 {
+    const float4 *x4 = (const float4 *)x;
+#pragma unroll 1
+    for (int c0 = 0; c0 < GB; c0 += GS) {
+        // terms of the columns before c0
+        float acc[GS];
 #pragma unroll
-    for (int j = 0; j < GH; ++j) {
-        const float wt = w[C0 + j];
-        const float qf = IEEE ? __fdiv_rn(wt, s) : div_rn_recip(wt, s, rs);
-        const float cq = fminf(fmaxf(rintf(qf), fqmin), fqmax);
-        const float d = fmaf(-s, cq, wt);
-        push_half<C0>(w, sLA + (C0 + j) * LDL, d, j);
-        dD[C0 + j] = d;
-        dV[C0 + j] = s * cq;
-        dC[C0 + j] = code_byte1(cq);
-        if (wt_row && C0 + j < ncols) wt_row[C0 + j] = wt;
+        for (int r = 0; r < GS; ++r) acc[r] = 0.f;
+#pragma unroll 2
+        for (int g = 0; g < c0 / 4; ++g) {
+            const float4 dv = x4[g];
+#pragma unroll
+            for (int r = 0; r < GS; ++r) {
+                const float4 c = *(const float4 *)(sLA + (c0 + r) * LDL + 4 * g);
+                acc[r] = fmaf(dv.x, c.x, acc[r]);
+                acc[r] = fmaf(dv.y, c.y, acc[r]);
+                acc[r] = fmaf(dv.z, c.z, acc[r]);
+                acc[r] = fmaf(dv.w, c.w, acc[r]);
+            }
+        }
+        // the step's own columns, in order
+        float w[GS];
+#pragma unroll
+        for (int q = 0; q < GS / 4; ++q) {
+            const float4 v = x4[c0 / 4 + q];
+            w[4 * q] = v.x - acc[4 * q];
+            w[4 * q + 1] = v.y - acc[4 * q + 1];
+            w[4 * q + 2] = v.z - acc[4 * q + 2];
+            w[4 * q + 3] = v.w - acc[4 * q + 3];
+        }
+        float cf[GS][GS];  // cf[r][r2] = LtA[c0 + r, c0 + r2], r2 < r
+#pragma unroll
+        for (int r = 1; r < GS; ++r)
+#pragma unroll
+            for (int r2 = 0; r2 < r; ++r2) cf[r][r2] = sLA[(c0 + r) * LDL + c0 + r2];
+#pragma unroll
+        for (int r = 0; r < GS; ++r) {
+            const float wt = w[r];
+            const float qf = IEEE ? __fdiv_rn(wt, s) : div_rn_recip(wt, s, rs);
+            const float cq = fminf(fmaxf(rintf(qf), fqmin), fqmax);
+            const float d = fmaf(-s, cq, wt);
+#pragma unroll
+            for (int r2 = r + 1; r2 < GS; ++r2) w[r2] = fmaf(-d, cf[r2][r], w[r2]);
+            x[c0 + r] = d;
+            dV[c0 + r] = s * cq;
+            dC[c0 + r] = code_byte1(cq);
+            if (wt_row && c0 + r < ncols) wt_row[c0 + r] = wt;
+        }
     }
 }
 }  // namespace
@@ -81,58 +103,37 @@ __device__ __forceinline__ void gptq_half(float (&w)[GB], const float *sLA, floa
 __global__ void __launch_bounds__(32, 1) leaf_gptq_kernel(LeafArgs p, int Jb)
 {
     extern __shared__ __align__(16) float smem_g[];
-    float *sLA = smem_g;                     // GB x LDL: row j = LtA[col0 + 0..127, col0 + j]
-    float *sD = sLA + GB * LDL;              // 32 x LDO: residuals of the warp's rows
-    float *sV = sD + 32 * LDO;               // 32 x LDO: V
-    float *sWt = sV + 32 * LDO;              // 32 floats spare (alignment)
-    int8_t *sC = (int8_t *)(sWt + 32);       // 32 x LDO: codes
+    float *sLA = smem_g;          // GB x LDL: LtA[col0 + j, col0 + 0..127] in row j
+    float *sX = sLA + GB * LDL;   // 32 x LDX: the lanes' rows of W, then of the residuals
+    float *sV = sX + 32 * LDX;    // 32 x LDO: V
+    int8_t *sC = (int8_t *)(sV + 32 * LDO);  // 32 x LDO: codes
     const int lane = threadIdx.x;
     const int64_t row = (int64_t)blockIdx.x * 32 + lane;
     const int64_t col0 = (int64_t)Jb * GB;
-    const float *LAt = p.LAdT + col0 * GB;  // transposed diagonal block Jb, contiguous
-    pdl_wait();
-#pragma unroll 8
-    for (int r = 0; r < GB; ++r) cp_async16_g(sLA + r * LDL + 4 * lane, LAt + r * GB + 4 * lane);
-    asm volatile("cp.async.commit_group;" ::: "memory");
     const bool live = row < p.m;
     const int64_t rowc = live ? row : p.m - 1;
-    float w[GB];
-#pragma unroll
-    for (int c4 = 0; c4 < GB / 4; ++c4) {
-        const float4 v = *(const float4 *)(p.Wt + rowc * p.Np + col0 + 4 * c4);
-        w[4 * c4] = v.x; w[4 * c4 + 1] = v.y; w[4 * c4 + 2] = v.z; w[4 * c4 + 3] = v.w;
-    }
+    const float *LAt = p.LA32 + col0 * p.Np + col0;
+    pdl_wait();
+    // the factor's diagonal block (rows coalesced) and the lane's row of Wt
+#pragma unroll 8
+    for (int r = 0; r < GB; ++r) cp_async16_g(sLA + r * LDL + 4 * lane, LAt + (int64_t)r * p.Np + 4 * lane);
+    float *x = sX + lane * LDX;
+#pragma unroll 8
+    for (int c4 = 0; c4 < GB / 4; ++c4) cp_async16_g(x + 4 * c4, p.Wt + rowc * p.Np + col0 + 4 * c4);
+    asm volatile("cp.async.commit_group;" ::: "memory");
     const float s = p.scales[rowc], rs = __frcp_rn(s);
     const bool ieee = __any_sync(0xffffffffu, !(s >= 0x1p-60f && s <= 0x1p60f));
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncwarp();
     const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
-    float *dD = sD + lane * LDO, *dV = sV + lane * LDO;
+    float *dV = sV + lane * LDO;
     int8_t *dC = sC + lane * LDO;
     float *wt_row = p.wt_out && live ? p.wt_out + row * p.n + col0 : nullptr;
     const int ncols = (int)min64(GB, p.n - col0);
     if (ieee)
-        gptq_half<true, 0>(w, sLA, s, rs, fqmin, fqmax, dD, dV, dC, ncols, wt_row);
+        gptq_block<true>(x, sLA, s, rs, fqmin, fqmax, dV, dC, ncols, wt_row);
     else
-        gptq_half<false, 0>(w, sLA, s, rs, fqmin, fqmax, dD, dV, dC, ncols, wt_row);
-    // the first half's residuals reach the second half
-#pragma unroll 2
-    for (int j = 0; j < GH; ++j) {
-        const float d = dD[j];
-        const float *crow = sLA + j * LDL + GH;
-#pragma unroll
-        for (int g = 0; g < GH / 4; ++g) {
-            const float4 c = *(const float4 *)(crow + 4 * g);
-            w[GH + 4 * g] = fmaf(-d, c.x, w[GH + 4 * g]);
-            w[GH + 4 * g + 1] = fmaf(-d, c.y, w[GH + 4 * g + 1]);
-            w[GH + 4 * g + 2] = fmaf(-d, c.z, w[GH + 4 * g + 2]);
-            w[GH + 4 * g + 3] = fmaf(-d, c.w, w[GH + 4 * g + 3]);
-        }
-    }
-    if (ieee)
-        gptq_half<true, GH>(w, sLA, s, rs, fqmin, fqmax, dD, dV, dC, ncols, wt_row);
-    else
-        gptq_half<false, GH>(w, sLA, s, rs, fqmin, fqmax, dD, dV, dC, ncols, wt_row);
+        gptq_block<false>(x, sLA, s, rs, fqmin, fqmax, dV, dC, ncols, wt_row);
     __syncwarp();
     pdl_trigger();
     // row-coalesced writes: the warp walks its 32 rows, lanes along the columns
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(32, 1) leaf_gptq_kernel(LeafArgs p, int Jb)
         for (int c = lane; c < GB; c += 32) {
             const int64_t gc = col0 + c;
             float hi, lo;
-            split_tf32(sD[r * LDO + c], hi, lo);
+            split_tf32(sX[r * LDX + c], hi, lo);
             p.Dhi[gr * p.Np + gc] = hi;
             p.Dlo[gr * p.Np + gc] = lo;
             if (gc < p.n) {

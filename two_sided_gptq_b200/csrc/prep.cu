@@ -191,24 +191,6 @@ __global__ void normalize_split_kernel(const float *__restrict__ L, int64_t n, i
     }
 }
 
-// One-sided path: the transposed diagonal blocks of Lt, block J at
-// out + J * 128 * 128, out[J][j][i] = Lt[128J + i, 128J + j] (the coefficients
-// that column j pushes into the block's later columns, contiguous).  32 x 32
-// tiles through shared memory; grid (4, 4, Nt), 32 x 8 threads.
-__global__ void diag_blocks_t_kernel(const float *__restrict__ L32, int64_t Np, float *__restrict__ out)
-{
-    __shared__ float tile[32][33];
-    pdl_wait();
-    pdl_trigger();
-    const int64_t J = blockIdx.z;
-    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;  // source tile: rows r0.., columns c0.. of the block
-    const float *src = L32 + (J * 128) * Np + J * 128;
-    for (int y = threadIdx.y; y < 32; y += 8) tile[y][threadIdx.x] = src[(int64_t)(r0 + y) * Np + c0 + threadIdx.x];
-    __syncthreads();
-    float *dst = out + J * 128 * 128;
-    for (int y = threadIdx.y; y < 32; y += 8) dst[(int64_t)(c0 + y) * 128 + r0 + threadIdx.x] = tile[threadIdx.x][y];
-}
-
 static int grid_for(int64_t total, int threads)
 {
     int64_t b = (total + threads - 1) / threads;
@@ -236,9 +218,7 @@ cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, c
                         L.Np, (float *)(ws + L.LA32), (float *)(ws + L.LAhi), (float *)(ws + L.LAlo), st)) !=
         cudaSuccess)
         return e;
-    if (!LB)  // the one-sided path (B = I) has no output-side factor; its leaf reads transposed diagonal blocks
-        return launch_pdl(diag_blocks_t_kernel, dim3(4, 4, (unsigned)(L.Np / 128)), dim3(32, 8), 0, stream,
-                          (const float *)(ws + L.LA32), L.Np, (float *)(ws + L.XThi));
+    if (!LB) return cudaSuccess;  // the one-sided path (B = I) has no output-side factor
     return launch_pdl(normalize_split_kernel, dim3(grid_for(L.Mp * L.Mp, 256)), dim3(256), 0, stream, LB, m, L.Mp,
                       (float *)(ws + L.LB32), (float *)(ws + L.LBhi), (float *)(ws + L.LBlo), st);
 }
