@@ -18,7 +18,7 @@ Hessians", pith.science review of arXiv 2608.06291, and the arXiv abstract):
 * one-sided GPTQ, to which the method reduces when ``B = I`` ("Load-bearing
   premise": GPTQ's Hessian is ``E[xx^T] (x) I``).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 symmetric grid ``qmax = 2^(b-1)-1``, ``qmin = -qmax``; per-row step
 ``s_i = absmax_j |W_ij| / qmax`` in fp32 (1 for an all-zero row); ties round half
 to even; the decision ``clamp(rint(Wt/s))`` is taken in fp32; clamp error is part

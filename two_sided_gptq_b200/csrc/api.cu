@@ -399,7 +399,7 @@ bakron_status_t bakron_tune_leaf(const float *W_dev, int64_t m, int64_t n, const
     double best = 0.0;
     int best_leaf = 0;
     for (int leaf = 0; leaf <= 4 && s == BAKRON_OK; ++leaf) {
-        c.leaf = leaf == 0 ? 3 : leaf;  // round 0 is the warm-up
+        c.leaf = leaf == 0 ? 3 : leaf;  // iteration 0 is the warm-up
         if (cudaEventRecord(ev[0], st) != cudaSuccess) { s = BAKRON_ERR_CUDA; break; }
         s = bakron_solve(W_dev, m, n, LA_dev, LB_dev, q, V_dev, codes_dev, scales_dev, ws_dev, ws_bytes, &c, stream);
         if (s != BAKRON_OK) break;
