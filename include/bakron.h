@@ -298,6 +298,17 @@ bakron_status_t bakron_proxy_loss(const float *W_dev, const float *V_dev, const 
  * latest call on this workspace (BAKRON_OK if none), then clears it. */
 bakron_status_t bakron_get_status(void *ws_dev, size_t ws_bytes, bakron_stream_t stream);
 
+/* Failure-detection self-test: launches one thread that waits, with the same
+ * bounded-wait helper and deadline as the band-product kernels, on an
+ * mbarrier that nothing ever completes; after timeout_ms (1..10000) it gives
+ * up, records BAKRON_ERR_DEVICE_TIMEOUT in the status word at the start of
+ * ws_dev (>= 256 bytes, 16-byte aligned; cleared first) and returns, so the
+ * context stays usable.  Asynchronous on `stream`: read the result with
+ * bakron_get_status.  Returns BAKRON_ERR_INVALID_ARG for a timeout out of
+ * range, BAKRON_ERR_WORKSPACE / _ALIGNMENT for a bad workspace. */
+bakron_status_t bakron_selftest_wait_timeout(int32_t timeout_ms, void *ws_dev, size_t ws_bytes,
+                                             bakron_stream_t stream);
+
 /* Static description of a status code. */
 const char *bakron_status_string(bakron_status_t status);
 

@@ -96,6 +96,12 @@ def test_argument_errors_return_before_any_device_work(lib):
     a[11] = ctypes.byref(cfg)
     a[0] = fake + 4  # with LB = NULL accepted, validation goes on to the next check
     assert lib.bakron_solve(*a) == _native.Status.ERR_ALIGNMENT
+    # the bounded-wait self-test validates before it launches anything
+    assert lib.bakron_selftest_wait_timeout(0, fake, 256, None) == _native.Status.ERR_INVALID_ARG
+    assert lib.bakron_selftest_wait_timeout(10001, fake, 256, None) == _native.Status.ERR_INVALID_ARG
+    assert lib.bakron_selftest_wait_timeout(5, None, 256, None) == _native.Status.ERR_WORKSPACE
+    assert lib.bakron_selftest_wait_timeout(5, fake, 255, None) == _native.Status.ERR_WORKSPACE
+    assert lib.bakron_selftest_wait_timeout(5, fake + 8, 256, None) == _native.Status.ERR_ALIGNMENT
     assert lib.bakron_factor(fake, -1, fake, 4, fake, fake, fake, 1 << 30, None) == _native.Status.ERR_INVALID_ARG
     assert lib.bakron_factor(fake, 4, fake, 4, fake + 8, fake, fake, 1 << 30, None) == _native.Status.ERR_ALIGNMENT
     assert lib.bakron_factor(fake, 4, fake, 4, fake, fake, fake, 16, None) == _native.Status.ERR_WORKSPACE

@@ -1,0 +1,42 @@
+"""Failure detection on the GPU without a fault: a device wait that nothing
+completes gives up at its deadline, records BAKRON_ERR_DEVICE_TIMEOUT in the
+status word, and leaves the context usable for the next solve."""
+import numpy as np
+import pytest
+
+import workloads
+from parity import check_solve, oracle_factors
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import two_sided_gptq_b200 as bk
+
+    bk._lib()
+
+
+def test_bounded_wait_gives_up_and_context_stays_usable():
+    import torch
+
+    import two_sided_gptq_b200 as bk
+
+    ws = bk.workspace(256)
+    for timeout_ms in (5, 40):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        bk.selftest_wait_timeout(timeout_ms, ws)
+        e1.record()
+        assert bk.get_status(ws) == bk.Status.ERR_DEVICE_TIMEOUT
+        ms = e0.elapsed_time(e1)
+        assert timeout_ms * 0.9 <= ms < timeout_ms + 500, (timeout_ms, ms)
+        assert bk.get_status(ws) == bk.Status.OK  # reading clears it
+    # the context is intact: a solve right after runs and matches the oracle
+    W, A, B = workloads.random_problem(129, 257, seed=3)
+    LA, LB = oracle_factors(A, B)
+    check_solve(W, LA, LB, 4, label="after timeout")

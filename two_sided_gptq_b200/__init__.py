@@ -75,6 +75,14 @@ def get_status(ws, stream=None) -> Status:
     return Status(_lib().bakron_get_status(_ptr(ws), ws.numel(), _stream(stream)))
 
 
+def selftest_wait_timeout(timeout_ms: int, ws, stream=None) -> None:
+    """Launch the bounded-wait self-test (``bakron_selftest_wait_timeout``): a
+    device wait that nothing completes gives up after ``timeout_ms`` and records
+    ``Status.ERR_DEVICE_TIMEOUT`` in ``ws``; read it with :func:`get_status`."""
+    check(_lib().bakron_selftest_wait_timeout(int(timeout_ms), _ptr(ws), ws.numel(), _stream(stream)),
+          "bakron_selftest_wait_timeout")
+
+
 def factor(A, B=None, *, stream=None, ws=None, check_status=True):
     """``(LA, LB)`` with ``LA LA^T = A^{-1}``, ``LB LB^T = B^{-1}`` (lower, fp32)."""
     torch = _torch()

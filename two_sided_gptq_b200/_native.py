@@ -81,6 +81,7 @@ SIGNATURES = {
     "bakron_proxy_loss": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _vp, ctypes.POINTER(ctypes.c_double), _vp,
                                          _sz, _vp]),
     "bakron_get_status": (ctypes.c_int, [_vp, _sz, _vp]),
+    "bakron_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int32, _vp, _sz, _vp]),
     "bakron_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bakron_plan_stats": (ctypes.c_int, [_i64, _i64, ctypes.POINTER(Config), ctypes.POINTER(PlanStats)]),
     "bakron_version": (ctypes.c_char_p, []),

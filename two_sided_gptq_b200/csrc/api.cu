@@ -630,6 +630,18 @@ bakron_status_t bakron_proxy_loss(const float *W_dev, const float *V_dev, const 
     return BAKRON_OK;
 }
 
+bakron_status_t bakron_selftest_wait_timeout(int32_t timeout_ms, void *ws_dev, size_t ws_bytes,
+                                             bakron_stream_t stream)
+{
+    if (timeout_ms < 1 || timeout_ms > 10000) return BAKRON_ERR_INVALID_ARG;
+    if (!ws_dev || ws_bytes < kStatusBytes) return BAKRON_ERR_WORKSPACE;
+    if (!aligned16(ws_dev)) return BAKRON_ERR_ALIGNMENT;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemsetAsync(ws_dev, 0, kStatusBytes, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (launch_wait_timeout_selftest((DeviceStatus *)ws_dev, timeout_ms, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    return BAKRON_OK;
+}
+
 bakron_status_t bakron_get_status(void *ws_dev, size_t ws_bytes, bakron_stream_t stream)
 {
     if (!ws_dev || ws_bytes < kStatusBytes) return BAKRON_ERR_WORKSPACE;

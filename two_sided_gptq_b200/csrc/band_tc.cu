@@ -395,6 +395,22 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
     }
 }
 
+// Self-test of the bounded wait: one thread waits, with the band kernel's own
+// helper and deadline, on an mbarrier that no thread ever arrives on; when the
+// deadline passes it records BAKRON_ERR_DEVICE_TIMEOUT (where = 9000) and the
+// kernel returns, leaving the context usable.
+__global__ void wait_timeout_selftest_kernel(DeviceStatus *st, int timeout_ms)
+{
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        const uint64_t deadline = now_ns() + (uint64_t)timeout_ms * 1000000ull;
+        if (!mbar_wait(b, 0, deadline)) record_error(st, BAKRON_ERR_DEVICE_TIMEOUT, 9000);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 namespace {
 
@@ -465,6 +481,12 @@ bool make_gptq_maps(const GemmArgs &g, int64_t Mp, int64_t Np, TcMaps *m)
 cudaError_t launch_gptq_tc(const NodeParams &np, const GemmArgs &g, const TcMaps &maps, cudaStream_t stream)
 {
     return launch_pdl(band_tc_kernel<4>, dim3(np.l - np.h, np.Mt), dim3(kThreads), kSmem, stream, maps, np, g);
+}
+
+cudaError_t launch_wait_timeout_selftest(DeviceStatus *st, int timeout_ms, cudaStream_t stream)
+{
+    wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(st, timeout_ms);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gram_tc(const NodeParams &np, const GemmArgs &g, const TcMaps &maps, cudaStream_t stream)

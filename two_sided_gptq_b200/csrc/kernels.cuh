@@ -74,4 +74,8 @@ cudaError_t launch_proxy_loss(const float *W, const float *V, const float *A, co
 cudaError_t launch_factor(const float *A, int64_t n, float *L, double *work, DeviceStatus *st,
                           cudaStream_t stream);
 
+// One thread waits on an mbarrier nothing completes, with the band kernel's
+// bounded-wait helper; records BAKRON_ERR_DEVICE_TIMEOUT when it gives up.
+cudaError_t launch_wait_timeout_selftest(DeviceStatus *st, int timeout_ms, cudaStream_t stream);
+
 }  // namespace bakron
