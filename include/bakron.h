@@ -315,7 +315,9 @@ const char *bakron_status_string(bakron_status_t status);
 /* Schedule statistics of an m x n solve with the given config: number of
  * recursion nodes, leaf launches, and the algorithmic update FLOPs (2 x the
  * structurally non-zero multiply-adds of the band products over the tile
- * cut; the leaves' in-tile work excluded).  Host only; enqueues nothing. */
+ * cut; the leaves' in-tile work excluded).  With cfg->b_identity = 1 they
+ * describe the one-sided schedule (column blocks; its updates are counted as
+ * stage 1, stage 2 is 0).  Host only; enqueues nothing. */
 typedef struct {
     int64_t tiles_m, tiles_n, tile_diagonals;
     int64_t nodes, leaves;

@@ -194,3 +194,21 @@ def test_solve_batch_argument_errors_before_device_work(lib):
     assert lib.bakron_solve_batch(items, 2, ctypes.byref(q), None, st, 1) == _native.Status.ERR_WORKSPACE
     assert lib.bakron_solve_batch(items, 2, ctypes.byref(q), None, st, 0) == _native.Status.ERR_INVALID_ARG
 
+
+
+@pytest.mark.parametrize("shape", [(1, 1), (300, 260), (4096, 4096), (14336, 4096), (100, 1000)])
+def test_plan_stats_one_sided_closed_form(lib, shape):
+    """B = I schedule over Nt column blocks: Nt leaves, Nt - 1 nodes, and every
+    pair of blocks J < J' costs one 128^3 tile product per row tile, so the
+    update FLOPs are 2 T^3 Mt Nt (Nt - 1) / 2 (stage 2 empty)."""
+    from two_sided_gptq_b200 import _native
+
+    m, n = shape
+    T = 128
+    Mt, Nt = -(-m // T), -(-n // T)
+    s = _native.PlanStats()
+    cfg = _native.Config(0, 0, 0, 0, None, 0, 0, 1)
+    assert lib.bakron_plan_stats(m, n, ctypes.byref(cfg), ctypes.byref(s)) == 0
+    assert (s.leaves, s.nodes) == (Nt, Nt - 1)
+    assert s.stage2_flops == 0
+    assert s.update_flops == s.stage1_flops == T ** 3 * Mt * Nt * (Nt - 1)

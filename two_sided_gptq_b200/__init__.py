@@ -301,8 +301,10 @@ def last_profile_launches() -> list:
     return [{"kind": kinds[r.kind], "k": r.k, "h": r.h, "l": r.l, "ms": r.ms, "flops": r.flops} for r in buf[:n]]
 
 
-def plan_stats(m: int, n: int) -> dict:
-    """Schedule statistics of an m x n solve (host only)."""
+def plan_stats(m: int, n: int, one_sided: bool = False) -> dict:
+    """Schedule statistics of an m x n solve (host only); ``one_sided`` for
+    the B = I schedule over column blocks."""
     s = PlanStats()
-    check(_lib().bakron_plan_stats(m, n, None, ctypes.byref(s)), "bakron_plan_stats")
+    cfg = _config(b_identity=int(one_sided))
+    check(_lib().bakron_plan_stats(m, n, ctypes.byref(cfg), ctypes.byref(s)), "bakron_plan_stats")
     return {f: getattr(s, f) for f, _ in PlanStats._fields_}

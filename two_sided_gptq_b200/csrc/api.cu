@@ -338,6 +338,21 @@ void count_schedule(int k, int l, int Mt, int Nt, bakron_plan_stats_t *o)
     count_schedule(k + h, l - h, Mt, Nt, o);
 }
 
+// One-sided path: the recursion over column blocks; every update counts as
+// stage 1 (there is no second product).
+void count_schedule_gptq(int k, int l, int Mt, int Nt, bakron_plan_stats_t *o)
+{
+    if (l <= 1) {
+        o->leaves++;
+        return;
+    }
+    const int h = l / 2;
+    count_schedule_gptq(k, h, Mt, Nt, o);
+    o->stage1_flops += gptq_node_flops(NodeParams{k, h, l, Mt, Nt});
+    o->nodes++;
+    count_schedule_gptq(k + h, l - h, Mt, Nt, o);
+}
+
 }  // namespace
 
 extern "C" {
@@ -677,7 +692,10 @@ bakron_status_t bakron_plan_stats(int64_t m, int64_t n, const bakron_config_t *c
     out->tiles_m = (m + kTile - 1) / kTile;
     out->tiles_n = (n + kTile - 1) / kTile;
     out->tile_diagonals = out->tiles_m + out->tiles_n - 1;
-    count_schedule(0, (int)out->tile_diagonals, (int)out->tiles_m, (int)out->tiles_n, out);
+    if (conf.b_identity)
+        count_schedule_gptq(0, (int)out->tiles_n, (int)out->tiles_m, (int)out->tiles_n, out);
+    else
+        count_schedule(0, (int)out->tile_diagonals, (int)out->tiles_m, (int)out->tiles_n, out);
     out->update_flops = out->stage1_flops + out->stage2_flops;
     return BAKRON_OK;
 }
