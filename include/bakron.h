@@ -86,7 +86,14 @@ typedef struct {
  *               cuts on: 128 (default; the only supported value).
  *   gemm        0 = tcgen05 tensor-core 3xTF32 band GEMMs (default),
  *               1 = FP32 CUDA-core band GEMMs (cross-check).
- *   use_graph   reserved, must be 0.
+ *   use_graph   1: capture the solve's launches for this argument set
+ *               (every pointer, size, quantizer and config field, device) into
+ *               a CUDA graph on the first call, on a private stream of the
+ *               calling thread, and replay it on `stream` in later calls
+ *               (the programmatic launches become programmatic graph edges;
+ *               a replay reads the buffers' current contents).  Up to 64
+ *               graphs are kept per process, oldest dropped first.  Not with
+ *               profile = 1 (BAKRON_ERR_INVALID_ARG).  0: launch directly.
  *   timeout_ms  limit for device-side bounded waits (default 200).
  *   wt_out      optional device pointer, m x n fp32: if not NULL it receives
  *               every entry's pre-rounding value Wt_ij (diagnostics). */

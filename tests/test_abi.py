@@ -85,6 +85,10 @@ def test_argument_errors_return_before_any_device_work(lib):
     a = list(args())
     a[11] = ctypes.byref(cfg)
     assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
+    # use_graph is 0 or 1, and not with per-launch profiling
+    for bad in (_native.Config(0, 0, 2, 0, None), _native.Config(0, 0, 1, 0, None, 1)):
+        a[11] = ctypes.byref(bad)
+        assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
     # b_identity is 0 or 1; LB may be NULL only on the one-sided path
     cfg = _native.Config(0, 0, 0, 0, None, 0, 0, 2)
     a[11] = ctypes.byref(cfg)

@@ -59,8 +59,8 @@ def _dev_f32(x, name):
     return x
 
 
-def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False, leaf=0, b_identity=False):
-    return Config(0, int(gemm), 0, int(timeout_ms), _ptr(wt_out), 1 if profile else 0, int(leaf),
+def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False, leaf=0, b_identity=False, graph=False):
+    return Config(0, int(gemm), 1 if graph else 0, int(timeout_ms), _ptr(wt_out), 1 if profile else 0, int(leaf),
                   1 if b_identity else 0)
 
 
@@ -111,7 +111,7 @@ def solve_workspace_size(m: int, n: int, gemm: int = 0) -> int:
 
 
 def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None, out=None, stream=None,
-          wt_out=None, check_status=True, timeout_ms=0, profile=False, leaf=0, shrink_grid=0):
+          wt_out=None, check_status=True, timeout_ms=0, profile=False, leaf=0, shrink_grid=0, graph=False):
     """BaKron solve on device tensors.  Returns ``(V, codes, scales)``.
 
     ``LB=None`` selects the one-sided path (B = I: GPTQ with Hessian A, over
@@ -123,7 +123,9 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     selects the leaf sweep structure (0 default,
     1 two-level CTA-wide, 2 single-level, 3 three warps per 32 x 32
     sub-tile, 4 six warps per 64 x 64 sub-tile; :func:`tune_leaf` picks one by
-    measurement).  ``out`` may supply ``(V, codes, scales)`` buffers and
+    measurement).  ``graph=True`` captures the solve's launches for this
+    argument set into a CUDA graph on the first call and replays it on later
+    calls with the same buffers.  ``out`` may supply ``(V, codes, scales)`` buffers and
     ``ws`` a workspace; ``check_status=False`` skips the synchronising status
     read (for timing).
     """
@@ -136,7 +138,7 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     m, n = W.shape
     if LA.shape != (n, n) or (not one_sided and LB.shape != (m, m)):
         raise ValueError("LA must be n x n and LB m x m")
-    cfg = _config(gemm, timeout_ms, wt_out, profile, leaf, one_sided)
+    cfg = _config(gemm, timeout_ms, wt_out, profile, leaf, one_sided, graph)
     if out is None:
         V = torch.empty((m, n), dtype=torch.float32, device=W.device)
         codes = torch.empty((m, n), dtype=torch.int8, device=W.device)

@@ -107,7 +107,8 @@ bakron_status_t read_config(const bakron_config_t *c, Config &out)
     if (c->tile != 0 && c->tile != kTile) return BAKRON_ERR_INVALID_ARG;
     if (c->gemm < 0 || c->gemm > 1) return BAKRON_ERR_INVALID_ARG;
     out.gemm = c->gemm;
-    if (c->use_graph != 0) return BAKRON_ERR_INVALID_ARG;
+    if (c->use_graph < 0 || c->use_graph > 1) return BAKRON_ERR_INVALID_ARG;
+    out.use_graph = c->use_graph;
     if (c->timeout_ms < 0) return BAKRON_ERR_INVALID_ARG;
     if (c->timeout_ms > 0) out.timeout_ms = c->timeout_ms;
     out.wt_out = c->wt_out;
@@ -116,6 +117,7 @@ bakron_status_t read_config(const bakron_config_t *c, Config &out)
     if (c->leaf != 0) out.leaf = c->leaf - 1;  // 0 keeps the default
     if (c->b_identity < 0 || c->b_identity > 1) return BAKRON_ERR_INVALID_ARG;
     out.b_identity = c->b_identity;
+    if (out.use_graph && out.profile) return BAKRON_ERR_INVALID_ARG;  // per-launch events cannot be replayed
     return BAKRON_OK;
 }
 
@@ -213,6 +215,79 @@ cudaError_t run_schedule_gptq(SolveCtx &c, const TcMaps &maps, int k, int l)
     return run_schedule_gptq(c, maps, k + h, l - h);
 }
 
+bakron_status_t enqueue_solve(const float *W, int64_t m, int64_t n, const float *LA, const float *LB,
+                              const bakron_quantizer_t *q, int qmin, int qmax, float *V, int8_t *codes,
+                              float *scales, const SolveLayout &L, char *w, const Config &conf,
+                              cudaStream_t stream);
+
+// CUDA graph mode (cfg.use_graph): the launches of one argument set
+// (pointers, sizes, grid, config, device) are captured once, on a private
+// stream of the calling thread, into an executable graph that later calls
+// replay on the caller's stream.  The programmatic launches become
+// programmatic graph edges, so the replay keeps the overlap of each kernel's
+// prologue with its predecessor.  Kernel arguments hold only pointers and
+// sizes, so a replay reads the buffers' current contents.  At most
+// kGraphCacheSize graphs are kept (oldest dropped first; a graph still
+// running is freed when it completes).
+struct GraphKey {
+    const void *p[9];
+    int64_t m, n;
+    size_t ws_bytes;
+    int v[8];
+    bool operator==(const GraphKey &o) const
+    {
+        return std::memcmp(p, o.p, sizeof(p)) == 0 && m == o.m && n == o.n && ws_bytes == o.ws_bytes &&
+               std::memcmp(v, o.v, sizeof(v)) == 0;
+    }
+};
+constexpr size_t kGraphCacheSize = 64;
+std::mutex g_graph_mu;
+std::vector<std::pair<GraphKey, cudaGraphExec_t>> g_graphs;  // oldest first
+
+// Launches the cached graph for `key` on `stream` (the cache lock is held
+// while the launch is enqueued, so no other thread can drop it meanwhile).
+bool launch_cached_graph(const GraphKey &key, cudaStream_t stream, bakron_status_t *out)
+{
+    std::lock_guard<std::mutex> lk(g_graph_mu);
+    for (auto &e : g_graphs)
+        if (e.first == key) {
+            *out = cudaGraphLaunch(e.second, stream) == cudaSuccess ? BAKRON_OK : BAKRON_ERR_CUDA;
+            return true;
+        }
+    return false;
+}
+
+template <class Enqueue>
+bakron_status_t launch_graph(const GraphKey &key, cudaStream_t stream, Enqueue enqueue)
+{
+    bakron_status_t r = BAKRON_OK;
+    if (launch_cached_graph(key, stream, &r)) return r;
+    thread_local cudaStream_t cap[64] = {};
+    const int dev = key.v[7];
+    if (dev < 0 || dev >= 64) return BAKRON_ERR_CUDA;
+    if (!cap[dev] && cudaStreamCreateWithFlags(&cap[dev], cudaStreamNonBlocking) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
+    if (cudaStreamBeginCapture(cap[dev], cudaStreamCaptureModeThreadLocal) != cudaSuccess) return BAKRON_ERR_CUDA;
+    r = enqueue(cap[dev]);
+    cudaGraph_t graph = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(cap[dev], &graph);
+    if (r != BAKRON_OK || e != cudaSuccess) {
+        if (graph) cudaGraphDestroy(graph);
+        return r != BAKRON_OK ? r : BAKRON_ERR_CUDA;
+    }
+    cudaGraphExec_t exec = nullptr;
+    const cudaError_t ei = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (ei != cudaSuccess) return BAKRON_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_graph_mu);
+    g_graphs.emplace_back(key, exec);
+    if (g_graphs.size() > kGraphCacheSize) {
+        cudaGraphExecDestroy(g_graphs.front().second);
+        g_graphs.erase(g_graphs.begin());
+    }
+    return cudaGraphLaunch(exec, stream) == cudaSuccess ? BAKRON_OK : BAKRON_ERR_CUDA;
+}
+
 bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *LA, const float *LB,
                              const bakron_quantizer_t *q, float *V, int8_t *codes, float *scales,
                              void *ws, size_t ws_bytes, const bakron_config_t *cfg,
@@ -236,8 +311,28 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
     L.compute(m, n, kTile);
     if (ws_bytes < L.total) return BAKRON_ERR_WORKSPACE;
     if (configure_device() != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (conf.use_graph) {
+        GraphKey key{};
+        const void *ptrs[] = {W, LA, LB, V, codes, scales, ws, conf.wt_out, q->row_scale};
+        for (int i = 0; i < 9; ++i) key.p[i] = ptrs[i];
+        key.m = m; key.n = n; key.ws_bytes = ws_bytes;
+        key.v[0] = qmin; key.v[1] = qmax; key.v[2] = q->row_scale ? 0 : q->shrink_grid; key.v[3] = conf.gemm;
+        key.v[4] = conf.leaf; key.v[5] = conf.timeout_ms; key.v[6] = conf.b_identity;
+        if (cudaGetDevice(&key.v[7]) != cudaSuccess) return BAKRON_ERR_CUDA;
+        return launch_graph(key, stream, [&](cudaStream_t cap) {
+            return enqueue_solve(W, m, n, LA, LB, q, qmin, qmax, V, codes, scales, L, (char *)ws, conf, cap);
+        });
+    }
+    return enqueue_solve(W, m, n, LA, LB, q, qmin, qmax, V, codes, scales, L, (char *)ws, conf, stream);
+}
 
-    char *w = (char *)ws;
+// Every launch of one solve, in order, on `stream` (no argument checks: the
+// caller has made them).
+bakron_status_t enqueue_solve(const float *W, int64_t m, int64_t n, const float *LA, const float *LB,
+                              const bakron_quantizer_t *q, int qmin, int qmax, float *V, int8_t *codes,
+                              float *scales, const SolveLayout &L, char *w, const Config &conf,
+                              cudaStream_t stream)
+{
     DeviceStatus *st = (DeviceStatus *)(w + L.status);
     if (cudaMemsetAsync(st, 0, kStatusBytes, stream) != cudaSuccess) return BAKRON_ERR_CUDA;
     t_prof.on = conf.profile != 0;
