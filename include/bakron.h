@@ -82,6 +82,11 @@ typedef struct {
 } bakron_quantizer_t;
 
 /* Solver configuration (NULL = defaults; zero fields take defaults).
+ * The environment can change the defaults of four fields: BAKRON_LEAF (0..4),
+ * BAKRON_GEMM (0..1), BAKRON_TIMEOUT_MS (1..600000) and BAKRON_GRAPH (0..1,
+ * ignored when profile = 1); a non-zero field set by the caller wins.  A
+ * variable that is set but not an integer in its range makes every call that
+ * reads a config return BAKRON_ERR_INVALID_ARG.
  *   tile        side T of the square tiles whose anti-diagonals the recursion
  *               cuts on: 128 (default; the only supported value).
  *   gemm        0 = tcgen05 tensor-core 3xTF32 band GEMMs (default),

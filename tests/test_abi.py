@@ -3,6 +3,7 @@ function include/bakron.h declares, and its host-only entry points behave."""
 import ctypes
 import os
 import re
+import sys
 
 import pytest
 
@@ -216,3 +217,29 @@ def test_plan_stats_one_sided_closed_form(lib, shape):
     assert (s.leaves, s.nodes) == (Nt, Nt - 1)
     assert s.stage2_flops == 0
     assert s.update_flops == s.stage1_flops == T ** 3 * Mt * Nt * (Nt - 1)
+
+
+def _plan_status_under_env(env):
+    import subprocess
+
+    code = ("import ctypes, sys; sys.path.insert(0, %r); from two_sided_gptq_b200 import _native; "
+            "lib = _native.load(); s = _native.PlanStats(); "
+            "print(lib.bakron_plan_stats(256, 256, None, ctypes.byref(s)))") % ROOT
+    e = dict(os.environ)
+    e.update(env)
+    out = subprocess.run([sys.executable, "-c", code], env=e, capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    return int(out.stdout.strip())
+
+
+def test_environment_overrides_are_validated():
+    """BAKRON_LEAF / _GEMM / _TIMEOUT_MS / _GRAPH change defaults; a malformed
+    or out-of-range value makes config-reading calls fail with INVALID_ARG."""
+    from two_sided_gptq_b200 import _native
+
+    ok, bad = _native.Status.OK, _native.Status.ERR_INVALID_ARG
+    assert _plan_status_under_env({"BAKRON_LEAF": "4", "BAKRON_GEMM": "1", "BAKRON_TIMEOUT_MS": "50",
+                                   "BAKRON_GRAPH": "1"}) == ok
+    for env in ({"BAKRON_LEAF": "5"}, {"BAKRON_GEMM": "2"}, {"BAKRON_TIMEOUT_MS": "0"},
+                {"BAKRON_TIMEOUT_MS": "12ms"}, {"BAKRON_GRAPH": "-1"}):
+        assert _plan_status_under_env(env) == bad, env

@@ -147,6 +147,22 @@ def test_tune_leaf_picks_a_measured_structure():
     check_solve(W, LA, LB, 4, leaf=leaf, label=f"mid/tuned-leaf{leaf}")
 
 
+def test_tune_leaf_cache(tmp_path):
+    """With a cache file the first call measures and stores, the second returns
+    the stored measurement for the same (m, n, bits, GPU)."""
+    import torch
+
+    import two_sided_gptq_b200 as bk
+
+    W, A, B, LA, LB = named("mid")
+    Wd, LAd, LBd = (torch.from_numpy(x).cuda() for x in (W, LA.astype(np.float32), LB.astype(np.float32)))
+    path = str(tmp_path / "tune.json")
+    first = bk.tune_leaf(Wd, LAd, LBd, bits=4, cache=path)
+    key = bk.tune_cache_key(1024, 1024, 4, torch.cuda.get_device_name(0))
+    assert bk.tune_cache_get(path, key) == first
+    assert bk.tune_leaf(Wd, LAd, LBd, bits=4, cache=path) == first
+
+
 @pytest.mark.parametrize("case", [("mid", 4, 100), ((300, 260), 3, 64), ((129, 257), 2, 20)])
 def test_mse_searched_steps(case):
     """shrink_grid: the device's searched steps equal the oracle's (a row whose

@@ -156,14 +156,70 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     return V, codes, scales
 
 
-def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, timeout_ms=0):
+def tune_cache_key(m: int, n: int, bits: int, device_name: str) -> str:
+    """Key of a leaf-structure measurement in the autotune cache."""
+    return f"{int(m)}x{int(n)}/int{int(bits)}/{device_name}"
+
+
+def tune_cache_get(path: str, key: str):
+    """``(leaf, ms_list)`` stored under ``key`` in the JSON file ``path``, or None."""
+    import json
+    import os
+
+    if not path or not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            entry = json.load(f).get(key)
+    except (OSError, ValueError):
+        return None
+    if not isinstance(entry, dict) or entry.get("leaf") not in (1, 2, 3, 4):
+        return None
+    return int(entry["leaf"]), [float(x) for x in entry.get("ms", [])]
+
+
+def tune_cache_put(path: str, key: str, leaf: int, ms) -> None:
+    """Store a measurement under ``key`` in the JSON file ``path`` (written to a
+    temporary file and renamed, so readers never see a partial file)."""
+    import json
+    import os
+    import tempfile
+
+    data = {}
+    if os.path.exists(path):
+        try:
+            with open(path) as f:
+                data = json.load(f)
+        except (OSError, ValueError):
+            data = {}
+    data[key] = {"leaf": int(leaf), "ms": [float(x) for x in ms]}
+    d = os.path.dirname(os.path.abspath(path))
+    fd, tmp = tempfile.mkstemp(dir=d, prefix=".bakron_tune_")
+    with os.fdopen(fd, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=True)
+    os.replace(tmp, path)
+
+
+def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, timeout_ms=0, cache=None):
     """Leaf structure chosen by measurement (``bakron_tune_leaf``): one timed
     solve per structure on this problem.  Returns ``(leaf, [ms_leaf1, ...,
-    ms_leaf4])``; pass ``leaf`` to :func:`solve`."""
+    ms_leaf4])``; pass ``leaf`` to :func:`solve`.
+
+    ``cache`` (or the ``BAKRON_TUNE_CACHE`` environment variable) names a JSON
+    file keyed by (m, n, bits, GPU name): a stored measurement is returned
+    without timing, a new one is stored."""
+    import os
+
     torch = _torch()
     lib = _lib()
     _dev_f32(W, "W"), _dev_f32(LA, "LA"), _dev_f32(LB, "LB")
     m, n = W.shape
+    cache = cache or os.environ.get("BAKRON_TUNE_CACHE")
+    key = tune_cache_key(m, n, bits, torch.cuda.get_device_name(W.device)) if cache else None
+    if cache:
+        hit = tune_cache_get(cache, key)
+        if hit is not None:
+            return hit
     cfg = _config(gemm, timeout_ms)
     if out is None:
         out = (torch.empty((m, n), dtype=torch.float32, device=W.device),
@@ -180,7 +236,10 @@ def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, time
                                _ptr(scales), _ptr(ws), ws.numel(), ctypes.byref(cfg), st, ctypes.byref(leaf), ms),
           "bakron_tune_leaf")
     check(lib.bakron_get_status(_ptr(ws), ws.numel(), st), "bakron_tune_leaf (device)")
-    return int(leaf.value), [float(x) for x in ms]
+    result = int(leaf.value), [float(x) for x in ms]
+    if cache:
+        tune_cache_put(cache, key, *result)
+    return result
 
 
 def solve_batch(problems, bits=4, *, streams, outs=None, workspaces=None, gemm=0, leaf=0, shrink_grid=0,

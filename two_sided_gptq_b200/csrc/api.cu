@@ -100,15 +100,37 @@ double gptq_node_flops(const NodeParams &np)
     return f;
 }
 
+// Environment override of a default: false if the variable is set but not an
+// integer in [lo, hi].
+bool env_int(const char *name, int lo, int hi, int &v)
+{
+    const char *e = std::getenv(name);
+    if (!e || !*e) return true;
+    char *end = nullptr;
+    const long x = std::strtol(e, &end, 10);
+    if (*end != '\0' || x < lo || x > hi) return false;
+    v = (int)x;
+    return true;
+}
+
 bakron_status_t read_config(const bakron_config_t *c, Config &out)
 {
     out = Config();
+    // defaults that BAKRON_LEAF, BAKRON_GEMM, BAKRON_TIMEOUT_MS and BAKRON_GRAPH
+    // override; a non-zero field of the caller's config overrides both
+    int leaf = 0, gemm = 0, graph = 0;
+    if (!env_int("BAKRON_LEAF", 0, 4, leaf) || !env_int("BAKRON_GEMM", 0, 1, gemm) ||
+        !env_int("BAKRON_TIMEOUT_MS", 1, 600000, out.timeout_ms) || !env_int("BAKRON_GRAPH", 0, 1, graph))
+        return BAKRON_ERR_INVALID_ARG;
+    if (leaf != 0) out.leaf = leaf - 1;
+    out.gemm = gemm;
+    if (!c || !c->profile) out.use_graph = graph;
     if (!c) return BAKRON_OK;
     if (c->tile != 0 && c->tile != kTile) return BAKRON_ERR_INVALID_ARG;
     if (c->gemm < 0 || c->gemm > 1) return BAKRON_ERR_INVALID_ARG;
-    out.gemm = c->gemm;
+    if (c->gemm) out.gemm = c->gemm;
     if (c->use_graph < 0 || c->use_graph > 1) return BAKRON_ERR_INVALID_ARG;
-    out.use_graph = c->use_graph;
+    if (c->use_graph) out.use_graph = c->use_graph;
     if (c->timeout_ms < 0) return BAKRON_ERR_INVALID_ARG;
     if (c->timeout_ms > 0) out.timeout_ms = c->timeout_ms;
     out.wt_out = c->wt_out;
