@@ -99,3 +99,22 @@ def test_aggregate_rate_counts_every_rank():
     assert one == pytest.approx(4096 * 4096 / 0.010)
     assert bench.aggregate_rate(8, 4096, 4096, 10.0) == pytest.approx(8 * one)
     assert bench.max_over_ranks(3.25, None) == 3.25
+
+
+def test_working_set_matches_the_library_layout():
+    """bench.py's working-set note uses the same workspace size as the library
+    (bakron_solve_workspace_size, a host-only query) and says whether a step's
+    data exceeds the L2."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+
+    import two_sided_gptq_b200 as bk
+
+    lib = bk._lib()
+    for m, n in ((4096, 4096), (64, 128), (14336, 4096), (300, 260)):
+        ws = bench.working_set_bytes(m, n)[2]
+        assert abs(ws - lib.bakron_solve_workspace_size(m, n, None)) <= 4096, (m, n)
+    args = type("Args", (), {"gpus": 1})()
+    assert "exceeds" in bench.config_block(workloads.WORKLOADS["bench"], args)["l2"]
+    assert "fits" in bench.config_block(workloads.WORKLOADS["tiny"], args)["l2"]
