@@ -18,8 +18,11 @@
  *     named *_dev are CUDA device pointers, *_host are host pointers.  Every
  *     device pointer must be 16-byte aligned (else BAKRON_ERR_ALIGNMENT).
  *   - The caller owns every buffer.  The library never allocates device or
- *     pinned memory, never frees or retains caller memory; all scratch lives
- *     in the caller's workspace, whose size the *_workspace_size query gives.
+ *     pinned memory buffers, never frees or retains caller memory; all scratch
+ *     lives in the caller's workspace, whose size the *_workspace_size query
+ *     gives.  (Exceptions, all driver-side: bakron_solve_noalloc's fixed
+ *     scratch array, reserved when the library loads; and in CUDA graph mode a
+ *     private stream per calling thread and the cached executable graphs.)
  *   - Calls are stream-ordered and asynchronous on `stream` (a cudaStream_t;
  *     NULL = legacy default stream).  Argument errors are returned at once and
  *     nothing is enqueued.  Errors found on the device (non-SPD pivot,
