@@ -6,6 +6,7 @@ Each test names the statement it checks.  Pages: pith.science review of
 "If this is right" = Corollary 3.4's bound, "Load-bearing premise" = GPTQ's
 one-sided Hessian) and the arXiv abstract.
 """
+import os
 from fractions import Fraction
 
 import numpy as np
@@ -137,6 +138,17 @@ def test_prop_3_1_hand_worked_2x2(oracle_mod):
     codes, Wt = o.solve(W, LtA, LtB, s, qmin, qmax)
     np.testing.assert_allclose(Wt, expect_wt, rtol=0, atol=1e-15)
     assert np.array_equal(codes, expect)
+    # the same example stored as a fixture (tests/golden/prop31_2x2.txt)
+    g = {}
+    for line in open(os.path.join(os.path.dirname(__file__), "golden", "prop31_2x2.txt")):
+        if line.strip() and not line.startswith("#"):
+            k, *v = line.split()
+            g[k] = v
+    assert [float(x) for x in g["W"]] == W.ravel().tolist() and [float(x) for x in g["s"]] == s.tolist()
+    assert [F(x) for x in g["Wt"]] == [Wf[0][0], wt01, wt10, wt11]  # exact
+    assert [int(x) for x in g["codes"]] == codes.ravel().tolist()
+    np.testing.assert_allclose(Wt.ravel(), [float(F(x)) for x in g["Wt"]], rtol=0, atol=1e-15)
+    assert F(g["LtA10"][0]) == F(-1, 2) and F(g["LtB10"][0]) == F(-2, 3)
     assert np.array_equal(o.naive(W, A, B, s, qmin, qmax)[0], expect)
     # the swapped-roles solve gives different pre-rounding values here
     _, Wt_sw = o.solve(W, LtB, LtA, s, qmin, qmax)
