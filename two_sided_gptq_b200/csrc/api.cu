@@ -313,7 +313,7 @@ bakron_status_t launch_graph(const GraphKey &key, cudaStream_t stream, Enqueue e
 bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *LA, const float *LB,
                              const bakron_quantizer_t *q, float *V, int8_t *codes, float *scales,
                              void *ws, size_t ws_bytes, const bakron_config_t *cfg,
-                             cudaStream_t stream, bool user_scales_on_device)
+                             cudaStream_t stream, bool user_scales_on_device, bool direct_only = false)
 {
     if (m < 1 || n < 1 || m > kMaxSide || n > kMaxSide) return BAKRON_ERR_INVALID_ARG;
     Config conf;
@@ -333,7 +333,7 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
     L.compute(m, n, kTile);
     if (ws_bytes < L.total) return BAKRON_ERR_WORKSPACE;
     if (configure_device() != cudaSuccess) return BAKRON_ERR_CUDA;
-    if (conf.use_graph) {
+    if (conf.use_graph && !direct_only) {
         GraphKey key{};
         const void *ptrs[] = {W, LA, LB, V, codes, scales, ws, conf.wt_out, q->row_scale};
         for (int i = 0; i < 9; ++i) key.p[i] = ptrs[i];
@@ -533,7 +533,9 @@ bakron_status_t bakron_tune_leaf(const float *W_dev, int64_t m, int64_t n, const
     for (int leaf = 0; leaf <= 4 && s == BAKRON_OK; ++leaf) {
         c.leaf = leaf == 0 ? 3 : leaf;  // iteration 0 is the warm-up
         if (cudaEventRecord(ev[0], st) != cudaSuccess) { s = BAKRON_ERR_CUDA; break; }
-        s = bakron_solve(W_dev, m, n, LA_dev, LB_dev, q, V_dev, codes_dev, scales_dev, ws_dev, ws_bytes, &c, stream);
+        // timed with direct launches (a first graph call would time its capture)
+        s = solve_device(W_dev, m, n, LA_dev, LB_dev, q, V_dev, codes_dev, scales_dev, ws_dev, ws_bytes, &c,
+                         (cudaStream_t)stream, true, true);
         if (s != BAKRON_OK) break;
         if (cudaEventRecord(ev[1], st) != cudaSuccess || cudaEventSynchronize(ev[1]) != cudaSuccess) {
             s = BAKRON_ERR_CUDA;
