@@ -18,8 +18,9 @@ import ctypes
 from . import _native
 from ._native import BakronError, BatchItem, Config, PlanStats, Profile, ProfileLaunch, Quantizer, Status, check
 
-__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile", "last_profile_launches", "tune_leaf", "solve_batch", "gram",
-           "workspace", "get_status",
+__all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile",
+           "last_profile_launches", "tune_leaf", "tune_cache_key", "tune_cache_get", "tune_cache_put",
+           "solve_batch", "gram", "selftest_wait_timeout", "workspace", "get_status",
            "BakronError", "Status", "version", "library_path"]
 
 
