@@ -32,7 +32,7 @@ TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 : BF16 tensor peak ratio
 FALLBACK_BF16_TFLOPS = 1590.0
 LEAF_BYTES_PER_WEIGHT = 25  # read Wt 4 + diagonal factor blocks 8; write code 1, V 4, D hi/lo 8
 LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 255), 3: ("leaf_warp_kernel", 7 * 63),
-                4: ("leaf_wide_kernel", 3 * 127)}
+                4: ("leaf_wide_kernel", 3 * 127), 5: ("leaf_cluster_kernel", 7 * 63)}
 # DRAM traffic of the band products from an ncu capture of one solve's 124
 # band launches (profiles/band_tc_4096_dram.md); reported only while the
 # kernel sources hash to the value the capture was taken with.
@@ -163,11 +163,20 @@ def load_inputs(name, rank, dist):
     return W, A, B
 
 
-def cpu_baseline(W, A, B, bits, target_s=15.0, single_thread=False):
+def oracle_factors(A, B):
+    """The oracle's normalised FP64 factors (computed once per run)."""
+    import oracle
+
+    return oracle.normalize(oracle.factor(A)), oracle.normalize(oracle.factor(B))
+
+
+def cpu_baseline(W, A, B, bits, target_s=15.0, single_thread=False, factors=None, rows=None):
     """Oracle (FP64 anti-diagonal pull, OpenMP over each diagonal) timed on a
     bounded sample: the top r rows, a closed sub-problem (rows < r never depend
-    on later rows), with r chosen for about ``target_s`` of work; the time is
-    scaled to the full matrix by the ratio of multiply-adds r n (r+n) : m n (m+n)."""
+    on later rows), with r chosen for about ``target_s`` of work (or given as
+    ``rows``; r = m is the whole matrix and needs no scaling); a partial time
+    is scaled to the full matrix by the ratio of multiply-adds
+    r n (r+n) : m n (m+n)."""
     import numpy as np
 
     import oracle
@@ -175,8 +184,7 @@ def cpu_baseline(W, A, B, bits, target_s=15.0, single_thread=False):
     m, n = W.shape
     qmin, qmax = oracle.grid(bits)
     s = oracle.scales(W, qmax)
-    LtA = oracle.normalize(oracle.factor(A))
-    LtB = oracle.normalize(oracle.factor(B))
+    LtA, LtB = factors if factors is not None else oracle_factors(A, B)
     threads = oracle.num_threads()
 
     def run(r):
@@ -184,39 +192,45 @@ def cpu_baseline(W, A, B, bits, target_s=15.0, single_thread=False):
         oracle.solve(W[:r], LtA, np.ascontiguousarray(LtB[:r, :r]), s[:r], qmin, qmax, mode="pull", nthreads=threads)
         return time.perf_counter() - t0
 
-    r0 = min(m, 128)
-    t0 = run(r0)
     work = lambda r: r * n * (r + n)
-    r = r0
-    while r < m and t0 * work(min(m, 2 * r)) / work(r0) <= target_s:
-        r = min(m, 2 * r)
-    t = run(r) if r != r0 else t0
+    if rows is not None:
+        r = min(m, rows)
+        t = run(r)
+    else:
+        r0 = min(m, 128)
+        t0 = run(r0)
+        r = r0
+        while r < m and t0 * work(min(m, 2 * r)) / work(r0) <= target_s:
+            r = min(m, 2 * r)
+        t = run(r) if r != r0 else t0
     t_full = t * work(m) / work(r)
+    sample = (f"the whole {m}x{n} workload, {t:.2f} s measured" if r == m else
+              f"top {r} of {m} rows of the {m}x{n} workload (closed sub-problem), {t:.2f} s measured, "
+              f"scaled x{work(m) / work(r):.2f} by multiply-add count to the whole matrix")
     out = {"value": m * n / t_full, "unit": "weights/s", "cores": threads, "kind": "oracle",
-           "sample": f"top {r} of {m} rows of the {m}x{n} workload (closed sub-problem), {t:.2f} s measured, "
-                     f"scaled x{work(m) / work(r):.2f} by multiply-add count",
-           "sample_seconds": t, "nproc": os.cpu_count()}
+           "sample": sample, "sample_seconds": t, "nproc": os.cpu_count()}
     if single_thread and threads > 1:
         r1 = min(m, 64)
         t1 = time.perf_counter()
         oracle.solve(W[:r1], LtA, np.ascontiguousarray(LtB[:r1, :r1]), s[:r1], qmin, qmax, mode="pull", nthreads=1)
         t1 = time.perf_counter() - t1
         out["single_thread_value"] = m * n / (t1 * work(m) / work(r1))
-        out["single_thread_sample"] = f"top {r1} rows, 1 thread, {t1:.2f} s measured"
+        out["single_thread_sample"] = f"top {r1} rows, 1 thread, {t1:.2f} s measured, scaled by multiply-add count"
     return out
 
 
 def band_levels(launches):
     """Band-product time and tensor-pipe fraction per recursion level (node
-    width l in tile diagonals), medians over the profiled steps."""
+    width l in tile diagonals; separate or fused stage launches), medians over
+    the profiled steps.  FLOPs are the structurally non-zero ones."""
     by = {}
     for step in launches:
         acc = {}
         for r in step:
-            if r["kind"] in ("stage1", "stage2"):
+            if r["kind"] in ("stage1", "stage2", "fused"):
                 a = acc.setdefault(r["l"], [0.0, 0.0, 0])
                 a[0] += r["ms"]
-                a[1] += r["flops"]
+                a[1] += r["structural_flops"]
                 a[2] += 1
         for l, a in acc.items():
             by.setdefault(l, []).append(a)
@@ -241,10 +255,25 @@ def run_reference(args):
     w = workloads.WORKLOADS[args.workload]
     os.environ.setdefault("BAKRON_WORKLOAD_CACHE", os.path.join(tempfile.gettempdir(), "bakron_workloads"))
     W, A, B = workloads.generate(args.workload)
-    target = max(2.0, 40.0 / max(1, args.steps + args.warmup))
+    factors = oracle_factors(A, B)
+    # Every step solves the whole matrix when (steps + warm-up) such solves fit
+    # the budget (the run must end within a few minutes); otherwise each step
+    # takes the largest top-rows sub-problem that does, scaled (stated in the
+    # line's sample).
+    budget_s = 200.0
+    probe = cpu_baseline(W, A, B, w.bits, factors=factors, rows=min(w.m, 256))
+    full_s = w.m * w.n / probe["value"]
+    rows = None
+    if full_s * (args.steps + args.warmup) <= budget_s:
+        rows = w.m
+    else:
+        per_step = budget_s / (args.steps + args.warmup)
+        rows = min(w.m, 256)
+        while rows < w.m and full_s * (2 * rows) * w.n * (2 * rows + w.n) / (w.m * w.n * (w.m + w.n)) <= per_step:
+            rows = min(w.m, 2 * rows)
     for _ in range(args.warmup):
-        cpu_baseline(W, A, B, w.bits, target_s=target)
-    vals = [cpu_baseline(W, A, B, w.bits, target_s=target) for _ in range(args.steps)]
+        cpu_baseline(W, A, B, w.bits, factors=factors, rows=rows)
+    vals = [cpu_baseline(W, A, B, w.bits, factors=factors, rows=rows) for _ in range(args.steps)]
     v = statistics.median(x["value"] for x in vals)
     ms = w.m * w.n / v * 1e3
     cb = dict(vals[-1])
@@ -371,11 +400,12 @@ def main():
     plan = bk.plan_stats(m, n)
     bf16, hbm, src = peaks()
     tf32_peak = bf16 * TF32_PER_BF16
-    gemm_ms = pr["stage1_ms"] + pr["stage2_ms"]
+    gemm_ms = pr["stage1_ms"] + pr["stage2_ms"] + pr["fused_ms"]
     # a one-tile-diagonal problem (m, n <= 128) has no band products
-    achieved = 3.0 * plan["update_flops"] / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
+    achieved = 3.0 * plan["structural_flops"] / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
     leaf_bytes = LEAF_BYTES_PER_WEIGHT * m * n
-    launches_per_step = 4 + int(plan["leaves"]) + 2 * int(plan["nodes"])
+    launches_per_step = int(pr["prep_launches"] + pr["leaf_launches"] + pr["stage1_launches"] +
+                            pr["stage2_launches"] + pr["fused_launches"])
 
     # e2e through the host-buffer entry point: H2D of W, LA, LB and D2H of V,
     # codes, scales inside the timed region, every step
@@ -460,17 +490,22 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_block(w, args),
             "roofline": {
-                "bound": "tensor", "kernel": "band_tc_kernel (stage 1 + stage 2 band products)",
+                "bound": "tensor",
+                "kernel": "band products: band_tc_kernel (stage 1, stage 2) and band_fused_kernel (both stages)",
                 "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s", "frac": achieved / tf32_peak,
                 "traffic": (BAND_TRAFFIC["bytes_per_launch"]
                             if BAND_TRAFFIC["sources_sha256"] == band_sources_sha256() else None),
                 "traffic_source": BAND_TRAFFIC["profile"],
                 "peak_source": f"{src} bf16 {bf16:.1f} TFLOP/s x {TF32_PER_BF16:.4f} (nominal TF32:BF16), burst",
-                "flops_per_step": 3.0 * plan["update_flops"],
-                "flops_note": "3 TF32 MMAs per multiply-add (3xTF32) x algorithmic tile-product FLOPs of the schedule",
-                "band_ms_per_step": gemm_ms},
+                "flops_per_step": 3.0 * plan["structural_flops"],
+                "flops_note": "3 TF32 MMAs per multiply-add (3xTF32) x the structurally non-zero multiply-adds of "
+                              "the schedule's band products (2 per multiply-add)",
+                "flops_issued_per_step": 3.0 * plan["update_flops"],
+                "flops_issued_note": "tile-dense: the zero upper triangles of the diagonal factor tiles included",
+                "band_ms_per_step": gemm_ms,
+                "fused_nodes_per_step": int(pr["fused_launches"])},
             "band_levels": levels,
-            "leaf": {"kernel": LEAF_KERNELS[leaf][0], "structure": leaf, "tune_ms": dict(zip((1, 2, 3, 4), leaf_tune_ms)),
+            "leaf": {"kernel": LEAF_KERNELS[leaf][0], "structure": leaf, "tune_ms": dict(zip(bk.LEAF_STRUCTURES, leaf_tune_ms)),
                      "ms_per_step": pr["leaf_ms"],
                      "launches_per_step": pr["leaf_launches"],
                      "achieved_gbs": leaf_bytes / (pr["leaf_ms"] / 1e3) / 1e9, "hbm_peak_gbs": hbm,

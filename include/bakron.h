@@ -21,8 +21,9 @@
  *     pinned memory buffers, never frees or retains caller memory; all scratch
  *     lives in the caller's workspace, whose size the *_workspace_size query
  *     gives.  (Exceptions, all driver-side: bakron_solve_noalloc's fixed
- *     scratch array, reserved when the library loads; and in CUDA graph mode a
- *     private stream per calling thread and the cached executable graphs.)
+ *     scratch array, reserved on a device by the first call there; and in
+ *     CUDA graph mode a private stream per calling thread and the cached
+ *     executable graphs.)
  *   - Calls are stream-ordered and asynchronous on `stream` (a cudaStream_t;
  *     NULL = legacy default stream).  Argument errors are returned at once and
  *     nothing is enqueued.  Errors found on the device (non-SPD pivot,
@@ -85,9 +86,10 @@ typedef struct {
 } bakron_quantizer_t;
 
 /* Solver configuration (NULL = defaults; zero fields take defaults).
- * The environment can change the defaults of four fields: BAKRON_LEAF (0..4),
- * BAKRON_GEMM (0..1), BAKRON_TIMEOUT_MS (1..600000) and BAKRON_GRAPH (0..1,
- * ignored when profile = 1); a non-zero field set by the caller wins.  A
+ * The environment can change the defaults of five fields: BAKRON_LEAF (0..5),
+ * BAKRON_GEMM (0..1), BAKRON_TIMEOUT_MS (1..600000), BAKRON_GRAPH (0..1,
+ * ignored when profile = 1) and BAKRON_FUSE (1..65535, the default
+ * fuse_width); a non-zero field set by the caller wins.  A
  * variable that is set but not an integer in its range makes every call that
  * reads a config return BAKRON_ERR_INVALID_ARG.
  *   tile        side T of the square tiles whose anti-diagonals the recursion
@@ -114,12 +116,14 @@ typedef struct {
     int32_t profile;  /* 1: time every kernel class with CUDA events on `stream`;
                          the call then synchronises `stream` before returning and
                          the durations are read with bakron_get_profile(). */
-    int32_t leaf;     /* leaf sweep structure: 0 = default (3); 1 = each tile as
+    int32_t leaf;     /* leaf sweep structure: 0 = default (5); 1 = each tile as
                          2 x 2 sub-tiles of 64 swept by the whole CTA; 2 = one
                          anti-diagonal sweep over the whole 128 x 128 tile; 3 =
                          4 x 4 sub-tiles of 32, each swept by three warps; 4 =
-                         2 x 2 sub-tiles of 64, each swept by six warps
-                         (bakron_tune_leaf picks one by measurement). */
+                         2 x 2 sub-tiles of 64, each swept by six warps; 5 = as
+                         3 with each tile on a cluster of four CTAs, one per
+                         row block of sub-tiles (bakron_tune_leaf picks one by
+                         measurement). */
     int32_t b_identity; /* 1: B = I (one-sided GPTQ with Hessian A, the case the
                            two-sided solve reduces to when B = I).  LB_dev may be
                            NULL and is not read; rows are independent, so the
@@ -128,6 +132,13 @@ typedef struct {
                            instead of tile diagonals.  The leaf and gemm
                            fields are ignored (the update always runs on the
                            tensor cores, 3xTF32). */
+    int32_t fuse_width; /* recursion nodes at most this many tile diagonals
+                           wide run both band products in one launch, one CTA
+                           per target tile, with X kept in tensor memory
+                           (stage 1 and stage 2 fused); wider nodes run them as
+                           two launches.  0 = default (2), 1 = never fuse,
+                           2..65535 = that width.  Ignored with gemm = 1 and on
+                           the one-sided path. */
 } bakron_config_t;
 
 /* Per-kernel-class device time of the latest profiled bakron_solve on the
@@ -137,20 +148,26 @@ typedef struct {
 typedef struct {
     double prep_ms, leaf_ms, stage1_ms, stage2_ms, total_ms;
     int64_t prep_launches, leaf_launches, stage1_launches, stage2_launches;
+    double fused_ms;        /* nodes whose two band products ran as one launch */
+    int64_t fused_launches;
 } bakron_profile_t;
 bakron_status_t bakron_get_profile(bakron_profile_t *out);
 
 /* One launch of the latest profiled bakron_solve on the calling host thread,
  * in launch order: kind 0 prep (the four preparation kernels together), 1 leaf
  * sweep of tile diagonal k, 2 / 3 stage 1 / stage 2 band product of the
- * recursion node over tile diagonals [k, k+l) split at k+h; ms its
+ * recursion node over tile diagonals [k, k+l) split at k+h, 4 both band
+ * products of such a node in one fused launch; ms its
  * CUDA-event interval; flops the algorithmic FLOPs of a band product (2 T^3
- * per 128 x 128 x 128 tile product; 0 for other kinds).  One-sided path:
+ * per 128 x 128 x 128 tile product, both products for kind 4; 0 for other
+ * kinds).  One-sided path:
  * kind 1 is the leaf of column block k, kind 2 the update of column blocks
  * [k+h, k+l) by blocks [k, k+h). */
 typedef struct {
     int32_t kind, k, h, l;
     double ms, flops;
+    double structural_flops; /* flops without the structurally zero upper
+                                triangles of the diagonal factor tiles */
 } bakron_profile_launch_t;
 /* Copies min(count, cap) records to `out` (may be NULL) and returns count. */
 int64_t bakron_get_profile_launches(bakron_profile_launch_t *out, int64_t cap);
@@ -209,11 +226,12 @@ bakron_status_t bakron_solve(const float *W_dev, int64_t m, int64_t n, const flo
                              const bakron_config_t *cfg, bakron_stream_t stream);
 
 /* Leaf structure picked by measurement (the schedule's leaf size: 4 x 4
- * sub-tiles of 32, 2 x 2 of 64, or the whole 128 x 128 tile per sweep).  Runs
+ * sub-tiles of 32, 2 x 2 of 64, or the whole 128 x 128 tile per sweep; one
+ * CTA or a cluster of four per tile).  Runs
  * bakron_solve on the caller's problem once per structure after one warm-up
  * solve, timing each with CUDA events on `stream` (the call synchronises
  * `stream`), and writes the fastest structure (a bakron_config_t.leaf value,
- * 1..4) to *leaf_out and the four times in ms to ms_out[0..3] (leaf 1..4;
+ * 1..5) to *leaf_out and the five times in ms to ms_out[0..4] (leaf 1..5;
  * ms_out may be NULL).  Arguments as for bakron_solve; cfg->leaf is ignored
  * and cfg->profile must be 0.  V, codes and scales hold the last solve's
  * results (all structures give the same codes up to rounding ties).  Device
@@ -269,20 +287,30 @@ bakron_status_t bakron_solve_host(const float *W_host, int64_t m, int64_t n, con
  * memory at start-up and forbid allocation afterwards so that their footprint
  * stays fixed.  They cannot obtain the workspace bakron_solve asks for.  This
  * entry point runs the same solve with its workspace in a device array that
- * the library itself declares: BAKRON_NOALLOC_SCRATCH_BYTES bytes, reserved
- * on every GPU that loads the library and held until the process exits.
+ * the library itself declares: BAKRON_NOALLOC_SCRATCH_BYTES bytes per GPU,
+ * held until the process exits.
  *
  *   Arguments as bakron_solve, without ws/ws_bytes.  The problem must fit
  *   the array: bakron_solve_workspace_size(m, n, cfg) <=
  *   BAKRON_NOALLOC_SCRATCH_BYTES (true for any m, n <= 512); larger problems
  *   return BAKRON_ERR_WORKSPACE and nothing is enqueued.  cfg->profile must be
- *   0 (BAKRON_ERR_INVALID_ARG otherwise).
+ *   0 (BAKRON_ERR_INVALID_ARG otherwise).  The kernels are always launched
+ *   directly: cfg->use_graph and BAKRON_GRAPH are ignored here, since graph
+ *   capture and instantiation make the driver allocate.
  *   device_status_host: NULL keeps the call asynchronous (device-detected
  *   errors are then not reported); otherwise the call synchronises `stream`
- *   and stores the device status (a bakron_status_t value) there.
- *   The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any
- *   stream capture.  The library calls no cudaMalloc or cudaFree here.
+ *   and stores the device status (a bakron_status_t value) there, and a
+ *   `stream` that is being captured into a graph is refused with
+ *   BAKRON_ERR_INVALID_ARG before anything is enqueued.
+ *   Set-up on the first call on each device: the library looks up the array's
+ *   device address (once per device, with that device current).  Under CUDA's
+ *   default lazy module loading that first call is also when the driver loads
+ *   the array's code module and reserves the array on that device (at library
+ *   load only with CUDA_MODULE_LOADING=EAGER), so it can fail with
+ *   BAKRON_ERR_CUDA if the device's memory is already full.  Make one call on
+ *   every device at start-up, before the caller fixes its memory and before
+ *   any stream capture.  After that the library calls no cudaMalloc or
+ *   cudaFree here.
  *   Every call on a device shares the one array and leaves its contents
  *   behind; the solve clears what must start at zero.  Calls that overlap on
  *   the GPU (other streams, other host threads) race on the array: issue them
@@ -294,13 +322,16 @@ bakron_status_t bakron_solve_noalloc(const float *W_dev, int64_t m, int64_t n, c
                                      bakron_stream_t stream, int32_t *device_status_host);
 
 /* ------------------------------------------------------------ proxy loss */
-/* Bytes of workspace bakron_proxy_loss needs. */
+/* Bytes of workspace bakron_proxy_loss needs: the status block plus one FP64
+ * partial sum per 64 x 64 tile of W. */
 size_t bakron_proxy_loss_workspace_size(int64_t m, int64_t n);
 
 /* Proxy loss l = tr((W-V)^T B (W-V) A) = ||B^{1/2}(V-W)A^{1/2}||_F^2
  * (Corollary 3.4's distortion; the review's "||vec(W)-vec(V)||_H^2",
  * H = A (x) B).  W_dev, V_dev m x n; A_dev n x n; B_dev m x m (symmetric).
- * Products in FP32 on the GPU, final reduction in FP64.  The result is
+ * Products in FP32 on the GPU, reduction in FP64: each 64 x 64 tile's sum
+ * goes to its own slot in the workspace and the slots are added in a fixed
+ * order, so repeated calls give bit-identical results.  The result is
  * written to *out_dev (a device double) and, if out_host is not NULL, also
  * to *out_host, in which case the call synchronises `stream`. */
 bakron_status_t bakron_proxy_loss(const float *W_dev, const float *V_dev, const float *A_dev,
@@ -324,6 +355,22 @@ bakron_status_t bakron_get_status(void *ws_dev, size_t ws_bytes, bakron_stream_t
 bakron_status_t bakron_selftest_wait_timeout(int32_t timeout_ms, void *ws_dev, size_t ws_bytes,
                                              bakron_stream_t stream);
 
+/* Failure-detection self-test of the band-product kernel's abort path: runs
+ * the stage-1 band kernel (the tcgen05 3xTF32 product, two CTAs) on a small
+ * problem laid out in ws_dev with its copy-issuing thread told to issue
+ * nothing, so the MMA issuer's and the epilogue's bounded waits run out after
+ * timeout_ms (1..10000).  The kernel then takes the path a real timeout takes:
+ * records BAKRON_ERR_DEVICE_TIMEOUT in the status word at the start of ws_dev
+ * (where = 2001 for the MMA issuer, 3001 for the epilogue; cleared first),
+ * stops, drains what it issued (nothing), frees its tensor memory and exits,
+ * leaving the context usable.  ws_dev: at least
+ * bakron_selftest_band_abort_workspace_size() bytes, 16-byte aligned; its
+ * contents are not read.  Asynchronous on `stream`: read the result with
+ * bakron_get_status. */
+size_t bakron_selftest_band_abort_workspace_size(void);
+bakron_status_t bakron_selftest_band_abort(int32_t timeout_ms, void *ws_dev, size_t ws_bytes,
+                                           bakron_stream_t stream);
+
 /* Static description of a status code. */
 const char *bakron_status_string(bakron_status_t status);
 
@@ -338,6 +385,10 @@ typedef struct {
     int64_t nodes, leaves;
     double update_flops;   /* algorithmic (tile-dense) FLOPs of all band products */
     double stage1_flops, stage2_flops;
+    double structural_flops; /* 2 x the structurally non-zero multiply-adds of
+                                all band products: a product with the factor
+                                tile on the diagonal (lower triangular) counts
+                                T^2 (T+1)/2 of them instead of T^3 */
 } bakron_plan_stats_t;
 bakron_status_t bakron_plan_stats(int64_t m, int64_t n, const bakron_config_t *cfg,
                                   bakron_plan_stats_t *out);

@@ -41,7 +41,7 @@ def oracle_factors(A, B):
     return LA, LB
 
 
-def gpu_solve(W, LA32, LB32, bits, gemm=0, row_scale=None, leaf=0):
+def gpu_solve(W, LA32, LB32, bits, gemm=0, row_scale=None, leaf=0, fuse_width=0):
     import torch
 
     import two_sided_gptq_b200 as bk
@@ -52,26 +52,83 @@ def gpu_solve(W, LA32, LB32, bits, gemm=0, row_scale=None, leaf=0):
     LBd = None if LB32 is None else torch.from_numpy(np.ascontiguousarray(LB32)).to(dev)  # None: B = I
     wt = torch.empty_like(Wd)
     rs = None if row_scale is None else torch.from_numpy(np.asarray(row_scale, np.float32)).to(dev)
-    V, codes, scales = bk.solve(Wd, LAd, LBd, bits=bits, gemm=gemm, wt_out=wt, row_scale=rs, leaf=leaf)
+    V, codes, scales = bk.solve(Wd, LAd, LBd, bits=bits, gemm=gemm, wt_out=wt, row_scale=rs, leaf=leaf,
+                                fuse_width=fuse_width)
     torch.cuda.synchronize()
     return V.cpu().numpy(), codes.cpu().numpy().astype(np.int32), scales.cpu().numpy(), wt.cpu().numpy()
 
 
-def check_solve(W, LA32, LB32, bits, gemm=0, row_scale=None, label="", leaf=0):
+CANARY = 0xA5  # guard byte around every buffer of a canary-checked solve
+GUARD = 4096  # guard bytes on each side (a multiple of 256 keeps 16-byte alignment)
+
+
+def gpu_solve_canaries(W, LA32, LB32, bits, leaf=0, fuse_width=0, gemm=0):
+    """The GPU solve with its workspace and outputs (V, codes, steps) carved
+    out of larger buffers whose guard zones, and the gap after the
+    workspace's 256-byte status block (the next buffer starts 1 KiB in), hold
+    CANARY bytes: a substitute for an out-of-bounds checker.  Asserts that no
+    guard byte changed; returns host arrays like gpu_solve (no pre-rounding
+    values)."""
+    import torch
+
+    import two_sided_gptq_b200 as bk
+
+    m, n = W.shape
+
+    def guarded(nbytes):
+        raw = torch.full((nbytes + 2 * GUARD,), CANARY, dtype=torch.uint8, device="cuda")
+        return raw, raw[GUARD:GUARD + nbytes]
+
+    ws_bytes = bk.solve_workspace_size(m, n, gemm)
+    raw_ws, ws = guarded(ws_bytes)
+    raw_v, v = guarded(4 * m * n)
+    raw_c, c = guarded(m * n)
+    raw_s, sc = guarded(4 * m)
+    V = v.view(torch.float32).view(m, n)
+    codes = c.view(torch.int8).view(m, n)
+    scales = sc.view(torch.float32)
+    Wd = torch.from_numpy(np.ascontiguousarray(W)).cuda()
+    LAd = torch.from_numpy(np.ascontiguousarray(LA32)).cuda()
+    LBd = None if LB32 is None else torch.from_numpy(np.ascontiguousarray(LB32)).cuda()
+    bk.solve(Wd, LAd, LBd, bits=bits, gemm=gemm, ws=ws, out=(V, codes, scales), leaf=leaf, fuse_width=fuse_width)
+    torch.cuda.synchronize()
+    for name, raw, size in (("workspace", raw_ws, ws_bytes), ("V", raw_v, 4 * m * n), ("codes", raw_c, m * n),
+                            ("steps", raw_s, 4 * m)):
+        h = raw.cpu().numpy()
+        assert np.all(h[:GUARD] == CANARY), f"write before the {name} buffer"
+        assert np.all(h[GUARD + size:] == CANARY), f"write after the {name} buffer"
+    gap = raw_ws[GUARD + 256:GUARD + 1024].cpu().numpy()
+    assert np.all(gap == CANARY), "write into the gap after the status block"
+    return V.cpu().numpy(), codes.cpu().numpy().astype(np.int32), scales.cpu().numpy()
+
+
+def check_solve(W, LA32, LB32, bits, gemm=0, row_scale=None, label="", leaf=0, fuse_width=0):
     """Run the GPU solve on (W, LA32, LB32) and check it teacher-forced
     against the oracle using the same fp32 factors (widened to FP64).
     Returns the report dict (asserts the contract)."""
+    V, codes, s_gpu, wt_gpu = gpu_solve(W, LA32, LB32, bits, gemm, row_scale, leaf, fuse_width)
+    return check_outputs(W, LA32, LB32, bits, V, codes, s_gpu, wt_gpu, row_scale, label)
+
+
+def check_outputs(W, LA32, LB32, bits, V, codes, s_gpu, wt_gpu=None, row_scale=None, label=""):
+    """Check one solve's outputs (host arrays: V fp32, codes int, steps fp32,
+    optionally the pre-rounding values) teacher-forced against the oracle on
+    the same fp32 factors.  LB32 None means B = I.  Returns the report dict
+    (asserts the contract)."""
     qmin, qmax = oracle.grid(bits)
-    V, codes, s_gpu, wt_gpu = gpu_solve(W, LA32, LB32, bits, gemm, row_scale, leaf)
+    codes = np.asarray(codes).astype(np.int32)
     s = oracle.scales(W, qmax) if row_scale is None else np.asarray(row_scale, np.float32)
-    assert np.array_equal(s_gpu.view(np.uint32), s.view(np.uint32)), f"{label}: steps differ"
+    assert np.array_equal(np.asarray(s_gpu, np.float32).view(np.uint32), s.view(np.uint32)), f"{label}: steps differ"
     LtA = oracle.normalize(LA32.astype(np.float64))
     # B = I (the one-sided path): the pull with an identity row factor
     LtB = np.eye(W.shape[0]) if LB32 is None else oracle.normalize(LB32.astype(np.float64))
     r = oracle.forced_check(W, LtA, LtB, s, qmin, qmax, codes, tie_eps=TIE_EPS)
     m, n = W.shape
     r["label"] = label
-    r["wt_max_abs_err"] = float(np.abs(wt_gpu.astype(np.float64) - r["Wt"]).max())
+    if wt_gpu is not None:
+        r["wt_max_abs_err"] = float(np.abs(wt_gpu.astype(np.float64) - r["Wt"]).max())
+    else:
+        r["wt_max_abs_err"] = float("nan")
     r["wt_scale"] = float(np.abs(r["Wt"]).max())
     # codes within the grid, V = s * code exactly in fp32
     assert codes.min() >= qmin and codes.max() <= qmax

@@ -53,7 +53,8 @@ def test_host_only_queries(lib):
     assert ws >= 4 * (5 * 4096 * 4096 + 6 * 4096 * 4096)
     assert lib.bakron_solve_host_workspace_size(100, 70, None) > lib.bakron_solve_workspace_size(100, 70, None)
     assert lib.bakron_factor_workspace_size(300, 200) >= 2 * 300 * 300 * 8
-    assert lib.bakron_proxy_loss_workspace_size(3, 4) == 256
+    assert lib.bakron_proxy_loss_workspace_size(3, 4) == 1024 + 8  # status block (aligned) + one tile sum
+    assert lib.bakron_proxy_loss_workspace_size(4096, 4096) == 1024 + 8 * 64 * 64
     bad = _native.Config(64, 0, 0, 0, None)  # unsupported tile
     assert lib.bakron_solve_workspace_size(10, 10, ctypes.byref(bad)) == 0
 
@@ -94,6 +95,11 @@ def test_argument_errors_return_before_any_device_work(lib):
     cfg = _native.Config(0, 0, 0, 0, None, 0, 0, 2)
     a[11] = ctypes.byref(cfg)
     assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
+    # fuse_width is 0 (default), 1 (never) or a width up to 65535
+    for fw in (-1, 65536):
+        cfg = _native.Config(0, 0, 0, 0, None, 0, 0, 0, fw)
+        a[11] = ctypes.byref(cfg)
+        assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
     a = list(args())
     a[4] = None
     assert lib.bakron_solve(*a) == _native.Status.ERR_INVALID_ARG
@@ -107,11 +113,19 @@ def test_argument_errors_return_before_any_device_work(lib):
     assert lib.bakron_selftest_wait_timeout(5, None, 256, None) == _native.Status.ERR_WORKSPACE
     assert lib.bakron_selftest_wait_timeout(5, fake, 255, None) == _native.Status.ERR_WORKSPACE
     assert lib.bakron_selftest_wait_timeout(5, fake + 8, 256, None) == _native.Status.ERR_ALIGNMENT
+    need = lib.bakron_selftest_band_abort_workspace_size()
+    assert need >= 256 + 6 * 256 * 256 * 4
+    assert lib.bakron_selftest_band_abort(0, fake, need, None) == _native.Status.ERR_INVALID_ARG
+    assert lib.bakron_selftest_band_abort(5, None, need, None) == _native.Status.ERR_WORKSPACE
+    assert lib.bakron_selftest_band_abort(5, fake, need - 1, None) == _native.Status.ERR_WORKSPACE
+    assert lib.bakron_selftest_band_abort(5, fake + 8, need, None) == _native.Status.ERR_ALIGNMENT
     assert lib.bakron_factor(fake, -1, fake, 4, fake, fake, fake, 1 << 30, None) == _native.Status.ERR_INVALID_ARG
     assert lib.bakron_factor(fake, 4, fake, 4, fake + 8, fake, fake, 1 << 30, None) == _native.Status.ERR_ALIGNMENT
     assert lib.bakron_factor(fake, 4, fake, 4, fake, fake, fake, 16, None) == _native.Status.ERR_WORKSPACE
     assert lib.bakron_proxy_loss(fake, fake, fake, fake, 0, 4, fake, None, fake, 256, None) == \
         _native.Status.ERR_INVALID_ARG
+    assert lib.bakron_proxy_loss(fake, fake, fake, fake, 4, 4, fake, None, fake, 1031, None) == \
+        _native.Status.ERR_WORKSPACE
 
 
 def _brute_schedule_flops(Mt, Nt, T=128):
@@ -124,6 +138,7 @@ def _brute_schedule_flops(Mt, Nt, T=128):
     stage 2 one per needed X(I, J') with I <= I' for every target (I', J')."""
     tiles = [(I, J) for I in range(Mt) for J in range(Nt)]
     total = [0.0, 0.0]
+    diag = [0, 0]  # products whose factor tile is on the diagonal (lower triangular)
 
     def rec(k, l):
         if l <= 1:
@@ -139,13 +154,16 @@ def _brute_schedule_flops(Mt, Nt, T=128):
                     need.add((I, J2))
         for (I, J2) in need:
             total[0] += sum(1 for (a, b) in src if a == I and b <= J2)
+            diag[0] += sum(1 for (a, b) in src if a == I and b == J2)
         for (I2, J2) in tgt:
             total[1] += sum(1 for (I, Jx) in need if Jx == J2 and I <= I2)
+            diag[1] += sum(1 for (I, Jx) in need if Jx == J2 and I == I2)
         rec(k + h, l - h)
 
     rec(0, Mt + Nt - 1)
     f = 2.0 * T ** 3
-    return total[0] * f, total[1] * f
+    structural = (total[0] + total[1] - diag[0] - diag[1]) * f + (diag[0] + diag[1]) * T * T * (T + 1)
+    return total[0] * f, total[1] * f, structural
 
 
 @pytest.mark.parametrize("shape", [(1, 1), (1, 5), (4, 1), (3, 3), (5, 8), (9, 4), (7, 11)])
@@ -155,11 +173,12 @@ def test_plan_stats_matches_bruteforce_count(lib, shape):
     Mt, Nt = shape
     s = _native.PlanStats()
     assert lib.bakron_plan_stats(Mt * 128, Nt * 128, None, ctypes.byref(s)) == 0
-    f1, f2 = _brute_schedule_flops(Mt, Nt)
+    f1, f2, fs = _brute_schedule_flops(Mt, Nt)
     assert s.tiles_m == Mt and s.tiles_n == Nt and s.tile_diagonals == Mt + Nt - 1
     assert s.leaves == Mt + Nt - 1 and s.nodes == Mt + Nt - 2
     assert s.stage1_flops == pytest.approx(f1, rel=0, abs=0)
     assert s.stage2_flops == pytest.approx(f2, rel=0, abs=0)
+    assert s.structural_flops == pytest.approx(fs, rel=0, abs=0)
 
 
 def test_plan_stats_4096_cubic_work(lib):
@@ -233,13 +252,14 @@ def _plan_status_under_env(env):
 
 
 def test_environment_overrides_are_validated():
-    """BAKRON_LEAF / _GEMM / _TIMEOUT_MS / _GRAPH change defaults; a malformed
+    """BAKRON_LEAF / _GEMM / _TIMEOUT_MS / _GRAPH / _FUSE change defaults; a malformed
     or out-of-range value makes config-reading calls fail with INVALID_ARG."""
     from two_sided_gptq_b200 import _native
 
     ok, bad = _native.Status.OK, _native.Status.ERR_INVALID_ARG
-    assert _plan_status_under_env({"BAKRON_LEAF": "4", "BAKRON_GEMM": "1", "BAKRON_TIMEOUT_MS": "50",
-                                   "BAKRON_GRAPH": "1"}) == ok
-    for env in ({"BAKRON_LEAF": "5"}, {"BAKRON_GEMM": "2"}, {"BAKRON_TIMEOUT_MS": "0"},
-                {"BAKRON_TIMEOUT_MS": "12ms"}, {"BAKRON_GRAPH": "-1"}):
+    assert _plan_status_under_env({"BAKRON_LEAF": "5", "BAKRON_GEMM": "1", "BAKRON_TIMEOUT_MS": "50",
+                                   "BAKRON_GRAPH": "1", "BAKRON_FUSE": "8"}) == ok
+    for env in ({"BAKRON_LEAF": "6"}, {"BAKRON_GEMM": "2"}, {"BAKRON_TIMEOUT_MS": "0"},
+                {"BAKRON_TIMEOUT_MS": "12ms"}, {"BAKRON_GRAPH": "-1"}, {"BAKRON_FUSE": "0"},
+                {"BAKRON_FUSE": "65536"}):
         assert _plan_status_under_env(env) == bad, env

@@ -40,3 +40,30 @@ def test_bounded_wait_gives_up_and_context_stays_usable():
     W, A, B = workloads.random_problem(129, 257, seed=3)
     LA, LB = oracle_factors(A, B)
     check_solve(W, LA, LB, 4, label="after timeout")
+
+
+def test_band_kernel_abort_path_records_timeout_and_context_stays_usable():
+    """The band-product kernel itself (tcgen05 MMAs, TMEM, TMA pipeline) with
+    its copy-issuing thread told to issue nothing: the MMA issuer's and the
+    epilogue's bounded waits run out with nothing in flight; the kernel records
+    the timeout with the waiting role, frees its tensor memory and exits."""
+    import torch
+
+    import two_sided_gptq_b200 as bk
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    ws = bk.selftest_band_abort(5)
+    e1.record()
+    torch.cuda.synchronize()
+    code, where = (int(x) for x in ws[:8].view(torch.int32).cpu())
+    assert code == int(bk.Status.ERR_DEVICE_TIMEOUT)
+    assert where in (2001, 3001), where  # the MMA issuer or the epilogue gave up
+    assert bk.get_status(ws) == bk.Status.ERR_DEVICE_TIMEOUT
+    assert bk.get_status(ws) == bk.Status.OK
+    assert 4.5 <= e0.elapsed_time(e1) < 500
+    # tensor memory was released and the context is intact: a full solve with
+    # tensor-core band products right after matches the oracle
+    W, A, B = workloads.random_problem(300, 390, seed=5)
+    LA, LB = oracle_factors(A, B)
+    check_solve(W, LA, LB, 4, label="after band abort")

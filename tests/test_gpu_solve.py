@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 import workloads
-from parity import check_solve, gpu_solve, oracle_factors
+from parity import check_outputs, check_solve, gpu_solve, gpu_solve_canaries, oracle_factors
 
 pytestmark = pytest.mark.gpu
 
@@ -62,6 +62,20 @@ def test_ragged_shapes(shape, gemm):
     check_solve(W, LA, LB, 4, gemm=gemm, label=f"{m}x{n}/gemm{gemm}")
 
 
+@pytest.mark.parametrize("leaf", [3, 5])
+@pytest.mark.parametrize("shape", RAGGED)
+def test_ragged_shapes_write_only_their_buffers(shape, leaf):
+    """Canary-padded workspace and outputs (guard zones of a known byte
+    pattern before and after every buffer): no kernel of the solve writes
+    outside what it was given, on every ragged shape; the codes still pass
+    the oracle contract."""
+    m, n = shape
+    W, A, B = workloads.random_problem(m, n, seed=m * 1000 + n)
+    LA, LB = oracle_factors(A, B)
+    V, codes, s = gpu_solve_canaries(W, LA, LB, 4, leaf=leaf)
+    check_outputs(W, LA, LB, 4, V, codes, s, label=f"{m}x{n}/canary/leaf{leaf}")
+
+
 @pytest.mark.parametrize("bits", [2, 3, 8])
 def test_other_grids(bits):
     W, A, B = workloads.random_problem(300, 260, seed=bits)
@@ -110,8 +124,25 @@ def test_leaf_variants(case):
         W, A, B = workloads.random_problem(m, n, seed=m + 7 * n)
         LA, LB = oracle_factors(A, B)
         label = f"{m}x{n}"
-    for leaf in (1, 2, 3, 4):
+    for leaf in (1, 2, 3, 4, 5):
         check_solve(W, LA, LB, 4, leaf=leaf, label=f"{label}/leaf{leaf}")
+
+
+@pytest.mark.parametrize("case", ["mid", (300, 260), (129, 1000), (1000, 129), (640, 384)])
+def test_fused_node_widths(case):
+    """Both band products of a node in one launch (X in tensor memory) against
+    the two-launch form: the same oracle contract whether no node, the narrow
+    nodes (the default) or every node runs fused."""
+    if case == "mid":
+        W, A, B, LA, LB = named("mid")
+        label = "mid"
+    else:
+        m, n = case
+        W, A, B = workloads.random_problem(m, n, seed=3 * m + n)
+        LA, LB = oracle_factors(A, B)
+        label = f"{m}x{n}"
+    for fw in (1, 2, 0, 65535):
+        check_solve(W, LA, LB, 4, fuse_width=fw, label=f"{label}/fuse{fw}")
 
 
 @pytest.mark.slow
@@ -142,7 +173,7 @@ def test_tune_leaf_picks_a_measured_structure():
     W, A, B, LA, LB = named("mid")
     Wd, LAd, LBd = (torch.from_numpy(x).cuda() for x in (W, LA.astype(np.float32), LB.astype(np.float32)))
     leaf, ms = bk.tune_leaf(Wd, LAd, LBd, bits=4)
-    assert leaf in (1, 2, 3, 4) and all(t > 0 for t in ms)
+    assert leaf in (1, 2, 3, 4, 5) and all(t > 0 for t in ms)
     assert ms[leaf - 1] == min(ms)
     check_solve(W, LA, LB, 4, leaf=leaf, label=f"mid/tuned-leaf{leaf}")
 

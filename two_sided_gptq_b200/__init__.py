@@ -20,8 +20,12 @@ from ._native import BakronError, BatchItem, Config, PlanStats, Profile, Profile
 
 __all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_profile",
            "last_profile_launches", "tune_leaf", "tune_cache_key", "tune_cache_get", "tune_cache_put",
-           "solve_batch", "gram", "selftest_wait_timeout", "workspace", "get_status",
+           "solve_batch", "gram", "selftest_wait_timeout", "selftest_band_abort", "workspace", "get_status",
            "BakronError", "Status", "version", "library_path"]
+
+
+# bakron_config_t.leaf values bakron_tune_leaf times (one ms_out entry each)
+LEAF_STRUCTURES = (1, 2, 3, 4, 5)
 
 
 def _lib():
@@ -60,9 +64,9 @@ def _dev_f32(x, name):
     return x
 
 
-def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False, leaf=0, b_identity=False, graph=False):
+def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False, leaf=0, b_identity=False, graph=False, fuse_width=0):
     return Config(0, int(gemm), 1 if graph else 0, int(timeout_ms), _ptr(wt_out), 1 if profile else 0, int(leaf),
-                  1 if b_identity else 0)
+                  1 if b_identity else 0, int(fuse_width))
 
 
 def workspace(nbytes: int, device=None):
@@ -82,6 +86,19 @@ def selftest_wait_timeout(timeout_ms: int, ws, stream=None) -> None:
     ``Status.ERR_DEVICE_TIMEOUT`` in ``ws``; read it with :func:`get_status`."""
     check(_lib().bakron_selftest_wait_timeout(int(timeout_ms), _ptr(ws), ws.numel(), _stream(stream)),
           "bakron_selftest_wait_timeout")
+
+
+def selftest_band_abort(timeout_ms: int, ws=None, stream=None):
+    """Launch the band kernel's abort-path self-test (``bakron_selftest_band_abort``):
+    the stage-1 band kernel with no copies issued, whose bounded waits run out
+    after ``timeout_ms``.  Returns the workspace; its status word then reads
+    ``Status.ERR_DEVICE_TIMEOUT`` (read it with :func:`get_status`)."""
+    need = _lib().bakron_selftest_band_abort_workspace_size()
+    if ws is None:
+        ws = workspace(need)
+    check(_lib().bakron_selftest_band_abort(int(timeout_ms), _ptr(ws), ws.numel(), _stream(stream)),
+          "bakron_selftest_band_abort")
+    return ws
 
 
 def factor(A, B=None, *, stream=None, ws=None, check_status=True):
@@ -112,7 +129,8 @@ def solve_workspace_size(m: int, n: int, gemm: int = 0) -> int:
 
 
 def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None, out=None, stream=None,
-          wt_out=None, check_status=True, timeout_ms=0, profile=False, leaf=0, shrink_grid=0, graph=False):
+          wt_out=None, check_status=True, timeout_ms=0, profile=False, leaf=0, shrink_grid=0, graph=False,
+          fuse_width=0):
     """BaKron solve on device tensors.  Returns ``(V, codes, scales)``.
 
     ``LB=None`` selects the one-sided path (B = I: GPTQ with Hessian A, over
@@ -121,10 +139,12 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     ``gemm=0`` uses the tcgen05 3xTF32 band products, ``gemm=1`` the FP32
     CUDA-core ones; ``shrink_grid`` > 1 searches each row's step for the least
     round-to-nearest error over that many shrink factors in [1/2, 1]; ``leaf``
-    selects the leaf sweep structure (0 default,
+    selects the leaf sweep structure (0 default (5),
     1 two-level CTA-wide, 2 single-level, 3 three warps per 32 x 32
-    sub-tile, 4 six warps per 64 x 64 sub-tile; :func:`tune_leaf` picks one by
-    measurement).  ``graph=True`` captures the solve's launches for this
+    sub-tile, 4 six warps per 64 x 64 sub-tile, 5 as 3 with each tile on a
+    cluster of four CTAs; :func:`tune_leaf` picks one by measurement).  ``fuse_width`` (0 default, 1 never) runs the two band
+    products of recursion nodes at most that many tile diagonals wide as one
+    launch per target tile.  ``graph=True`` captures the solve's launches for this
     argument set into a CUDA graph on the first call and replays it on later
     calls with the same buffers.  ``out`` may supply ``(V, codes, scales)`` buffers and
     ``ws`` a workspace; ``check_status=False`` skips the synchronising status
@@ -139,7 +159,7 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     m, n = W.shape
     if LA.shape != (n, n) or (not one_sided and LB.shape != (m, m)):
         raise ValueError("LA must be n x n and LB m x m")
-    cfg = _config(gemm, timeout_ms, wt_out, profile, leaf, one_sided, graph)
+    cfg = _config(gemm, timeout_ms, wt_out, profile, leaf, one_sided, graph, fuse_width)
     if out is None:
         V = torch.empty((m, n), dtype=torch.float32, device=W.device)
         codes = torch.empty((m, n), dtype=torch.int8, device=W.device)
@@ -158,8 +178,9 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
 
 
 def tune_cache_key(m: int, n: int, bits: int, device_name: str) -> str:
-    """Key of a leaf-structure measurement in the autotune cache."""
-    return f"{int(m)}x{int(n)}/int{int(bits)}/{device_name}"
+    """Key of a leaf-structure measurement in the autotune cache (the library
+    version is part of it: a new build re-measures)."""
+    return f"{int(m)}x{int(n)}/int{int(bits)}/{device_name}/{version()}"
 
 
 def tune_cache_get(path: str, key: str):
@@ -174,7 +195,7 @@ def tune_cache_get(path: str, key: str):
             entry = json.load(f).get(key)
     except (OSError, ValueError):
         return None
-    if not isinstance(entry, dict) or entry.get("leaf") not in (1, 2, 3, 4):
+    if not isinstance(entry, dict) or entry.get("leaf") not in LEAF_STRUCTURES:
         return None
     return int(entry["leaf"]), [float(x) for x in entry.get("ms", [])]
 
@@ -204,7 +225,7 @@ def tune_cache_put(path: str, key: str, leaf: int, ms) -> None:
 def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, timeout_ms=0, cache=None):
     """Leaf structure chosen by measurement (``bakron_tune_leaf``): one timed
     solve per structure on this problem.  Returns ``(leaf, [ms_leaf1, ...,
-    ms_leaf4])``; pass ``leaf`` to :func:`solve`.
+    ms_leaf5])``; pass ``leaf`` to :func:`solve`.
 
     ``cache`` (or the ``BAKRON_TUNE_CACHE`` environment variable) names a JSON
     file keyed by (m, n, bits, GPU name): a stored measurement is returned
@@ -231,7 +252,7 @@ def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, time
         ws = workspace(lib.bakron_solve_workspace_size(m, n, ctypes.byref(cfg)), W.device)
     q = Quantizer(int(bits), 0, 0, None)
     leaf = ctypes.c_int32(0)
-    ms = (ctypes.c_double * 4)()
+    ms = (ctypes.c_double * len(LEAF_STRUCTURES))()
     st = _stream(stream)
     check(lib.bakron_tune_leaf(_ptr(W), m, n, _ptr(LA), _ptr(LB), ctypes.byref(q), _ptr(V), _ptr(codes),
                                _ptr(scales), _ptr(ws), ws.numel(), ctypes.byref(cfg), st, ctypes.byref(leaf), ms),
@@ -353,14 +374,17 @@ def last_profile() -> dict:
 
 def last_profile_launches() -> list:
     """Every launch of the latest ``solve(..., profile=True)`` on this thread, in
-    launch order: dicts with kind ("prep", "leaf", "stage1", "stage2"), the
-    recursion node (k, h, l) in tile diagonals, ms and algorithmic FLOPs."""
+    launch order: dicts with kind ("prep", "leaf", "stage1", "stage2", "fused":
+    both band products of a node in one launch), the recursion node (k, h, l)
+    in tile diagonals, ms, FLOPs (tile-dense) and structural FLOPs (without
+    the zero upper triangles of the diagonal factor tiles)."""
     lib = _lib()
     n = lib.bakron_get_profile_launches(None, 0)
     buf = (ProfileLaunch * max(1, n))()
     lib.bakron_get_profile_launches(buf, n)
-    kinds = ("prep", "leaf", "stage1", "stage2")
-    return [{"kind": kinds[r.kind], "k": r.k, "h": r.h, "l": r.l, "ms": r.ms, "flops": r.flops} for r in buf[:n]]
+    kinds = ("prep", "leaf", "stage1", "stage2", "fused")
+    return [{"kind": kinds[r.kind], "k": r.k, "h": r.h, "l": r.l, "ms": r.ms, "flops": r.flops,
+             "structural_flops": r.structural_flops} for r in buf[:n]]
 
 
 def plan_stats(m: int, n: int, one_sided: bool = False) -> dict:

@@ -45,27 +45,29 @@ class BatchItem(ctypes.Structure):
 class Config(ctypes.Structure):
     _fields_ = [("tile", ctypes.c_int32), ("gemm", ctypes.c_int32), ("use_graph", ctypes.c_int32),
                 ("timeout_ms", ctypes.c_int32), ("wt_out", ctypes.c_void_p), ("profile", ctypes.c_int32),
-                ("leaf", ctypes.c_int32), ("b_identity", ctypes.c_int32)]
+                ("leaf", ctypes.c_int32), ("b_identity", ctypes.c_int32), ("fuse_width", ctypes.c_int32)]
 
 
 class Profile(ctypes.Structure):
     _fields_ = [("prep_ms", ctypes.c_double), ("leaf_ms", ctypes.c_double), ("stage1_ms", ctypes.c_double),
                 ("stage2_ms", ctypes.c_double), ("total_ms", ctypes.c_double),
                 ("prep_launches", ctypes.c_int64), ("leaf_launches", ctypes.c_int64),
-                ("stage1_launches", ctypes.c_int64), ("stage2_launches", ctypes.c_int64)]
+                ("stage1_launches", ctypes.c_int64), ("stage2_launches", ctypes.c_int64),
+                ("fused_ms", ctypes.c_double), ("fused_launches", ctypes.c_int64)]
 
 
 class PlanStats(ctypes.Structure):
     _fields_ = [("tiles_m", ctypes.c_int64), ("tiles_n", ctypes.c_int64), ("tile_diagonals", ctypes.c_int64),
                 ("nodes", ctypes.c_int64), ("leaves", ctypes.c_int64), ("update_flops", ctypes.c_double),
-                ("stage1_flops", ctypes.c_double), ("stage2_flops", ctypes.c_double)]
+                ("stage1_flops", ctypes.c_double), ("stage2_flops", ctypes.c_double),
+                ("structural_flops", ctypes.c_double)]
 
 
 # name -> (restype, argtypes); every function declared in include/bakron.h
 _vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
 class ProfileLaunch(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("k", ctypes.c_int32), ("h", ctypes.c_int32), ("l", ctypes.c_int32),
-                ("ms", ctypes.c_double), ("flops", ctypes.c_double)]
+                ("ms", ctypes.c_double), ("flops", ctypes.c_double), ("structural_flops", ctypes.c_double)]
 
 
 SIGNATURES = {
@@ -82,6 +84,8 @@ SIGNATURES = {
                                          _sz, _vp]),
     "bakron_get_status": (ctypes.c_int, [_vp, _sz, _vp]),
     "bakron_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int32, _vp, _sz, _vp]),
+    "bakron_selftest_band_abort_workspace_size": (_sz, []),
+    "bakron_selftest_band_abort": (ctypes.c_int, [ctypes.c_int32, _vp, _sz, _vp]),
     "bakron_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bakron_plan_stats": (ctypes.c_int, [_i64, _i64, ctypes.POINTER(Config), ctypes.POINTER(PlanStats)]),
     "bakron_version": (ctypes.c_char_p, []),

@@ -26,17 +26,27 @@ using namespace bakron;
 
 namespace {
 
-constexpr const char *kVersion = "bakron-b200 0.1";
+constexpr const char *kVersion = "bakron-b200 0.2";
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Leaf structures bakron_tune_leaf times (bakron_config_t.leaf 1..5).
+constexpr int kLeafStructures = 5;
+
+// Nodes at most this many tile diagonals wide run fused by default (measured
+// on B200 at 4096^2: width 2 trims the profiled band time, wider fusing is
+// slower than two launches).
+constexpr int kDefaultFuseWidth = 2;
+
 struct Config {
-    int tile = kTile, gemm = 0, use_graph = 0, timeout_ms = 200, profile = 0, leaf = 2, b_identity = 0;
+    // leaf: structure 5 (a cluster of four CTAs per tile), the fastest measured
+    int tile = kTile, gemm = 0, use_graph = 0, timeout_ms = 200, profile = 0, leaf = 4, b_identity = 0;
+    int fuse_width = kDefaultFuseWidth;
     float *wt_out = nullptr;
 };
 
 // Event-pair timing of kernel classes (profile mode): kind 0 prep, 1 leaf,
-// 2 stage 1, 3 stage 2.
+// 2 stage 1, 3 stage 2, 4 fused node (both stages).
 struct Profiler {
     bool on = false;
     cudaStream_t stream = nullptr;
@@ -72,17 +82,24 @@ thread_local Profiler t_prof;
 thread_local bakron_profile_t t_last_profile = {};
 thread_local std::vector<bakron_profile_launch_t> t_last_launches;
 
-// Algorithmic FLOPs of one stage of one recursion node: 2 T^3 per tile
-// product over the node's items.
-double node_stage_flops(const NodeParams &np, int stage)
+// FLOPs of one stage of one recursion node: 2 T^3 per tile product over the
+// node's items (tile-dense, as issued), or, with `structural`, 2 x the
+// multiply-adds that are structurally non-zero: the factor tile on the
+// diagonal (J = J' in stage 1, I = I' in stage 2) is lower triangular, so its
+// product has T^2 (T + 1) / 2 of them.
+double node_stage_flops(const NodeParams &np, int stage, bool structural = false)
 {
     const double t3 = 2.0 * kTile * (double)kTile * kTile;
+    const double tri = (double)kTile * kTile * (kTile + 1);
     double f = 0.0;
     const int cols = stage == 1 ? np.l : np.l - np.h;
     for (int I = 0; I < np.Mt; ++I)
         for (int x = 0; x < cols; ++x) {
             Item it = stage == 1 ? stage1_item(np, x, I) : stage2_item(np, x, I);
-            if (it.valid) f += t3 * (it.k1 - it.k0);
+            if (!it.valid) continue;
+            f += t3 * (it.k1 - it.k0);
+            // the contraction range ends at the diagonal tile when it reaches it
+            if (structural && it.k1 - 1 == it.ra) f -= t3 - tri;
         }
     return f;
 }
@@ -119,8 +136,9 @@ bakron_status_t read_config(const bakron_config_t *c, Config &out)
     // defaults that BAKRON_LEAF, BAKRON_GEMM, BAKRON_TIMEOUT_MS and BAKRON_GRAPH
     // override; a non-zero field of the caller's config overrides both
     int leaf = 0, gemm = 0, graph = 0;
-    if (!env_int("BAKRON_LEAF", 0, 4, leaf) || !env_int("BAKRON_GEMM", 0, 1, gemm) ||
-        !env_int("BAKRON_TIMEOUT_MS", 1, 600000, out.timeout_ms) || !env_int("BAKRON_GRAPH", 0, 1, graph))
+    if (!env_int("BAKRON_LEAF", 0, 5, leaf) || !env_int("BAKRON_GEMM", 0, 1, gemm) ||
+        !env_int("BAKRON_TIMEOUT_MS", 1, 600000, out.timeout_ms) || !env_int("BAKRON_GRAPH", 0, 1, graph) ||
+        !env_int("BAKRON_FUSE", 1, 65535, out.fuse_width))
         return BAKRON_ERR_INVALID_ARG;
     if (leaf != 0) out.leaf = leaf - 1;
     out.gemm = gemm;
@@ -135,10 +153,12 @@ bakron_status_t read_config(const bakron_config_t *c, Config &out)
     if (c->timeout_ms > 0) out.timeout_ms = c->timeout_ms;
     out.wt_out = c->wt_out;
     out.profile = c->profile ? 1 : 0;
-    if (c->leaf < 0 || c->leaf > 4) return BAKRON_ERR_INVALID_ARG;
+    if (c->leaf < 0 || c->leaf > 5) return BAKRON_ERR_INVALID_ARG;
     if (c->leaf != 0) out.leaf = c->leaf - 1;  // 0 keeps the default
     if (c->b_identity < 0 || c->b_identity > 1) return BAKRON_ERR_INVALID_ARG;
     out.b_identity = c->b_identity;
+    if (c->fuse_width < 0 || c->fuse_width > 65535) return BAKRON_ERR_INVALID_ARG;
+    if (c->fuse_width != 0) out.fuse_width = c->fuse_width;
     if (out.use_graph && out.profile) return BAKRON_ERR_INVALID_ARG;  // per-launch events cannot be replayed
     return BAKRON_OK;
 }
@@ -177,6 +197,7 @@ cudaError_t configure_device()
     if ((e = leaf_configure()) != cudaSuccess) return e;
     if ((e = leaf_gptq_configure()) != cudaSuccess) return e;
     if ((e = band_tc_configure()) != cudaSuccess) return e;
+    if ((e = band_fused_configure()) != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) g_configured[dev] = true;
     return cudaSuccess;
 }
@@ -185,7 +206,7 @@ struct SolveCtx {
     LeafArgs leaf;
     GemmArgs s1, s2;
     TcMaps m1, m2;
-    int gemm, leaf_variant;
+    int gemm, leaf_variant, fuse_width;
     cudaStream_t stream;
 };
 
@@ -211,8 +232,15 @@ cudaError_t run_schedule(const SolveCtx &c, int k, int l)
     cudaError_t e = run_schedule(c, k, h);
     if (e != cudaSuccess) return e;
     NodeParams np{k, h, l, c.leaf.Mt, c.leaf.Nt};
-    if ((e = run_band(c, 1, np)) != cudaSuccess) return e;
-    if ((e = run_band(c, 2, np)) != cudaSuccess) return e;
+    if (c.gemm == 0 && l <= c.fuse_width) {
+        t_prof.begin(4, np);
+        e = launch_band_fused(np, c.s2, c.m1, c.m2, c.stream);
+        t_prof.end();
+        if (e != cudaSuccess) return e;
+    } else {
+        if ((e = run_band(c, 1, np)) != cudaSuccess) return e;
+        if ((e = run_band(c, 2, np)) != cudaSuccess) return e;
+    }
     return run_schedule(c, k + h, l - h);
 }
 
@@ -339,7 +367,7 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
         for (int i = 0; i < 9; ++i) key.p[i] = ptrs[i];
         key.m = m; key.n = n; key.ws_bytes = ws_bytes;
         key.v[0] = qmin; key.v[1] = qmax; key.v[2] = q->row_scale ? 0 : q->shrink_grid; key.v[3] = conf.gemm;
-        key.v[4] = conf.leaf; key.v[5] = conf.timeout_ms; key.v[6] = conf.b_identity;
+        key.v[4] = conf.leaf | (conf.fuse_width << 8); key.v[5] = conf.timeout_ms; key.v[6] = conf.b_identity;
         if (cudaGetDevice(&key.v[7]) != cudaSuccess) return BAKRON_ERR_CUDA;
         return launch_graph(key, stream, [&](cudaStream_t cap) {
             return enqueue_solve(W, m, n, LA, LB, q, qmin, qmax, V, codes, scales, L, (char *)ws, conf, cap);
@@ -371,6 +399,7 @@ bakron_status_t enqueue_solve(const float *W, int64_t m, int64_t n, const float 
     SolveCtx c;
     c.gemm = conf.gemm;
     c.leaf_variant = conf.leaf;
+    c.fuse_width = conf.fuse_width;
     c.stream = stream;
     c.leaf.LA32 = (const float *)(w + L.LA32);
     c.leaf.LB32 = (const float *)(w + L.LB32);
@@ -412,8 +441,9 @@ bakron_status_t enqueue_solve(const float *W, int64_t m, int64_t n, const float 
         t_prof.on = false;
         if (cudaStreamSynchronize(stream) != cudaSuccess) return BAKRON_ERR_CUDA;
         bakron_profile_t pr = {};
-        double *ms[4] = {&pr.prep_ms, &pr.leaf_ms, &pr.stage1_ms, &pr.stage2_ms};
-        int64_t *cnt[4] = {&pr.prep_launches, &pr.leaf_launches, &pr.stage1_launches, &pr.stage2_launches};
+        double *ms[5] = {&pr.prep_ms, &pr.leaf_ms, &pr.stage1_ms, &pr.stage2_ms, &pr.fused_ms};
+        int64_t *cnt[5] = {&pr.prep_launches, &pr.leaf_launches, &pr.stage1_launches, &pr.stage2_launches,
+                           &pr.fused_launches};
         t_last_launches.clear();
         for (size_t i = 0; i < t_prof.kinds.size() && 2 * i + 1 < t_prof.used; ++i) {
             float dt = 0.f;
@@ -428,7 +458,15 @@ bakron_status_t enqueue_solve(const float *W, int64_t m, int64_t n, const float 
             r.h = np.h;
             r.l = np.l;
             r.ms = dt;
-            r.flops = kind < 2 ? 0.0 : conf.b_identity ? gptq_node_flops(np) : node_stage_flops(np, kind - 1);
+            r.flops = kind < 2              ? 0.0
+                      : conf.b_identity     ? gptq_node_flops(np)
+                      : kind == 4           ? node_stage_flops(np, 1) + node_stage_flops(np, 2)
+                                            : node_stage_flops(np, kind - 1);
+            // the one-sided update's factor tiles are all off the diagonal
+            r.structural_flops = kind < 2          ? 0.0
+                                 : conf.b_identity ? r.flops
+                                 : kind == 4       ? node_stage_flops(np, 1, true) + node_stage_flops(np, 2, true)
+                                                   : node_stage_flops(np, kind - 1, true);
             t_last_launches.push_back(r);
         }
         pr.prep_launches *= conf.b_identity ? 3 : 4;  // scales, padded copy, the factor normalisations
@@ -439,6 +477,17 @@ bakron_status_t enqueue_solve(const float *W, int64_t m, int64_t n, const float 
     }
     return BAKRON_OK;
 }
+
+}  // namespace
+
+bakron_status_t bakron::solve_direct(const float *W, int64_t m, int64_t n, const float *LA, const float *LB,
+                                     const bakron_quantizer_t *q, float *V, int8_t *codes, float *scales,
+                                     void *ws, size_t ws_bytes, const bakron_config_t *cfg, cudaStream_t stream)
+{
+    return solve_device(W, m, n, LA, LB, q, V, codes, scales, ws, ws_bytes, cfg, stream, true, true);
+}
+
+namespace {
 
 void count_schedule(int k, int l, int Mt, int Nt, bakron_plan_stats_t *o)
 {
@@ -451,6 +500,7 @@ void count_schedule(int k, int l, int Mt, int Nt, bakron_plan_stats_t *o)
     NodeParams np{k, h, l, Mt, Nt};
     o->stage1_flops += node_stage_flops(np, 1);
     o->stage2_flops += node_stage_flops(np, 2);
+    o->structural_flops += node_stage_flops(np, 1, true) + node_stage_flops(np, 2, true);
     o->nodes++;
     count_schedule(k + h, l - h, Mt, Nt, o);
 }
@@ -465,7 +515,9 @@ void count_schedule_gptq(int k, int l, int Mt, int Nt, bakron_plan_stats_t *o)
     }
     const int h = l / 2;
     count_schedule_gptq(k, h, Mt, Nt, o);
-    o->stage1_flops += gptq_node_flops(NodeParams{k, h, l, Mt, Nt});
+    const double f = gptq_node_flops(NodeParams{k, h, l, Mt, Nt});
+    o->stage1_flops += f;
+    o->structural_flops += f;  // no diagonal factor tile in the one-sided update
     o->nodes++;
     count_schedule_gptq(k + h, l - h, Mt, Nt, o);
 }
@@ -530,7 +582,7 @@ bakron_status_t bakron_tune_leaf(const float *W_dev, int64_t m, int64_t n, const
     bakron_status_t s = BAKRON_OK;
     double best = 0.0;
     int best_leaf = 0;
-    for (int leaf = 0; leaf <= 4 && s == BAKRON_OK; ++leaf) {
+    for (int leaf = 0; leaf <= kLeafStructures && s == BAKRON_OK; ++leaf) {
         c.leaf = leaf == 0 ? 3 : leaf;  // iteration 0 is the warm-up
         if (cudaEventRecord(ev[0], st) != cudaSuccess) { s = BAKRON_ERR_CUDA; break; }
         // timed with direct launches (a first graph call would time its capture)
@@ -738,8 +790,8 @@ bakron_status_t bakron_factor(const float *A_dev, int64_t n, const float *B_dev,
 
 size_t bakron_proxy_loss_workspace_size(int64_t m, int64_t n)
 {
-    if (m < 1 || n < 1) return 0;
-    return kStatusBytes;
+    if (m < 1 || n < 1 || m > kMaxSide || n > kMaxSide) return 0;
+    return align_up(kStatusBytes) + (size_t)proxy_loss_parts(m, n) * sizeof(double);
 }
 
 bakron_status_t bakron_proxy_loss(const float *W_dev, const float *V_dev, const float *A_dev,
@@ -749,13 +801,14 @@ bakron_status_t bakron_proxy_loss(const float *W_dev, const float *V_dev, const 
 {
     if (m < 1 || n < 1 || m > kMaxSide || n > kMaxSide) return BAKRON_ERR_INVALID_ARG;
     if (!W_dev || !V_dev || !A_dev || !B_dev || !out_dev) return BAKRON_ERR_INVALID_ARG;
-    if (!ws_dev || ws_bytes < kStatusBytes) return BAKRON_ERR_WORKSPACE;
-    if (!aligned16(W_dev) || !aligned16(V_dev) || !aligned16(A_dev) || !aligned16(B_dev) ||
+    if (!ws_dev || ws_bytes < bakron_proxy_loss_workspace_size(m, n)) return BAKRON_ERR_WORKSPACE;
+    if (!aligned16(W_dev) || !aligned16(V_dev) || !aligned16(A_dev) || !aligned16(B_dev) || !aligned16(ws_dev) ||
         ((uintptr_t)out_dev & 7u))
         return BAKRON_ERR_ALIGNMENT;
     cudaStream_t s = (cudaStream_t)stream;
     if (cudaMemsetAsync(ws_dev, 0, kStatusBytes, s) != cudaSuccess) return BAKRON_ERR_CUDA;
-    if (launch_proxy_loss(W_dev, V_dev, A_dev, B_dev, m, n, out_dev, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    double *part = (double *)((char *)ws_dev + align_up(kStatusBytes));
+    if (launch_proxy_loss(W_dev, V_dev, A_dev, B_dev, m, n, out_dev, part, s) != cudaSuccess) return BAKRON_ERR_CUDA;
     if (out_host) {
         if (cudaMemcpyAsync(out_host, out_dev, sizeof(double), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
             cudaStreamSynchronize(s) != cudaSuccess)
@@ -773,6 +826,23 @@ bakron_status_t bakron_selftest_wait_timeout(int32_t timeout_ms, void *ws_dev, s
     cudaStream_t s = (cudaStream_t)stream;
     if (cudaMemsetAsync(ws_dev, 0, kStatusBytes, s) != cudaSuccess) return BAKRON_ERR_CUDA;
     if (launch_wait_timeout_selftest((DeviceStatus *)ws_dev, timeout_ms, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    return BAKRON_OK;
+}
+
+size_t bakron_selftest_band_abort_workspace_size(void) { return align_up(kStatusBytes) + kBandAbortBufBytes; }
+
+bakron_status_t bakron_selftest_band_abort(int32_t timeout_ms, void *ws_dev, size_t ws_bytes, bakron_stream_t stream)
+{
+    if (timeout_ms < 1 || timeout_ms > 10000) return BAKRON_ERR_INVALID_ARG;
+    if (!ws_dev || ws_bytes < bakron_selftest_band_abort_workspace_size()) return BAKRON_ERR_WORKSPACE;
+    if (!aligned16(ws_dev)) return BAKRON_ERR_ALIGNMENT;
+    if (configure_device() != cudaSuccess) return BAKRON_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    char *w = (char *)ws_dev;
+    if (cudaMemsetAsync(w, 0, kStatusBytes, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (launch_band_abort_selftest((DeviceStatus *)w, (float *)(w + align_up(kStatusBytes)), timeout_ms, s) !=
+        cudaSuccess)
+        return BAKRON_ERR_CUDA;
     return BAKRON_OK;
 }
 

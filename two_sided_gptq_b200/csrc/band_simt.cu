@@ -79,12 +79,13 @@ cudaError_t launch_band_simt(int stage, const NodeParams &np, const GemmArgs &g,
 // Proxy loss l = sum_ij (B E)_ij (E A)_ij with E = W - V (Corollary 3.4's
 // ||B^{1/2}(V-W)A^{1/2}||_F^2 written as tr(E^T B E A)).  One CTA per 64 x 64
 // output tile computes both products in FP32 and reduces their elementwise
-// product in FP64.
+// product in FP64 into its own slot of `part`; one more CTA adds the slots in
+// a fixed order, so the result does not depend on the order the CTAs finish.
 __global__ void __launch_bounds__(256) proxy_loss_kernel(const float *__restrict__ W,
                                                         const float *__restrict__ V,
                                                         const float *__restrict__ A,
                                                         const float *__restrict__ B, int64_t m,
-                                                        int64_t n, double *out)
+                                                        int64_t n, double *tile_sums)
 {
     constexpr int TB = 64, KB = 16;
     __shared__ float Xs[KB][TB + 4];
@@ -149,17 +150,37 @@ __global__ void __launch_bounds__(256) proxy_loss_kernel(const float *__restrict
     if (tid == 0) {
         double s = 0.0;
         for (int w = 0; w < 8; ++w) s += red[w];
-        atomicAdd(out, s);
+        tile_sums[(int64_t)blockIdx.y * gridDim.x + blockIdx.x] = s;
     }
 }
 
-cudaError_t launch_proxy_loss(const float *W, const float *V, const float *A, const float *B,
-                              int64_t m, int64_t n, double *out, cudaStream_t stream)
+// out = sum of the per-tile partial sums: each thread adds a strided subset in
+// index order, then a fixed tree over the threads.
+__global__ void __launch_bounds__(256) proxy_loss_finish_kernel(const double *__restrict__ part, int64_t count,
+                                                               double *out)
 {
-    cudaError_t e = cudaMemsetAsync(out, 0, sizeof(double), stream);
-    if (e != cudaSuccess) return e;
+    __shared__ double red[256];
+    double s = 0.0;
+    for (int64_t i = threadIdx.x; i < count; i += 256) s += part[i];
+    red[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = 128; w; w >>= 1) {
+        if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) *out = red[0];
+}
+
+int64_t proxy_loss_parts(int64_t m, int64_t n) { return ((n + 63) / 64) * ((m + 63) / 64); }
+
+cudaError_t launch_proxy_loss(const float *W, const float *V, const float *A, const float *B,
+                              int64_t m, int64_t n, double *out, double *part, cudaStream_t stream)
+{
     dim3 grid((unsigned)((n + 63) / 64), (unsigned)((m + 63) / 64));
-    proxy_loss_kernel<<<grid, 256, 0, stream>>>(W, V, A, B, m, n, out);
+    proxy_loss_kernel<<<grid, 256, 0, stream>>>(W, V, A, B, m, n, part);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    proxy_loss_finish_kernel<<<1, 256, 0, stream>>>(part, proxy_loss_parts(m, n), out);
     return cudaGetLastError();
 }
 

@@ -22,8 +22,11 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tcgen05.cuh"
 
 namespace bakron {
+
+using namespace tc;
 
 namespace {
 constexpr int T = kTile;
@@ -39,119 +42,6 @@ constexpr uint32_t kTmemCols = 2 * T;  // two accumulator buffers
 // Instruction descriptor: D fp32, A/B tf32, K-major both, N = 128, M = 128.
 constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(T >> 3) << 17) |
                             ((uint32_t)(T >> 4) << 24);
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ uint64_t now_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait: false if the deadline passed first.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t deadline)
-{
-    while (!mbar_try_wait(bar, parity))
-        if (now_ns() > deadline) return false;
-    return true;
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"((uint64_t)map), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-// UMMA shared-memory descriptor, K-major, 128-byte swizzle: 8-row atoms of
-// 128 B rows, atoms 1024 B apart (SBO), LBO unused (1), version 1.
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr)
-{
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-__device__ __forceinline__ void umma_tf32(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate));
-}
-__device__ __forceinline__ void umma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-// Tile store (stage 1) and tile add-reduction (stage 2) from shared memory
-// through the tensor map, tracked as one bulk async-group.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, uint32_t src)
-{
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
-                 ::"l"((uint64_t)map), "r"(x), "r"(y), "r"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void tma_add_2d(const CUtensorMap *map, int x, int y, uint32_t src)
-{
-    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];"
-                 ::"l"((uint64_t)map), "r"(x), "r"(y), "r"(src)
-                 : "memory");
-}
-// Commit the bulk stores and wait until they have read their shared-memory
-// source (the global writes complete with the grid).
-__device__ __forceinline__ void bulk_commit_and_wait_read()
-{
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// L2 prefetch of one box through a tensor map (a hint; no completion).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, int y)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"((uint64_t)map), "r"(x),
-                 "r"(y)
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
-{
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 }  // namespace
 
@@ -238,7 +128,7 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer
         int issued = 0;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < (g.test_no_tma ? 0 : nk); ++kb) {
             const int s = kb % kStages;
             if (kb >= kStages && !mbar_wait(empty_bar(s), ((kb / kStages) - 1) & 1, deadline)) {
                 record_error(g.st, BAKRON_ERR_DEVICE_TIMEOUT, 1000 + STAGE);
@@ -285,9 +175,9 @@ band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
                     const uint64_t ah = umma_desc(base + off), al = umma_desc(base + kTileBytes + off);
                     const uint64_t bh = umma_desc(base + 2 * kTileBytes + off),
                                    bl = umma_desc(base + 3 * kTileBytes + off);
-                    umma_tf32(tmem_d, al, bh, (kc | k8) != 0);
-                    umma_tf32(tmem_d, ah, bl, 1);
-                    umma_tf32(tmem_d, ah, bh, 1);
+                    umma_tf32(tmem_d, al, bh, kIdesc, (kc | k8) != 0);
+                    umma_tf32(tmem_d, ah, bl, kIdesc, 1);
+                    umma_tf32(tmem_d, ah, bh, kIdesc, 1);
                 }
                 umma_commit(empty_bar(s));
             }
@@ -487,6 +377,20 @@ cudaError_t launch_wait_timeout_selftest(DeviceStatus *st, int timeout_ms, cudaS
 {
     wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(st, timeout_ms);
     return cudaGetLastError();
+}
+
+cudaError_t launch_band_abort_selftest(DeviceStatus *st, float *buf, int timeout_ms, cudaStream_t stream)
+{
+    // stage 1 of node (k 0, h 1, l 2) on a 2 x 2 tile grid: two valid items
+    // (X^T tiles (0, 0) and (1, 0)), each with one chunk of contraction
+    constexpr int64_t n2 = 256;
+    float *a_hi = buf, *a_lo = buf + n2 * n2, *b_hi = buf + 2 * n2 * n2, *b_lo = buf + 3 * n2 * n2;
+    float *o_hi = buf + 4 * n2 * n2, *o_lo = buf + 5 * n2 * n2;
+    GemmArgs g{a_hi, a_lo, b_hi, b_lo, n2, n2, o_hi, o_lo, nullptr, n2, st, timeout_ms, 1};
+    TcMaps maps;
+    if (!make_tc_maps(1, 2, 2, g, &maps)) return cudaErrorInvalidValue;
+    const NodeParams np{0, 1, 2, 2, 2};
+    return launch_band_tc(1, np, g, maps, stream);
 }
 
 cudaError_t launch_gram_tc(const NodeParams &np, const GemmArgs &g, const TcMaps &maps, cudaStream_t stream)

@@ -28,6 +28,7 @@ struct GemmArgs {
     int64_t ldo;
     DeviceStatus *st;
     int timeout_ms;
+    int test_no_tma;  // self-test only: the producer issues no copies, so the waits run out
 };
 
 cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, const float *LB, int qmin,
@@ -36,6 +37,9 @@ cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, c
 
 cudaError_t leaf_configure();
 cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stream);
+// Leaf with one tile per cluster of four CTAs (leaf_cluster.cu).
+cudaError_t leaf_cluster_configure();
+cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, cudaStream_t stream);
 
 // FP32 CUDA-core band products (reference kernels for the tensor-core path).
 cudaError_t launch_band_simt(int stage, const NodeParams &np, const GemmArgs &g, cudaStream_t stream);
@@ -52,6 +56,12 @@ bool make_tc_maps(int stage, int Mt, int Nt, const GemmArgs &g, TcMaps *maps);
 cudaError_t launch_band_tc(int stage, const NodeParams &np, const GemmArgs &g, const TcMaps &maps,
                            cudaStream_t stream);
 
+// Both band products of a node in one launch (band_fused.cu): m1 = the
+// stage-1 maps (LtA, Delta), m2 = the stage-2 maps (LtB, output Wt).
+cudaError_t band_fused_configure();
+cudaError_t launch_band_fused(const NodeParams &np, const GemmArgs &g, const TcMaps &m1, const TcMaps &m2,
+                              cudaStream_t stream);
+
 // One-sided (B = I) path: the leaf over a 128-column block and the update.
 cudaError_t leaf_gptq_configure();
 cudaError_t launch_leaf_gptq(const LeafArgs &p, int Jb, cudaStream_t stream);
@@ -66,16 +76,32 @@ cudaError_t launch_gram_prep(const float *X, int64_t N, int64_t d, int64_t Dp, i
 cudaError_t launch_gram_finish(const float *G, int64_t d, int64_t Dp, int64_t N, float damping, float *A,
                                cudaStream_t stream);
 
-// Proxy loss (FP32 products, FP64 reduction) into *out (device double).
+// Proxy loss (FP32 products, FP64 reduction) into *out (device double);
+// `part` holds proxy_loss_parts(m, n) doubles (per-tile partial sums).
+int64_t proxy_loss_parts(int64_t m, int64_t n);
 cudaError_t launch_proxy_loss(const float *W, const float *V, const float *A, const float *B,
-                              int64_t m, int64_t n, double *out, cudaStream_t stream);
+                              int64_t m, int64_t n, double *out, double *part, cudaStream_t stream);
 
 // FP64 factorisation: L (n x n, fp32) = chol(A^{-1}); work = n*n doubles.
 cudaError_t launch_factor(const float *A, int64_t n, float *L, double *work, DeviceStatus *st,
                           cudaStream_t stream);
 
+// bakron_solve with direct launches only: never the CUDA graph path, whatever
+// cfg->use_graph or BAKRON_GRAPH ask for (graph capture and instantiation make
+// the driver allocate).  Arguments and checks as bakron_solve.
+bakron_status_t solve_direct(const float *W, int64_t m, int64_t n, const float *LA, const float *LB,
+                             const bakron_quantizer_t *q, float *V, int8_t *codes, float *scales, void *ws,
+                             size_t ws_bytes, const bakron_config_t *cfg, cudaStream_t stream);
+
 // One thread waits on an mbarrier nothing completes, with the band kernel's
 // bounded-wait helper; records BAKRON_ERR_DEVICE_TIMEOUT when it gives up.
 cudaError_t launch_wait_timeout_selftest(DeviceStatus *st, int timeout_ms, cudaStream_t stream);
+
+// The stage-1 band kernel on a 256 x 256 problem laid out in `buf` (six
+// 256 x 256 fp32 arrays, 16-byte aligned) with its producer issuing no copies:
+// the MMA and epilogue waits run out, record BAKRON_ERR_DEVICE_TIMEOUT and the
+// kernel takes its abort path (nothing is in flight).
+constexpr size_t kBandAbortBufBytes = (size_t)6 * 256 * 256 * sizeof(float);
+cudaError_t launch_band_abort_selftest(DeviceStatus *st, float *buf, int timeout_ms, cudaStream_t stream);
 
 }  // namespace bakron

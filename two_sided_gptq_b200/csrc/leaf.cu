@@ -26,8 +26,11 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "leaf_common.cuh"
 
 namespace bakron {
+
+using namespace leafk;
 
 namespace {
 constexpr int T = kTile;           // 128
@@ -40,11 +43,6 @@ constexpr int kThreads = 512;
 constexpr size_t kSmemNested = ((size_t)2 * T * RS + 2 * S * BS + S * ZS + 2 * T) * sizeof(float);
 constexpr size_t kSmemSingle = ((size_t)3 * T * RS1 + 2 * T) * sizeof(float);
 static_assert(kSmemNested <= 232448 && kSmemSingle <= 232448, "leaf shared memory");
-
-__device__ __forceinline__ void group_sync(int id, int nthreads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 __device__ __forceinline__ float4 mask4(float4 v, int len)  // keep the first len (<= 4) components
 {
@@ -60,19 +58,6 @@ __device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc)
     acc = fmaf(a.y, b.y, acc);
     acc = fmaf(a.z, b.z, acc);
     return fmaf(a.w, b.w, acc);
-}
-
-// Two FP32 fused multiply-adds in one packed instruction (sm_100), each
-// rounded to nearest like fmaf.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
-{
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
 }
 
 // Rounding decision clamp(rint(wt / s)) with the IEEE fp32 quotient.  Fast
@@ -182,15 +167,6 @@ __device__ void write_outputs(const LeafArgs &p, const float *sDt, const float *
 // with K contiguous (generic pointers into smem or global memory).  16 warps,
 // each owning a 16 x 16 block of D as two m16n8 tiles; mma.sync m16n8k8 TF32
 // in 3xTF32 form.
-__device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
 __device__ void accumulate_product(float (&acc)[2][4], const float *a, int lda, const float *b, int ldb)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -416,59 +392,7 @@ constexpr size_t kSmemWarp =
 static_assert(kSmemWarp <= 232448, "leaf shared memory");
 }  // namespace
 
-// acc (a 16 x 8*NT block at (i0, j0) of a 32 x 32 product) += sum_{k<K} A[i][k] Bm[j][k]
-template <int NT>
-__device__ __forceinline__ void mma_block(float (&acc)[NT][4], const float *A, int lda, const float *Bm, int ldb,
-                                          int K, int i0, int j0)
-{
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-#pragma unroll 4
-    for (int k0 = 0; k0 < K; k0 += 8) {
-        const float af[4] = {A[(i0 + g) * lda + k0 + t], A[(i0 + g + 8) * lda + k0 + t],
-                             A[(i0 + g) * lda + k0 + t + 4], A[(i0 + g + 8) * lda + k0 + t + 4]};
-        uint32_t ahi[4], alo[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            float h, l;
-            split_tf32(af[r], h, l);
-            ahi[r] = __float_as_uint(h);
-            alo[r] = __float_as_uint(l);
-        }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int j = j0 + nt * 8 + g;
-            const float bf[2] = {Bm[j * ldb + k0 + t], Bm[j * ldb + k0 + t + 4]};
-            uint32_t bhi[2], blo[2];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                float h, l;
-                split_tf32(bf[r], h, l);
-                bhi[r] = __float_as_uint(h);
-                blo[r] = __float_as_uint(l);
-            }
-            mma_tf32(acc[nt], alo, bhi);
-            mma_tf32(acc[nt], ahi, blo);
-            mma_tf32(acc[nt], ahi, bhi);
-        }
-    }
-}
-
 constexpr int kThreadsW = 384;  // warp variant: 3 warps per row block of sub-tiles
-
-// Byte of an integer-valued float in [-128, 127] (two's complement) without a
-// conversion instruction: adding 1.5 * 2^23 puts the integer in the low
-// mantissa bits.
-__device__ __forceinline__ int8_t code_byte(float c)
-{
-    return (int8_t)(__float_as_int(c + 12582912.0f) & 0xFF);
-}
-
-__device__ __forceinline__ void cp_async16(void *dst, const void *src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src)
-                 : "memory");
-}
 
 __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int K, int I_lo)
 {
@@ -564,7 +488,6 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
     }
     const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
     const int wp = warp / 3, role = warp - 3 * wp;  // row block of sub-tiles; 0 entries, 1 row side, 2 column side
-    const int i0 = (role & 1) * 16, j0 = 0;         // products: roles 0 and 1 take a 16 x 32 half each
     // column-side warp: its LtB[p,p] row rho (columns <= rho-2), fixed for the kernel
     float2 lbr[S3 / 2];
     if (role == 2) {
@@ -586,20 +509,11 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
         const int qv = e - wp;
         asm volatile("cp.async.wait_all;" ::: "memory");  // this phase's staged Wt blocks and strips
         __syncthreads();
-        // S[p,q] = LtB[p, 0:p] D[0:p, q] into the row block's slot
-        if (mine && role < 2 && wp > 0) {
-            float acc[4][4] = {};
-            mma_block<4>(acc, sLBs + lb_offset(e, wp), S3 * wp + 4, sDt + (qv * S3) * RS3, RS3, wp * S3, i0, j0);
-            const int g = lane >> 2, t = lane & 3;
-            float *o = sW + wp * S3 * WS3;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int j = j0 + nt * 8 + 2 * t;
-                o[(i0 + g) * WS3 + j] = acc[nt][0];
-                o[(i0 + g) * WS3 + j + 1] = acc[nt][1];
-                o[(i0 + g + 8) * WS3 + j] = acc[nt][2];
-                o[(i0 + g + 8) * WS3 + j + 1] = acc[nt][3];
-            }
+        // S[p,q] = LtB[p, 0:p] D[0:p, q] into the row block's slot (three warps)
+        if (mine && wp > 0) {
+            Block3 b;
+            product3(b, role, sLBs + lb_offset(e, wp), S3 * wp + 4, sDt + (qv * S3) * RS3, RS3, wp * S3);
+            store3(b, role, sW + wp * S3 * WS3, WS3);
         }
         // row-side warp: LtA[q,q] row b (columns <= b-2); entry warp: LtA[b][b-1]
         float2 la[S3 / 2];
@@ -618,23 +532,10 @@ __global__ void __launch_bounds__(kThreadsW, 1) leaf_warp_kernel(LeafArgs p, int
         // W0[p,q] = Wt[p,q] - R[p, 0:q] LtA[q, 0:q]^T - S[p,q] into the slot; R's
         // (p,q) block (holding the staged Wt) becomes S: the sweep adds the S terms
         // of the row-side sums through R
-        if (mine && role < 2) {
-            float acc[4][4] = {};
-            if (qv > 0)
-                mma_block<4>(acc, sR + (wp * S3) * RS3, RS3, sLA + la_offset(e, wp), S3 * qv + 4, qv * S3, i0, j0);
-            const int g = lane >> 2, t = lane & 3;
-            float *o = sW + wp * S3 * WS3;
-            float *rq = sR + (wp * S3) * RS3 + qv * S3;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int i = i0 + g + 8 * (h >> 1), j = j0 + nt * 8 + 2 * t + (h & 1);
-                    const float sv = wp > 0 ? o[i * WS3 + j] : 0.f;
-                    const float wt = rq[i * RS3 + j];
-                    o[i * WS3 + j] = wt - acc[nt][h] - sv;
-                    rq[i * RS3 + j] = sv;
-                }
+        if (mine) {  // three warps
+            Block3 b;
+            product3(b, role, sR + (wp * S3) * RS3, RS3, sLA + la_offset(e, wp), S3 * qv + 4, qv * S3);
+            finish3(b, role, sW + wp * S3 * WS3, WS3, sR + (wp * S3) * RS3 + qv * S3, RS3, wp > 0);
         }
         __syncthreads();
         stage_phase(e + 1);  // lands while this phase sweeps
@@ -1070,13 +971,16 @@ cudaError_t leaf_configure()
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(leaf_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemWide);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(leaf_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemSingle);
+    e = cudaFuncSetAttribute(leaf_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemSingle);
+    if (e != cudaSuccess) return e;
+    return leaf_cluster_configure();
 }
 
 cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stream)
 {
     int I_lo = max(0, K - (p.Nt - 1)), I_hi = min(p.Mt - 1, K);
     if (I_hi < I_lo) return cudaSuccess;
+    if (variant == 4) return launch_leaf_cluster(p, K, I_lo, I_hi - I_lo + 1, stream);
     if (variant == 3)
         return launch_pdl(leaf_wide_kernel, dim3(I_hi - I_lo + 1), dim3(kThreadsWide), kSmemWide, stream, p, K, I_lo);
     if (variant == 2)

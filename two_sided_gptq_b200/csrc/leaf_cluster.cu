@@ -1,0 +1,343 @@
+// leaf_cluster.cu -- the leaf sweep of one tile diagonal with each tile on a
+// cluster of four CTAs (Proposition 3.1's updates inside the tile, entries of
+// one entry anti-diagonal rounded in parallel: Theorem 3.2).
+//
+// The warp variant (leaf.cu) keeps a whole 128 x 128 tile in one CTA, cut into
+// 4 x 4 sub-tiles of 32 processed in sub-tile-diagonal phases; in the middle
+// phases up to four sub-tile sweeps share one SM's issue slots and
+// shared-memory bandwidth, and each dependent step gets slower.  Here CTA p of
+// a four-CTA cluster owns row block p of the tile: its R rows, its columns of
+// D, its sub-tiles (p, q), q = 0..3, swept in phase e = p + q by its three
+// warps exactly as the warp variant sweeps one sub-tile:
+//     S[p,q]  = sum_{p'<p} LtB[p,p'] D[p',q],
+//     W0[p,q] = Wt[p,q] - sum_{q'<q} R[p,q'] LtA[q,q']^T - S[p,q],
+// then 63 entry anti-diagonal steps (entry warp, row-side warp, column-side
+// warp; one 96-thread barrier per step).  The only data that crosses CTAs is
+// D[p',q] of the row blocks above, which the S product reads from their
+// shared memory (distributed shared memory) after the cluster barrier that
+// opens each phase; R and everything else stays local.  Every CTA passes the
+// same eight cluster barriers, so the waits are those of a hardware barrier
+// with equal trip counts.
+#include <cooperative_groups.h>
+
+#include <type_traits>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "leaf_common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace bakron {
+
+using namespace leafk;
+
+namespace {
+constexpr int T = kTile;
+constexpr int S3 = 32;            // sub-tile side
+constexpr int kThreadsC = 96;     // entry, row-side and column-side warps
+constexpr int RSC = T + 4;        // row stride of sR (32 rows x 128 columns)
+constexpr int DSC = S3 + 4;       // row stride of sDt (128 columns x 32 rows)
+constexpr int WSC = S3 + 4;       // row stride of the sub-tile slot
+constexpr int LSC = 3 * S3 + 4;   // row stride of strips of up to three 32-wide blocks
+constexpr size_t kSmemC = ((size_t)(S3 + 1) * RSC + (size_t)(T + 1) * DSC + (size_t)S3 * WSC +
+                           (size_t)3 * S3 * LSC + 3 * S3 + 4 * S3) * sizeof(float) +
+                          (size_t)S3 * T + 32;
+// Requested per CTA so that two CTAs never share an SM: the point of the
+// variant is one sub-tile sweep per SM.
+constexpr size_t kSmemCLaunch = 120 * 1024;
+static_assert(kSmemC <= kSmemCLaunch && 2 * kSmemCLaunch > 228 * 1024, "cluster leaf shared memory");
+}  // namespace
+
+__global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreadsC, 1)
+leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
+{
+    cg::cluster_group cluster = cg::this_cluster();
+    const int pp = (int)cluster.block_rank();  // row block of sub-tiles
+
+    extern __shared__ __align__(16) float smem_f[];
+    float *sR = smem_f;                       // (S3+1) x RSC: R of this row block (S before a sweep, Wt staged)
+    float *sDt = sR + (S3 + 1) * RSC;         // (T+1) x DSC: D transposed, this row block's rows, 0 until rounded
+    float *sW = sDt + (T + 1) * DSC;          // S3 x WSC: S, then W0 of the sub-tile being swept
+    float *sLA = sW + S3 * WSC;               // LtA[q, 0:q] strip, row stride 32 q + 4 (staged a phase ahead)
+    float *sLBs = sLA + S3 * LSC;             // LtB[p, 0:p] strip, row stride 32 p + 4 (loaded once)
+    float *sDr = sLBs + S3 * LSC;             // D[0:p, q] of the row blocks above: [column][32 p' + row], LSC
+    float *sLBd = sDr + S3 * LSC;             // S3: LtB[r][r-1] inside the row block (0 for r = 0)
+    float *scale = sLBd + S3;                 // S3
+    float *rcp = scale + S3;                  // S3
+    float *sPS = rcp + S3;                    // 2 x S3: column-side partial sums by column
+    float *sPU = sPS + 2 * S3;                // 2 x S3: row-side partial sums by column
+    int8_t *sCode = (int8_t *)(sPU + 2 * S3); // S3 x T codes (+32 spare bytes)
+
+    const int I = I_lo + (int)(blockIdx.x / 4), J = K - I;
+    const int64_t row0 = (int64_t)I * T, col0 = (int64_t)J * T;
+    const int64_t brow0 = row0 + pp * S3;  // first row of this row block
+    const int mr = (int)min64(T, p.m - row0), nc = (int)min64(T, p.n - col0);
+    const int mrb = max(0, min(S3, mr - pp * S3));  // rows of this row block inside the matrix
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float *LAt = p.LA32 + col0 * p.Np + col0;  // LtA diagonal block of the tile (global)
+    const float *LBt = p.LB32 + row0 * p.Mp + row0;  // LtB diagonal block of the tile (global)
+    const int lda_g = (int)p.Np, ldb_g = (int)p.Mp;
+    // Warm L2 with the factor rows this CTA reads (a hint; it may precede the
+    // dependency wait): all of the LtA diagonal block, this row block's LtB rows.
+    for (int idx = tid; idx < (T + S3) * (T / 32); idx += kThreadsC) {
+        const int r = idx / (T / 32), seg = idx % (T / 32);
+        const float *ptr = r < T ? LAt + r * lda_g + 32 * seg : LBt + (pp * S3 + r - T) * ldb_g + 32 * seg;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+    }
+    for (int idx = tid; idx < (S3 + 1) * RSC / 4; idx += kThreadsC)
+        ((float4 *)sR)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int idx = tid; idx < (T + 1) * DSC / 4; idx += kThreadsC)
+        ((float4 *)sDt)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();  // R is zero before the first staged block lands in it
+    pdl_wait();       // every global input (Wt, factors, steps) comes from earlier kernels
+
+    // Stage the sub-tile (pp, e - pp) of phase e, if it is this CTA's: its Wt
+    // block into R's block (untouched until then) and the strip LtA[q, 0:q].
+    auto stage_phase = [&](int e) {
+        const int q = e - pp;
+        if (q < 0 || q > 3) return;
+        if (q > 0) {
+            const int ld = S3 * q + 4, c4 = 8 * q;
+            for (int c = tid; c < S3 * c4; c += kThreadsC) {
+                const int j = c / c4, k4 = c - j * c4;
+                cp_async16(sLA + j * ld + 4 * k4, LAt + (q * S3 + j) * lda_g + 4 * k4);
+            }
+        }
+        for (int c = tid; c < S3 * 8; c += kThreadsC) {
+            const int i = c >> 3, k4 = c & 7;
+            cp_async16(sR + i * RSC + q * S3 + 4 * k4, p.Wt + (brow0 + i) * p.Np + col0 + q * S3 + 4 * k4);
+        }
+    };
+    stage_phase(0);
+    if (pp > 0) {  // LtB[p, 0:p], fixed for the kernel
+        const int ld = S3 * pp + 4, c4 = 8 * pp;
+        for (int c = tid; c < S3 * c4; c += kThreadsC) {
+            const int i = c / c4, k4 = c - i * c4;
+            cp_async16(sLBs + i * ld + 4 * k4, LBt + (pp * S3 + i) * ldb_g + 4 * k4);
+        }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (tid < S3) sLBd[tid] = tid > 0 ? LBt[(pp * S3 + tid) * ldb_g + pp * S3 + tid - 1] : 0.f;
+    const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
+    const int role = warp;                    // 0 entries, 1 row side, 2 column side
+    // column-side warp: its LtB[p,p] row rho (columns <= rho-2), fixed for the kernel
+    float2 lbr[S3 / 2];
+    if (role == 2) {
+#pragma unroll
+        for (int c = 0; c < S3 / 2; ++c) {
+            float2 v = *(const float2 *)(LBt + (pp * S3 + lane) * ldb_g + pp * S3 + 2 * c);
+            v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
+            v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
+            lbr[c] = v;
+        }
+    }
+    // Steps of this row block and their correctly rounded reciprocals; a step
+    // outside [2^-60, 2^60] switches the row block to the IEEE division (both
+    // give the correctly rounded quotient, so the choice never shows).
+    bool out_of_range = false;
+    if (tid < S3) {
+        const float s = tid < mrb ? p.scales[brow0 + tid] : 1.f;
+        scale[tid] = s;
+        rcp[tid] = __frcp_rn(s);
+        out_of_range = !(s >= 0x1p-60f && s <= 0x1p60f);
+    }
+    const bool exact_div = __syncthreads_or(out_of_range) != 0;
+
+    for (int e = 0; e < 7; ++e) {
+        const int q = e - pp;
+        const bool mine = q >= 0 && q <= 3;
+        // Every CTA of the cluster has finished phase e - 1, so the D blocks
+        // it rounded are final and visible (release / acquire at cluster scope).
+        cluster.sync();
+        asm volatile("cp.async.wait_all;" ::: "memory");  // this phase's staged Wt block and strip
+        if (mine && pp > 0) {
+            // D[p', q] (p' < p) from the other CTAs' shared memory, transposed
+            for (int c = tid; c < pp * S3 * 8; c += kThreadsC) {
+                const int pr = c / (S3 * 8), j = (c >> 3) % S3, r4 = c & 7;
+                const float *src = cluster.map_shared_rank(sDt, pr) + (q * S3 + j) * DSC + 4 * r4;
+                *(float4 *)(sDr + j * LSC + pr * S3 + 4 * r4) = *(const float4 *)src;
+            }
+        }
+        __syncthreads();
+        // S[p,q] = LtB[p, 0:p] D[0:p, q] into the slot (three warps)
+        if (mine && pp > 0) {
+            Block3 b;
+            product3(b, role, sLBs, S3 * pp + 4, sDr, LSC, pp * S3);
+            store3(b, role, sW, WSC);
+        }
+        // row-side warp: LtA[q,q] row b (columns <= b-2); entry warp: LtA[b][b-1]
+        float2 la[S3 / 2];
+        float la_new = 0.f;
+        if (mine && role == 1) {
+#pragma unroll
+            for (int c = 0; c < S3 / 2; ++c) {
+                float2 v = *(const float2 *)(LAt + (q * S3 + lane) * lda_g + q * S3 + 2 * c);
+                v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
+                v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
+                la[c] = v;
+            }
+        }
+        if (mine && role == 0 && lane > 0) la_new = LAt[(q * S3 + lane) * lda_g + q * S3 + lane - 1];
+        __syncthreads();
+        // W0[p,q] = Wt[p,q] - R[p, 0:q] LtA[q, 0:q]^T - S[p,q] into the slot; R's
+        // (p,q) block (holding the staged Wt) becomes S: the sweep adds the S
+        // terms of the row-side sums through R
+        if (mine) {  // three warps
+            Block3 b;
+            product3(b, role, sR, RSC, sLA, S3 * q + 4, q * S3);
+            finish3(b, role, sW, WSC, sR + q * S3, RSC, pp > 0);
+        }
+        __syncthreads();
+        stage_phase(e + 1);  // lands while this phase sweeps
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (mine) {
+            float *ps_buf = sPS, *pu_buf = sPU;
+            if (role == 0) {
+                // ---- entry warp (lane = column b): rounds entry (d - b, b) at step d
+                const int b = lane, tb = q * S3 + b;
+                auto row_consts = [&](int a, float &w0, float &lbn, float &sv, float &rv_, float &s0) {
+                    const int ac = min(max(a, 0), S3 - 1);
+                    w0 = sW[ac * WSC + b];
+                    lbn = sLBd[ac];
+                    sv = scale[ac];
+                    rv_ = rcp[ac];
+                    s0 = sR[ac * RSC + tb];  // S[a][b] until this entry overwrites it
+                };
+                auto sweep = [&](auto ieee_tag) {
+                    constexpr bool kIeee = decltype(ieee_tag)::value;
+                    float w0, lb_new, sc_s, sc_r, s_ab;
+                    row_consts(-b, w0, lb_new, sc_s, sc_r, s_ab);
+                    float d_prev = 0.f;
+#pragma unroll 2
+                    for (int d = 0; d < 2 * S3 - 1; ++d) {
+                        const int a = d - b;
+                        const int ac = min(max(a, 0), S3 - 1);
+                        // the values the previous step produced (the other warps' sums
+                        // leave out the newest row and column terms, added here)
+                        const float ps_in = d > 0 ? ps_buf[(d & 1) * S3 + b] : 0.f;
+                        const float pu_in = d > 0 ? pu_buf[(d & 1) * S3 + b] : 0.f;
+                        const float r_new = b > 0 ? sR[ac * RSC + tb - 1] : 0.f;
+                        float w0n, lbn_n, sn, rn, s_n;
+                        row_consts(a + 1, w0n, lbn_n, sn, rn, s_n);
+                        const float sc = fmaf(lb_new, d_prev, ps_in);
+                        const float wt = w0 - fmaf(r_new, la_new, pu_in) - sc;
+                        // clamp(rint(wt / s)) with the correctly rounded fp32 quotient
+                        const float qf = kIeee ? __fdiv_rn(wt, sc_s) : div_rn_recip(wt, sc_s, sc_r);
+                        const float cq = fminf(fmaxf(rintf(qf), fqmin), fqmax);
+                        const bool valid = a >= 0 && a < mrb && tb < nc;
+                        const float dl = valid ? fmaf(-sc_s, cq, wt) : 0.f;
+                        // invalid lanes write to spare slots instead of branching
+                        const int iR = valid ? a * RSC + tb : S3 * RSC + lane;
+                        const int iD = valid ? tb * DSC + a : T * DSC + lane;
+                        const int iC = valid ? a * T + tb : S3 * T + lane;
+                        const int iW = valid ? a * WSC + b : ac * WSC + S3 + (lane & 3);  // row padding
+                        sR[iR] = s_ab + sc + dl;
+                        sDt[iD] = dl;
+                        sCode[iC] = code_byte(cq);
+                        sW[iW] = wt;  // pre-rounding value, copied out when requested
+                        d_prev = dl;
+                        w0 = w0n; lb_new = lbn_n; sc_s = sn; sc_r = rn; s_ab = s_n;
+                        group_sync(1, kThreadsC);
+                    }
+                };
+                if (exact_div)
+                    sweep(std::true_type{});
+                else
+                    sweep(std::false_type{});
+            } else if (role == 1) {
+                // ---- row-side warp (lane = column b): sum_{c <= b-2} R[a+1][c] LtA[b][c]
+                // for the entry warp's next entry (a+1, b); column b-1 of that R
+                // row is written during this step, its coefficient here is zero
+                const int b = lane;
+                float4 rv[S3 / 4];
+#pragma unroll
+                for (int c = 0; c < S3 / 4; ++c) rv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                for (int d = 0; d < 2 * S3 - 1; ++d) {
+                    const int an = min(max(d - b + 1, 0), S3 - 1);
+                    const float *Rn = sR + an * RSC + q * S3;
+#pragma unroll
+                    for (int c = 0; c < S3 / 4; ++c)
+                        if (4 * c <= b - 2) rv[c] = *(const float4 *)(Rn + 4 * c);
+                    float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
+                    float2 u2 = make_float2(0.f, 0.f), u3 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int c = 0; c < S3 / 4; c += 2) {
+                        u0 = ffma2(make_float2(rv[c].x, rv[c].y), la[2 * c], u0);
+                        u1 = ffma2(make_float2(rv[c].z, rv[c].w), la[2 * c + 1], u1);
+                        u2 = ffma2(make_float2(rv[c + 1].x, rv[c + 1].y), la[2 * c + 2], u2);
+                        u3 = ffma2(make_float2(rv[c + 1].z, rv[c + 1].w), la[2 * c + 3], u3);
+                    }
+                    pu_buf[((d + 1) & 1) * S3 + b] = ((u0.x + u1.x) + (u2.x + u3.x)) + ((u0.y + u1.y) + (u2.y + u3.y));
+                    group_sync(1, kThreadsC);
+                }
+            } else {
+                // ---- column-side warp (lane = row rho): sum_{r <= rho-2} LtB[rho][r] D[r][b]
+                // for the entry warp's entry (rho, b = d+1-rho) at step d+1; row
+                // rho-1 of that D column is written during this step, its
+                // coefficient here is zero
+                const int rho = lane;
+                float4 dv[S3 / 4];
+#pragma unroll
+                for (int c = 0; c < S3 / 4; ++c) dv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                for (int d = 0; d < 2 * S3 - 1; ++d) {
+                    const int b = d + 1 - rho;
+                    const int bc = min(max(b, 0), S3 - 1);
+                    const float *Dc = sDt + (q * S3 + bc) * DSC;
+#pragma unroll
+                    for (int c = 0; c < S3 / 4; ++c)
+                        if (4 * c <= rho - 2) dv[c] = *(const float4 *)(Dc + 4 * c);
+                    float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+                    float2 s2 = make_float2(0.f, 0.f), s3 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int c = 0; c < S3 / 4; c += 2) {
+                        s0 = ffma2(make_float2(dv[c].x, dv[c].y), lbr[2 * c], s0);
+                        s1 = ffma2(make_float2(dv[c].z, dv[c].w), lbr[2 * c + 1], s1);
+                        s2 = ffma2(make_float2(dv[c + 1].x, dv[c + 1].y), lbr[2 * c + 2], s2);
+                        s3 = ffma2(make_float2(dv[c + 1].z, dv[c + 1].w), lbr[2 * c + 3], s3);
+                    }
+                    if (b == bc)
+                        ps_buf[((d + 1) & 1) * S3 + b] = ((s0.x + s1.x) + (s2.x + s3.x)) + ((s0.y + s1.y) + (s2.y + s3.y));
+                    group_sync(1, kThreadsC);
+                }
+            }
+        }
+        __syncthreads();
+        if (p.wt_out && mine) {  // the pre-rounding values of this phase's sub-tile
+            for (int idx = tid; idx < S3 * S3; idx += kThreadsC) {
+                const int r = idx / S3, c = idx % S3;
+                if (r < mrb && q * S3 + c < nc) p.wt_out[(brow0 + r) * p.n + col0 + q * S3 + c] = sW[r * WSC + c];
+            }
+        }
+    }
+    pdl_trigger();
+    for (int idx = tid; idx < S3 * T; idx += kThreadsC) {  // V = s * code, residual split
+        const int r = idx / T, c = idx % T;
+        if (r >= mrb || c >= nc) continue;
+        const int64_t gi = brow0 + r, gj = col0 + c;
+        const int8_t code = sCode[r * T + c];
+        p.codes[gi * p.n + gj] = code;
+        p.V[gi * p.n + gj] = scale[r] * (float)code;
+        float hi, lo;
+        split_tf32(sDt[c * DSC + r], hi, lo);
+        p.Dhi[gi * p.Np + gj] = hi;
+        p.Dlo[gi * p.Np + gj] = lo;
+    }
+    // the other CTAs may still read this CTA's D until their last phase
+    cluster.sync();
+}
+
+cudaError_t leaf_cluster_configure()
+{
+    return cudaFuncSetAttribute(leaf_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSmemCLaunch);
+}
+
+cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, cudaStream_t stream)
+{
+    return launch_pdl(leaf_cluster_kernel, dim3(4 * tiles), dim3(kThreadsC), kSmemCLaunch, stream, p, K, I_lo);
+}
+
+}  // namespace bakron

@@ -2,14 +2,18 @@
 // fixed device array that the library owns, for callers that may not
 // allocate device memory themselves (see include/bakron.h).
 //
-// The array is a file-scope __device__ variable, so the CUDA module loader
-// reserves it on every GPU that loads this library, and it stays reserved
-// until the process exits.  Host code cannot use the array's name as a device
-// address: the address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, and cached.
+// The array is a file-scope __device__ variable.  This file is its own code
+// module, and under CUDA's lazy module loading (the default) the driver loads
+// the module, and so reserves the array on a device, at the first use of the
+// array's address on that device; with CUDA_MODULE_LOADING=EAGER it is
+// reserved when the library loads.  It stays reserved until the process
+// exits.  Host code cannot use the array's name as a device address: the
+// address is looked up once per device with cudaGetSymbolAddress, with that
+// device current, and cached.
 #include <mutex>
 
 #include "common.cuh"
+#include "kernels.cuh"
 
 namespace {
 
@@ -54,16 +58,25 @@ extern "C" bakron_status_t bakron_solve_noalloc(const float *W_dev, int64_t m, i
     const size_t need = bakron_solve_workspace_size(m, n, cfg);
     if (need == 0) return BAKRON_ERR_INVALID_ARG;
     if (need > kScratchBytes) return BAKRON_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (device_status_host) {
+        // reading the status back synchronises the stream, which a stream
+        // being captured into a graph does not allow
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return BAKRON_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return BAKRON_ERR_INVALID_ARG;
+    }
     void *ws = nullptr;
     if (scratch_address(&ws) != cudaSuccess) return BAKRON_ERR_CUDA;
-    // bakron_solve clears the status block and rewrites every other part of
-    // the workspace it reads (the residual buffers are zeroed by its prep step),
-    // so nothing left by an earlier call leaks into this one.
-    bakron_status_t s = bakron_solve(W_dev, m, n, LA_dev, LB_dev, q, V_dev, codes_dev, scales_dev, ws,
-                                     kScratchBytes, cfg, stream);
+    // Direct launches only: the graph mode (cfg->use_graph, BAKRON_GRAPH)
+    // creates a stream and executable graphs, which allocate.  The solve
+    // clears the status block and rewrites every other part of the workspace
+    // it reads (the residual buffers are zeroed by its preparation step), so
+    // nothing left by an earlier call leaks into this one.
+    bakron_status_t s = bakron::solve_direct(W_dev, m, n, LA_dev, LB_dev, q, V_dev, codes_dev, scales_dev, ws,
+                                             kScratchBytes, cfg, st);
     if (s != BAKRON_OK) return s;
     if (device_status_host) {
-        cudaStream_t st = (cudaStream_t)stream;
         int32_t code = 0;
         if (cudaMemcpyAsync(&code, ws, sizeof(code), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
             cudaStreamSynchronize(st) != cudaSuccess)
