@@ -32,7 +32,8 @@ TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 : BF16 tensor peak ratio
 FALLBACK_BF16_TFLOPS = 1590.0
 LEAF_BYTES_PER_WEIGHT = 25  # read Wt 4 + diagonal factor blocks 8; write code 1, V 4, D hi/lo 8
 LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 255), 3: ("leaf_warp_kernel", 7 * 63),
-                4: ("leaf_wide_kernel", 3 * 127), 5: ("leaf_cluster_kernel", 7 * 63)}
+                4: ("leaf_wide_kernel", 3 * 127), 5: ("leaf_cluster_kernel<false>", 7 * 63),
+                6: ("leaf_cluster_kernel<true>", 7 * 63)}
 # DRAM traffic of the band products from an ncu capture of one solve's 124
 # band launches (profiles/band_tc_4096_dram.md); reported only while the
 # kernel sources hash to the value the capture was taken with.
@@ -313,6 +314,90 @@ def config_block(w, args):
             "parallelism": f"replicas x{args.gpus}", "l2": l2}
 
 
+def extra_measurements(args, bk, w, Wd, LA, LB, W, codes, ws, stream, dev, dist, leaf, fw, n_batch):
+    """End to end through the host-buffer entry point, several matrices at
+    once, and the one-sided path: (e2e ms, batch ms, one-sided ms) per step."""
+    import numpy as np
+    import torch
+
+    m, n = W.shape
+    # e2e through the host-buffer entry point: H2D of W, LA, LB and D2H of V,
+    # codes, scales inside the timed region, every step
+    Wh = torch.from_numpy(W).pin_memory()
+    LAh, LBh = LA.cpu().pin_memory(), LB.cpu().pin_memory()
+    Vh = torch.empty((m, n), dtype=torch.float32).pin_memory()
+    ch = torch.empty((m, n), dtype=torch.int8).pin_memory()
+    sh = torch.empty((m,), dtype=torch.float32).pin_memory()
+    wsh = bk.workspace(bk.solve_host_workspace_size(m, n), dev)
+    for _ in range(2):
+        bk.solve_host(Wh, LAh, LBh, bits=w.bits, V=Vh, codes=ch, scales=sh, ws=wsh, stream=stream, leaf=leaf,
+                      fuse_width=fw)
+    torch.cuda.synchronize()
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, args.steps // 2)
+    h0.record(stream)
+    for _ in range(e2e_steps):
+        bk.solve_host(Wh, LAh, LBh, bits=w.bits, V=Vh, codes=ch, scales=sh, ws=wsh, stream=stream, synchronize=False,
+                      leaf=leaf, fuse_width=fw)
+    h1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(h0.elapsed_time(h1) / e2e_steps, dist, dev)
+    assert np.array_equal(ch.numpy(), codes.cpu().numpy()), "host-buffer solve disagrees with device solve"
+
+    # several matrices at once (bakron_solve_batch on separate streams): one
+    # solve keeps few SMs busy during its leaf sweeps, so solves overlap
+    n_batch = 4
+    bstreams = [torch.cuda.Stream(device=dev) for _ in range(n_batch)]
+    bouts = [(torch.empty((m, n), dtype=torch.float32, device=dev), torch.empty((m, n), dtype=torch.int8, device=dev),
+              torch.empty((m,), dtype=torch.float32, device=dev)) for _ in range(n_batch)]
+    bws = [bk.workspace(bk.solve_workspace_size(m, n), dev) for _ in range(n_batch)]
+    probs = [(Wd, LA, LB)] * n_batch
+
+    def batch_step():
+        start = torch.cuda.Event()
+        start.record(stream)
+        for bs in bstreams:
+            bs.wait_event(start)
+        bk.solve_batch(probs, bits=w.bits, streams=bstreams, outs=bouts, workspaces=bws, leaf=leaf,
+                       check_status=False, fuse_width=fw)
+        for bs in bstreams:
+            done = torch.cuda.Event()
+            done.record(bs)
+            stream.wait_event(done)
+
+    for _ in range(2):
+        batch_step()
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b_steps = 3
+    b0.record(stream)
+    for _ in range(b_steps):
+        batch_step()
+    b1.record(stream)
+    torch.cuda.synchronize()
+    batch_ms = max_over_ranks(b0.elapsed_time(b1) / b_steps, dist, dev)
+    assert torch.equal(bouts[-1][1], codes), "batched solve disagrees with the single solve"
+    del bws, bouts
+
+    # the one-sided path (B = I: GPTQ with Hessian A) on the same W and A
+    o_out = (torch.empty_like(Wd), torch.empty((m, n), dtype=torch.int8, device=dev),
+             torch.empty((m,), dtype=torch.float32, device=dev))
+    for _ in range(2):
+        bk.solve(Wd, LA, None, bits=w.bits, ws=ws, out=o_out, stream=stream)
+    torch.cuda.synchronize()
+    o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    o_steps = 5
+    o0.record(stream)
+    for _ in range(o_steps):
+        bk.solve(Wd, LA, None, bits=w.bits, ws=ws, out=o_out, stream=stream, check_status=False)
+    o1.record(stream)
+    torch.cuda.synchronize()
+    one_ms = max_over_ranks(o0.elapsed_time(o1) / o_steps, dist, dev)
+    del o_out
+
+    return e2e_ms, batch_ms, one_ms
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -322,6 +407,11 @@ def main():
     ap.add_argument("--workload", default="bench")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=3)
+    ap.add_argument("--leaf", type=int, default=0,
+                    help="leaf structure (bakron_config_t.leaf); 0 picks it by measurement (bakron_tune_leaf)")
+    ap.add_argument("--fuse-width", type=int, default=0, help="bakron_config_t.fuse_width (0 = library default)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="profiling runs: skip the host-buffer, batched and one-sided measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -360,10 +450,15 @@ def main():
     stream = torch.cuda.current_stream()
 
     # the schedule's leaf structure, picked by measurement on this problem
-    leaf, leaf_tune_ms = bk.tune_leaf(Wd, LA, LB, bits=w.bits, ws=ws, out=out, stream=stream)
+    fw = args.fuse_width
+    if args.leaf > 0:
+        leaf, leaf_tune_ms = args.leaf, None
+    else:
+        leaf, leaf_tune_ms = bk.tune_leaf(Wd, LA, LB, bits=w.bits, ws=ws, out=out, stream=stream)
 
     def step():
-        bk.solve(Wd, LA, LB, bits=w.bits, ws=ws, out=out, check_status=False, stream=stream, leaf=leaf)
+        bk.solve(Wd, LA, LB, bits=w.bits, ws=ws, out=out, check_status=False, stream=stream, leaf=leaf,
+                 fuse_width=fw)
 
     for _ in range(args.warmup):
         step()
@@ -392,7 +487,7 @@ def main():
     prof, launches = [], []
     for _ in range(max(1, args.profile_steps)):
         bk.solve(Wd, LA, LB, bits=w.bits, ws=ws, out=out, check_status=False, stream=stream, profile=True,
-                 leaf=leaf)
+                 leaf=leaf, fuse_width=fw)
         prof.append(bk.last_profile())
         launches.append(bk.last_profile_launches())
     pr = {k: statistics.median(p[k] for p in prof) for k in prof[0]}
@@ -407,78 +502,11 @@ def main():
     launches_per_step = int(pr["prep_launches"] + pr["leaf_launches"] + pr["stage1_launches"] +
                             pr["stage2_launches"] + pr["fused_launches"])
 
-    # e2e through the host-buffer entry point: H2D of W, LA, LB and D2H of V,
-    # codes, scales inside the timed region, every step
-    Wh = torch.from_numpy(W).pin_memory()
-    LAh, LBh = LA.cpu().pin_memory(), LB.cpu().pin_memory()
-    Vh = torch.empty((m, n), dtype=torch.float32).pin_memory()
-    ch = torch.empty((m, n), dtype=torch.int8).pin_memory()
-    sh = torch.empty((m,), dtype=torch.float32).pin_memory()
-    wsh = bk.workspace(bk.solve_host_workspace_size(m, n), dev)
-    for _ in range(2):
-        bk.solve_host(Wh, LAh, LBh, bits=w.bits, V=Vh, codes=ch, scales=sh, ws=wsh, stream=stream, leaf=leaf)
-    torch.cuda.synchronize()
-    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(3, args.steps // 2)
-    h0.record(stream)
-    for _ in range(e2e_steps):
-        bk.solve_host(Wh, LAh, LBh, bits=w.bits, V=Vh, codes=ch, scales=sh, ws=wsh, stream=stream, synchronize=False,
-                      leaf=leaf)
-    h1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(h0.elapsed_time(h1) / e2e_steps, dist, dev)
-    assert np.array_equal(ch.numpy(), codes.cpu().numpy()), "host-buffer solve disagrees with device solve"
-
-    # several matrices at once (bakron_solve_batch on separate streams): one
-    # solve keeps few SMs busy during its leaf sweeps, so solves overlap
+    e2e_ms = batch_ms = one_ms = None
     n_batch = 4
-    bstreams = [torch.cuda.Stream(device=dev) for _ in range(n_batch)]
-    bouts = [(torch.empty((m, n), dtype=torch.float32, device=dev), torch.empty((m, n), dtype=torch.int8, device=dev),
-              torch.empty((m,), dtype=torch.float32, device=dev)) for _ in range(n_batch)]
-    bws = [bk.workspace(bk.solve_workspace_size(m, n), dev) for _ in range(n_batch)]
-    probs = [(Wd, LA, LB)] * n_batch
-
-    def batch_step():
-        start = torch.cuda.Event()
-        start.record(stream)
-        for bs in bstreams:
-            bs.wait_event(start)
-        bk.solve_batch(probs, bits=w.bits, streams=bstreams, outs=bouts, workspaces=bws, leaf=leaf,
-                       check_status=False)
-        for bs in bstreams:
-            done = torch.cuda.Event()
-            done.record(bs)
-            stream.wait_event(done)
-
-    for _ in range(2):
-        batch_step()
-    torch.cuda.synchronize()
-    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    b_steps = 3
-    b0.record(stream)
-    for _ in range(b_steps):
-        batch_step()
-    b1.record(stream)
-    torch.cuda.synchronize()
-    batch_ms = max_over_ranks(b0.elapsed_time(b1) / b_steps, dist, dev)
-    assert torch.equal(bouts[-1][1], codes), "batched solve disagrees with the single solve"
-    del bws, bouts
-
-    # the one-sided path (B = I: GPTQ with Hessian A) on the same W and A
-    o_out = (torch.empty_like(Wd), torch.empty((m, n), dtype=torch.int8, device=dev),
-             torch.empty((m,), dtype=torch.float32, device=dev))
-    for _ in range(2):
-        bk.solve(Wd, LA, None, bits=w.bits, ws=ws, out=o_out, stream=stream)
-    torch.cuda.synchronize()
-    o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    o_steps = 5
-    o0.record(stream)
-    for _ in range(o_steps):
-        bk.solve(Wd, LA, None, bits=w.bits, ws=ws, out=o_out, stream=stream, check_status=False)
-    o1.record(stream)
-    torch.cuda.synchronize()
-    one_ms = max_over_ranks(o0.elapsed_time(o1) / o_steps, dist, dev)
-    del o_out
+    if not args.no_extras:
+        e2e_ms, batch_ms, one_ms = extra_measurements(args, bk, w, Wd, LA, LB, W, codes, ws, stream, dev, dist,
+                                                      leaf, fw, n_batch)
 
     line = None
     if rank == 0:
@@ -505,7 +533,7 @@ def main():
                 "band_ms_per_step": gemm_ms,
                 "fused_nodes_per_step": int(pr["fused_launches"])},
             "band_levels": levels,
-            "leaf": {"kernel": LEAF_KERNELS[leaf][0], "structure": leaf, "tune_ms": dict(zip(bk.LEAF_STRUCTURES, leaf_tune_ms)),
+            "leaf": {"kernel": LEAF_KERNELS[leaf][0], "structure": leaf, "tune_ms": None if leaf_tune_ms is None else dict(zip(bk.LEAF_STRUCTURES, leaf_tune_ms)),
                      "ms_per_step": pr["leaf_ms"],
                      "launches_per_step": pr["leaf_launches"],
                      "achieved_gbs": leaf_bytes / (pr["leaf_ms"] / 1e3) / 1e9, "hbm_peak_gbs": hbm,
@@ -516,15 +544,18 @@ def main():
             "profile_ms": pr,
             "factor_ms": factor_ms,
             "cpu_baseline": cb,
-            "e2e": {"value": aggregate_rate(world, m, n, e2e_ms), "unit": "weights/s",
-                    "h2d_bytes_per_step": 4 * (m * n + n * n + m * m),
-                    "d2h_bytes_per_step": 4 * m * n + m * n + 4 * m},
-            "batch": {"matrices_per_step": n_batch, "streams": n_batch, "ms_per_step": batch_ms,
-                      "value": aggregate_rate(world, m, n, batch_ms / n_batch), "unit": "weights/s",
-                      "note": "bakron_solve_batch of the same workload on separate streams (not the headline)"},
-            "one_sided": {"ms_per_step": one_ms, "value": aggregate_rate(world, m, n, one_ms), "unit": "weights/s",
-                          "note": "B = I path (one-sided GPTQ with Hessian A, column-block recursion) on the same "
-                                  "W and A (not the headline)"},
+            "e2e": None if e2e_ms is None else {
+                "value": aggregate_rate(world, m, n, e2e_ms), "unit": "weights/s",
+                "h2d_bytes_per_step": 4 * (m * n + n * n + m * m),
+                "d2h_bytes_per_step": 4 * m * n + m * n + 4 * m},
+            "batch": None if batch_ms is None else {
+                "matrices_per_step": n_batch, "streams": n_batch, "ms_per_step": batch_ms,
+                "value": aggregate_rate(world, m, n, batch_ms / n_batch), "unit": "weights/s",
+                "note": "bakron_solve_batch of the same workload on separate streams (not the headline)"},
+            "one_sided": None if one_ms is None else {
+                "ms_per_step": one_ms, "value": aggregate_rate(world, m, n, one_ms), "unit": "weights/s",
+                "note": "B = I path (one-sided GPTQ with Hessian A, column-block recursion) on the same W and A "
+                        "(not the headline)"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "device_status": status.name,

@@ -86,7 +86,7 @@ typedef struct {
 } bakron_quantizer_t;
 
 /* Solver configuration (NULL = defaults; zero fields take defaults).
- * The environment can change the defaults of five fields: BAKRON_LEAF (0..5),
+ * The environment can change the defaults of five fields: BAKRON_LEAF (0..6),
  * BAKRON_GEMM (0..1), BAKRON_TIMEOUT_MS (1..600000), BAKRON_GRAPH (0..1,
  * ignored when profile = 1) and BAKRON_FUSE (1..65535, the default
  * fuse_width); a non-zero field set by the caller wins.  A
@@ -116,14 +116,16 @@ typedef struct {
     int32_t profile;  /* 1: time every kernel class with CUDA events on `stream`;
                          the call then synchronises `stream` before returning and
                          the durations are read with bakron_get_profile(). */
-    int32_t leaf;     /* leaf sweep structure: 0 = default (5); 1 = each tile as
+    int32_t leaf;     /* leaf sweep structure: 0 = default (6); 1 = each tile as
                          2 x 2 sub-tiles of 64 swept by the whole CTA; 2 = one
                          anti-diagonal sweep over the whole 128 x 128 tile; 3 =
                          4 x 4 sub-tiles of 32, each swept by three warps; 4 =
                          2 x 2 sub-tiles of 64, each swept by six warps; 5 = as
                          3 with each tile on a cluster of four CTAs, one per
-                         row block of sub-tiles (bakron_tune_leaf picks one by
-                         measurement). */
+                         row block of sub-tiles; 6 = as 5 with a fourth warp
+                         per CTA forming the older product terms of the next
+                         sub-tile during each sweep (bakron_tune_leaf picks
+                         one by measurement). */
     int32_t b_identity; /* 1: B = I (one-sided GPTQ with Hessian A, the case the
                            two-sided solve reduces to when B = I).  LB_dev may be
                            NULL and is not read; rows are independent, so the
@@ -231,7 +233,7 @@ bakron_status_t bakron_solve(const float *W_dev, int64_t m, int64_t n, const flo
  * bakron_solve on the caller's problem once per structure after one warm-up
  * solve, timing each with CUDA events on `stream` (the call synchronises
  * `stream`), and writes the fastest structure (a bakron_config_t.leaf value,
- * 1..5) to *leaf_out and the five times in ms to ms_out[0..4] (leaf 1..5;
+ * 1..6) to *leaf_out and the six times in ms to ms_out[0..5] (leaf 1..6;
  * ms_out may be NULL).  Arguments as for bakron_solve; cfg->leaf is ignored
  * and cfg->profile must be 0.  V, codes and scales hold the last solve's
  * results (all structures give the same codes up to rounding ties).  Device

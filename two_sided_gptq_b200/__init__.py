@@ -25,7 +25,7 @@ __all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_pr
 
 
 # bakron_config_t.leaf values bakron_tune_leaf times (one ms_out entry each)
-LEAF_STRUCTURES = (1, 2, 3, 4, 5)
+LEAF_STRUCTURES = (1, 2, 3, 4, 5, 6)
 
 
 def _lib():
@@ -139,10 +139,11 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     ``gemm=0`` uses the tcgen05 3xTF32 band products, ``gemm=1`` the FP32
     CUDA-core ones; ``shrink_grid`` > 1 searches each row's step for the least
     round-to-nearest error over that many shrink factors in [1/2, 1]; ``leaf``
-    selects the leaf sweep structure (0 default (5),
+    selects the leaf sweep structure (0 default (6),
     1 two-level CTA-wide, 2 single-level, 3 three warps per 32 x 32
     sub-tile, 4 six warps per 64 x 64 sub-tile, 5 as 3 with each tile on a
-    cluster of four CTAs; :func:`tune_leaf` picks one by measurement).  ``fuse_width`` (0 default, 1 never) runs the two band
+    cluster of four CTAs, 6 as 5 with the older product terms formed during
+    the sweeps; :func:`tune_leaf` picks one by measurement).  ``fuse_width`` (0 default, 1 never) runs the two band
     products of recursion nodes at most that many tile diagonals wide as one
     launch per target tile.  ``graph=True`` captures the solve's launches for this
     argument set into a CUDA graph on the first call and replays it on later
@@ -225,7 +226,7 @@ def tune_cache_put(path: str, key: str, leaf: int, ms) -> None:
 def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, timeout_ms=0, cache=None):
     """Leaf structure chosen by measurement (``bakron_tune_leaf``): one timed
     solve per structure on this problem.  Returns ``(leaf, [ms_leaf1, ...,
-    ms_leaf5])``; pass ``leaf`` to :func:`solve`.
+    ms_leaf6])``; pass ``leaf`` to :func:`solve`.
 
     ``cache`` (or the ``BAKRON_TUNE_CACHE`` environment variable) names a JSON
     file keyed by (m, n, bits, GPU name): a stored measurement is returned
@@ -265,7 +266,7 @@ def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, time
 
 
 def solve_batch(problems, bits=4, *, streams, outs=None, workspaces=None, gemm=0, leaf=0, shrink_grid=0,
-                check_status=True):
+                check_status=True, fuse_width=0):
     """Independent solves through ``bakron_solve_batch``: ``problems`` is a list
     of ``(W, LA, LB)`` device tensors, solve i runs on ``streams[i %
     len(streams)]`` (torch streams).  ``outs`` / ``workspaces`` may supply the
@@ -273,7 +274,7 @@ def solve_batch(problems, bits=4, *, streams, outs=None, workspaces=None, gemm=0
     ``(V, codes, scales)``."""
     torch = _torch()
     lib = _lib()
-    cfg = _config(gemm, leaf=leaf)
+    cfg = _config(gemm, leaf=leaf, fuse_width=fuse_width)
     items = (BatchItem * max(1, len(problems)))()
     res, wss = [], []
     for i, (W, LA, LB) in enumerate(problems):
@@ -324,7 +325,7 @@ def solve_host_workspace_size(m: int, n: int, gemm: int = 0) -> int:
 
 
 def solve_host(W, LA, LB, bits=4, *, V=None, codes=None, scales=None, gemm=0, ws=None, stream=None,
-               synchronize=True, leaf=0):
+               synchronize=True, leaf=0, fuse_width=0):
     """BaKron solve on HOST buffers (torch CPU tensors, ideally pinned): the
     library stages them through ``ws`` on the device and copies the results
     back.  Returns ``(V, codes, scales)`` host tensors."""
@@ -339,7 +340,7 @@ def solve_host(W, LA, LB, bits=4, *, V=None, codes=None, scales=None, gemm=0, ws
     V = torch.empty((m, n), dtype=torch.float32, pin_memory=True) if V is None else V
     codes = torch.empty((m, n), dtype=torch.int8, pin_memory=True) if codes is None else codes
     scales = torch.empty((m,), dtype=torch.float32, pin_memory=True) if scales is None else scales
-    cfg = _config(gemm, leaf=leaf, b_identity=int(LB is None))
+    cfg = _config(gemm, leaf=leaf, b_identity=int(LB is None), fuse_width=fuse_width)
     if ws is None:
         ws = workspace(lib.bakron_solve_host_workspace_size(m, n, ctypes.byref(cfg)))
     q = Quantizer(int(bits), 0, 0, 0)

@@ -30,8 +30,8 @@ constexpr const char *kVersion = "bakron-b200 0.2";
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Leaf structures bakron_tune_leaf times (bakron_config_t.leaf 1..5).
-constexpr int kLeafStructures = 5;
+// Leaf structures bakron_tune_leaf times (bakron_config_t.leaf 1..6).
+constexpr int kLeafStructures = 6;
 
 // Nodes at most this many tile diagonals wide run fused by default (measured
 // on B200 at 4096^2: width 2 trims the profiled band time, wider fusing is
@@ -39,8 +39,9 @@ constexpr int kLeafStructures = 5;
 constexpr int kDefaultFuseWidth = 2;
 
 struct Config {
-    // leaf: structure 5 (a cluster of four CTAs per tile), the fastest measured
-    int tile = kTile, gemm = 0, use_graph = 0, timeout_ms = 200, profile = 0, leaf = 4, b_identity = 0;
+    // leaf: structure 6 (a cluster of four CTAs per tile, older product terms
+    // formed during the sweeps), the fastest measured
+    int tile = kTile, gemm = 0, use_graph = 0, timeout_ms = 200, profile = 0, leaf = 5, b_identity = 0;
     int fuse_width = kDefaultFuseWidth;
     float *wt_out = nullptr;
 };
@@ -136,7 +137,7 @@ bakron_status_t read_config(const bakron_config_t *c, Config &out)
     // defaults that BAKRON_LEAF, BAKRON_GEMM, BAKRON_TIMEOUT_MS and BAKRON_GRAPH
     // override; a non-zero field of the caller's config overrides both
     int leaf = 0, gemm = 0, graph = 0;
-    if (!env_int("BAKRON_LEAF", 0, 5, leaf) || !env_int("BAKRON_GEMM", 0, 1, gemm) ||
+    if (!env_int("BAKRON_LEAF", 0, kLeafStructures, leaf) || !env_int("BAKRON_GEMM", 0, 1, gemm) ||
         !env_int("BAKRON_TIMEOUT_MS", 1, 600000, out.timeout_ms) || !env_int("BAKRON_GRAPH", 0, 1, graph) ||
         !env_int("BAKRON_FUSE", 1, 65535, out.fuse_width))
         return BAKRON_ERR_INVALID_ARG;
@@ -153,7 +154,7 @@ bakron_status_t read_config(const bakron_config_t *c, Config &out)
     if (c->timeout_ms > 0) out.timeout_ms = c->timeout_ms;
     out.wt_out = c->wt_out;
     out.profile = c->profile ? 1 : 0;
-    if (c->leaf < 0 || c->leaf > 5) return BAKRON_ERR_INVALID_ARG;
+    if (c->leaf < 0 || c->leaf > kLeafStructures) return BAKRON_ERR_INVALID_ARG;
     if (c->leaf != 0) out.leaf = c->leaf - 1;  // 0 keeps the default
     if (c->b_identity < 0 || c->b_identity > 1) return BAKRON_ERR_INVALID_ARG;
     out.b_identity = c->b_identity;

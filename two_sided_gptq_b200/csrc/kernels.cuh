@@ -37,9 +37,10 @@ cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, c
 
 cudaError_t leaf_configure();
 cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stream);
-// Leaf with one tile per cluster of four CTAs (leaf_cluster.cu).
+// Leaf with one tile per cluster of four CTAs (leaf_cluster.cu); overlap:
+// a fourth warp forms the older product terms during the sweeps.
 cudaError_t leaf_cluster_configure();
-cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, cudaStream_t stream);
+cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, bool overlap, cudaStream_t stream);
 
 // FP32 CUDA-core band products (reference kernels for the tensor-core path).
 cudaError_t launch_band_simt(int stage, const NodeParams &np, const GemmArgs &g, cudaStream_t stream);

@@ -18,6 +18,17 @@
 // opens each phase; R and everything else stays local.  Every CTA passes the
 // same eight cluster barriers, so the waits are those of a hardware barrier
 // with equal trip counts.
+//
+// Overlapped form (kOverlap, structure 6): of the two products only the
+// newest 32-deep terms, LtB[p,p-1] D[p-1,q] and R[p,q-1] LtA[q,q-1]^T, depend
+// on the phase just finished.  A fourth warp per CTA forms the older terms
+// of the CTA's next sub-tile,
+//     O_S = sum_{p' <= p-2} LtB[p,p'] D[p',q+1],
+//     O_U = sum_{q' <= q-1} R[p,q'] LtA[q+1,q']^T,
+// while the three sweep warps round the current one (it also stages the next
+// sub-tile's Wt block and LtA strip and fetches the older D blocks from the
+// other CTAs), so between two sweeps only the newest terms remain, shared by
+// all four warps.
 #include <cooperative_groups.h>
 
 #include <type_traits>
@@ -35,12 +46,12 @@ using namespace leafk;
 namespace {
 constexpr int T = kTile;
 constexpr int S3 = 32;            // sub-tile side
-constexpr int kThreadsC = 96;     // entry, row-side and column-side warps
+constexpr int kSweepThreads = 96;  // entry, row-side and column-side warps
 constexpr int RSC = T + 4;        // row stride of sR (32 rows x 128 columns)
 constexpr int DSC = S3 + 4;       // row stride of sDt (128 columns x 32 rows)
 constexpr int WSC = S3 + 4;       // row stride of the sub-tile slot
 constexpr int LSC = 3 * S3 + 4;   // row stride of strips of up to three 32-wide blocks
-constexpr size_t kSmemC = ((size_t)(S3 + 1) * RSC + (size_t)(T + 1) * DSC + (size_t)S3 * WSC +
+constexpr size_t kSmemC = ((size_t)(S3 + 1) * RSC + (size_t)(T + 1) * DSC + (size_t)3 * S3 * WSC +
                            (size_t)3 * S3 * LSC + 3 * S3 + 4 * S3) * sizeof(float) +
                           (size_t)S3 * T + 32;
 // Requested per CTA so that two CTAs never share an SM: the point of the
@@ -49,9 +60,11 @@ constexpr size_t kSmemCLaunch = 120 * 1024;
 static_assert(kSmemC <= kSmemCLaunch && 2 * kSmemCLaunch > 228 * 1024, "cluster leaf shared memory");
 }  // namespace
 
-__global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreadsC, 1)
+template <bool kOverlap>
+__global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kOverlap ? 128 : 96, 1)
 leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
 {
+    constexpr int kThreadsC = kOverlap ? 128 : 96;
     cg::cluster_group cluster = cg::this_cluster();
     const int pp = (int)cluster.block_rank();  // row block of sub-tiles
 
@@ -59,7 +72,9 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
     float *sR = smem_f;                       // (S3+1) x RSC: R of this row block (S before a sweep, Wt staged)
     float *sDt = sR + (S3 + 1) * RSC;         // (T+1) x DSC: D transposed, this row block's rows, 0 until rounded
     float *sW = sDt + (T + 1) * DSC;          // S3 x WSC: S, then W0 of the sub-tile being swept
-    float *sLA = sW + S3 * WSC;               // LtA[q, 0:q] strip, row stride 32 q + 4 (staged a phase ahead)
+    float *sOS = sW + S3 * WSC;               // S3 x WSC: older column-side terms O_S of the next sub-tile
+    float *sOU = sOS + S3 * WSC;              // S3 x WSC: older row-side terms O_U of the next sub-tile
+    float *sLA = sOU + S3 * WSC;              // LtA[q, 0:q] strip, row stride 32 q + 4 (staged a phase ahead)
     float *sLBs = sLA + S3 * LSC;             // LtB[p, 0:p] strip, row stride 32 p + 4 (loaded once)
     float *sDr = sLBs + S3 * LSC;             // D[0:p, q] of the row blocks above: [column][32 p' + row], LSC
     float *sLBd = sDr + S3 * LSC;             // S3: LtB[r][r-1] inside the row block (0 for r = 0)
@@ -89,27 +104,37 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
         ((float4 *)sR)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int idx = tid; idx < (T + 1) * DSC / 4; idx += kThreadsC)
         ((float4 *)sDt)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int idx = tid; idx < 2 * S3 * WSC / 4; idx += kThreadsC)  // O_S, O_U
+        ((float4 *)sOS)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();  // R is zero before the first staged block lands in it
     pdl_wait();       // every global input (Wt, factors, steps) comes from earlier kernels
 
-    // Stage the sub-tile (pp, e - pp) of phase e, if it is this CTA's: its Wt
-    // block into R's block (untouched until then) and the strip LtA[q, 0:q].
-    auto stage_phase = [&](int e) {
-        const int q = e - pp;
+    // Stage the sub-tile (pp, q) -- its Wt block into R's block (untouched
+    // until then) and the strip LtA[q, 0:q] -- with threads [t0, t0 + nt).
+    auto stage_subtile = [&](int q, int t0, int nt) {
         if (q < 0 || q > 3) return;
         if (q > 0) {
             const int ld = S3 * q + 4, c4 = 8 * q;
-            for (int c = tid; c < S3 * c4; c += kThreadsC) {
+            for (int c = tid - t0; c < S3 * c4; c += nt) {
                 const int j = c / c4, k4 = c - j * c4;
                 cp_async16(sLA + j * ld + 4 * k4, LAt + (q * S3 + j) * lda_g + 4 * k4);
             }
         }
-        for (int c = tid; c < S3 * 8; c += kThreadsC) {
+        for (int c = tid - t0; c < S3 * 8; c += nt) {
             const int i = c >> 3, k4 = c & 7;
             cp_async16(sR + i * RSC + q * S3 + 4 * k4, p.Wt + (brow0 + i) * p.Np + col0 + q * S3 + 4 * k4);
         }
     };
-    stage_phase(0);
+    // D[p', q] of CTA p' (rows of row block p') into sDr, transposed, for
+    // p' in [p0, p1), with threads [t0, t0 + nt)
+    auto gather_d = [&](int q, int p0, int p1, int t0, int nt) {
+        for (int c = tid - t0; c < (p1 - p0) * S3 * 8; c += nt) {
+            const int pr = p0 + c / (S3 * 8), j = (c >> 3) % S3, r4 = c & 7;
+            const float *src = cluster.map_shared_rank(sDt, pr) + (q * S3 + j) * DSC + 4 * r4;
+            *(float4 *)(sDr + j * LSC + pr * S3 + 4 * r4) = *(const float4 *)src;
+        }
+    };
+    stage_subtile(0 - pp, 0, kThreadsC);
     if (pp > 0) {  // LtB[p, 0:p], fixed for the kernel
         const int ld = S3 * pp + 4, c4 = 8 * pp;
         for (int c = tid; c < S3 * c4; c += kThreadsC) {
@@ -120,7 +145,7 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
     asm volatile("cp.async.commit_group;" ::: "memory");
     if (tid < S3) sLBd[tid] = tid > 0 ? LBt[(pp * S3 + tid) * ldb_g + pp * S3 + tid - 1] : 0.f;
     const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
-    const int role = warp;                    // 0 entries, 1 row side, 2 column side
+    const int role = warp;  // 0 entries, 1 row side, 2 column side, 3 (overlapped form) older products
     // column-side warp: its LtB[p,p] row rho (columns <= rho-2), fixed for the kernel
     float2 lbr[S3 / 2];
     if (role == 2) {
@@ -152,19 +177,50 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
         cluster.sync();
         asm volatile("cp.async.wait_all;" ::: "memory");  // this phase's staged Wt block and strip
         if (mine && pp > 0) {
-            // D[p', q] (p' < p) from the other CTAs' shared memory, transposed
-            for (int c = tid; c < pp * S3 * 8; c += kThreadsC) {
-                const int pr = c / (S3 * 8), j = (c >> 3) % S3, r4 = c & 7;
-                const float *src = cluster.map_shared_rank(sDt, pr) + (q * S3 + j) * DSC + 4 * r4;
-                *(float4 *)(sDr + j * LSC + pr * S3 + 4 * r4) = *(const float4 *)src;
-            }
+            // D[p', q] of the row blocks above: all of them, or (overlapped
+            // form) only the newest, p' = p - 1
+            if (kOverlap)
+                gather_d(q, pp - 1, pp, 0, kThreadsC);
+            else
+                gather_d(q, 0, pp, 0, kThreadsC);
         }
         __syncthreads();
-        // S[p,q] = LtB[p, 0:p] D[0:p, q] into the slot (three warps)
-        if (mine && pp > 0) {
-            Block3 b;
-            product3(b, role, sLBs, S3 * pp + 4, sDr, LSC, pp * S3);
-            store3(b, role, sW, WSC);
+        if (!kOverlap) {
+            // S[p,q] = LtB[p, 0:p] D[0:p, q] into the slot (three warps)
+            if (mine && pp > 0) {
+                Block3 b;
+                product3(b, role, sLBs, S3 * pp + 4, sDr, LSC, pp * S3);
+                store3(b, role, sW, WSC);
+            }
+            __syncthreads();
+            // W0[p,q] = Wt[p,q] - R[p, 0:q] LtA[q, 0:q]^T - S[p,q] into the slot;
+            // R's (p,q) block (holding the staged Wt) becomes S: the sweep adds
+            // the S terms of the row-side sums through R
+            if (mine) {
+                Block3 b;
+                product3(b, role, sR, RSC, sLA, S3 * q + 4, q * S3);
+                finish3(b, role, sW, WSC, sR + q * S3, RSC, pp > 0);
+            }
+        } else if (mine) {
+            // the newest terms, four warps (16 x 16 each):
+            //   S = O_S + LtB[p,p-1] D[p-1,q],  U = O_U + R[p,q-1] LtA[q,q-1]^T,
+            //   W0 = Wt - U - S into the slot, R's (p,q) block := S
+            const int i0 = 16 * (warp & 1), j0 = 16 * (warp >> 1);
+            float as[2][4] = {}, au[2][4] = {};
+            if (pp > 0) mma_block<2>(as, sLBs + S3 * (pp - 1), S3 * pp + 4, sDr + S3 * (pp - 1), LSC, S3, i0, j0);
+            if (q > 0) mma_block<2>(au, sR + S3 * (q - 1), RSC, sLA + S3 * (q - 1), S3 * q + 4, S3, i0, j0);
+            const int g = lane >> 2, t = lane & 3;
+            float *rq = sR + q * S3;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int i = i0 + g + 8 * (h >> 1), j = j0 + nt * 8 + 2 * t + (h & 1);
+                    const float sv = sOS[i * WSC + j] + as[nt][h];
+                    const float uv = sOU[i * WSC + j] + au[nt][h];
+                    sW[i * WSC + j] = rq[i * RSC + j] - uv - sv;
+                    rq[i * RSC + j] = sv;
+                }
         }
         // row-side warp: LtA[q,q] row b (columns <= b-2); entry warp: LtA[b][b-1]
         float2 la[S3 / 2];
@@ -180,18 +236,31 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
         }
         if (mine && role == 0 && lane > 0) la_new = LAt[(q * S3 + lane) * lda_g + q * S3 + lane - 1];
         __syncthreads();
-        // W0[p,q] = Wt[p,q] - R[p, 0:q] LtA[q, 0:q]^T - S[p,q] into the slot; R's
-        // (p,q) block (holding the staged Wt) becomes S: the sweep adds the S
-        // terms of the row-side sums through R
-        if (mine) {  // three warps
-            Block3 b;
-            product3(b, role, sR, RSC, sLA, S3 * q + 4, q * S3);
-            finish3(b, role, sW, WSC, sR + q * S3, RSC, pp > 0);
+        if (!kOverlap) {
+            stage_subtile(e + 1 - pp, 0, kThreadsC);  // lands while this phase sweeps
+            asm volatile("cp.async.commit_group;" ::: "memory");
         }
-        __syncthreads();
-        stage_phase(e + 1);  // lands while this phase sweeps
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        if (mine) {
+        if (kOverlap && role == 3) {
+            // ---- older-products warp: the next sub-tile (p, qn) of this CTA
+            const int qn = e + 1 - pp;
+            if (qn >= 0 && qn <= 3) {
+                stage_subtile(qn, 96, 32);
+                asm volatile("cp.async.commit_group;" ::: "memory");
+                if (pp >= 2) gather_d(qn, 0, pp - 1, 96, 32);  // D[p', qn], p' <= p - 2
+                asm volatile("cp.async.wait_all;" ::: "memory");
+                __syncwarp();
+                // O_S = LtB[p, 0:p-1] D[0:p-1, qn], O_U = R[p, 0:qn-1] LtA[qn, 0:qn-1]^T
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float os[4][4] = {}, ou[4][4] = {};
+                    if (pp >= 2) mma_block<4>(os, sLBs, S3 * pp + 4, sDr, LSC, S3 * (pp - 1), 16 * hh, 0);
+                    if (qn >= 2) mma_block<4>(ou, sR, RSC, sLA, S3 * qn + 4, S3 * (qn - 1), 16 * hh, 0);
+                    store_block<4>(os, sOS, WSC, 16 * hh, 0);
+                    store_block<4>(ou, sOU, WSC, 16 * hh, 0);
+                }
+            }
+        }
+        if (mine && role < 3) {
             float *ps_buf = sPS, *pu_buf = sPU;
             if (role == 0) {
                 // ---- entry warp (lane = column b): rounds entry (d - b, b) at step d
@@ -238,7 +307,7 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
                         sW[iW] = wt;  // pre-rounding value, copied out when requested
                         d_prev = dl;
                         w0 = w0n; lb_new = lbn_n; sc_s = sn; sc_r = rn; s_ab = s_n;
-                        group_sync(1, kThreadsC);
+                        group_sync(1, kSweepThreads);
                     }
                 };
                 if (exact_div)
@@ -270,7 +339,7 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
                         u3 = ffma2(make_float2(rv[c + 1].z, rv[c + 1].w), la[2 * c + 3], u3);
                     }
                     pu_buf[((d + 1) & 1) * S3 + b] = ((u0.x + u1.x) + (u2.x + u3.x)) + ((u0.y + u1.y) + (u2.y + u3.y));
-                    group_sync(1, kThreadsC);
+                    group_sync(1, kSweepThreads);
                 }
             } else {
                 // ---- column-side warp (lane = row rho): sum_{r <= rho-2} LtB[rho][r] D[r][b]
@@ -300,7 +369,7 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
                     }
                     if (b == bc)
                         ps_buf[((d + 1) & 1) * S3 + b] = ((s0.x + s1.x) + (s2.x + s3.x)) + ((s0.y + s1.y) + (s2.y + s3.y));
-                    group_sync(1, kThreadsC);
+                    group_sync(1, kSweepThreads);
                 }
             }
         }
@@ -331,13 +400,18 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
 
 cudaError_t leaf_cluster_configure()
 {
-    return cudaFuncSetAttribute(leaf_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(leaf_cluster_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemCLaunch);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(leaf_cluster_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kSmemCLaunch);
 }
 
-cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, cudaStream_t stream)
+cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, bool overlap, cudaStream_t stream)
 {
-    return launch_pdl(leaf_cluster_kernel, dim3(4 * tiles), dim3(kThreadsC), kSmemCLaunch, stream, p, K, I_lo);
+    if (overlap)
+        return launch_pdl(leaf_cluster_kernel<true>, dim3(4 * tiles), dim3(128), kSmemCLaunch, stream, p, K, I_lo);
+    return launch_pdl(leaf_cluster_kernel<false>, dim3(4 * tiles), dim3(96), kSmemCLaunch, stream, p, K, I_lo);
 }
 
 }  // namespace bakron
