@@ -32,14 +32,15 @@ TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 : BF16 tensor peak ratio
 FALLBACK_BF16_TFLOPS = 1590.0
 LEAF_BYTES_PER_WEIGHT = 25  # read Wt 4 + diagonal factor blocks 8; write code 1, V 4, D hi/lo 8
 LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 255), 3: ("leaf_warp_kernel", 7 * 63),
-                4: ("leaf_wide_kernel", 3 * 127), 5: ("leaf_cluster_kernel<false>", 7 * 63),
-                6: ("leaf_cluster_kernel<true>", 7 * 63)}
-# DRAM traffic of the band products from an ncu capture of one solve's 124
-# band launches (profiles/band_tc_4096_dram.md); reported only while the
+                4: ("leaf_wide_kernel", 3 * 127), 5: ("leaf_cluster_kernel<false, false>", 7 * 63),
+                6: ("leaf_cluster_kernel<true, false>", 7 * 63), 7: ("leaf_cluster_kernel<true, true>", 7 * 63)}
+# DRAM traffic of the band products from an ncu capture of one solve's 93
+# band launches (profiles/band_4096_dram.md); reported only while the band
 # kernel sources hash to the value the capture was taken with.
-BAND_TRAFFIC = {"sources_sha256": "840ed70f1274291316ac149120e418a50121b7b42f4630228ab356ba719bd5f3",
-                "bytes_per_launch": 27451538.6, "profile": "profiles/band_tc_4096_dram.md"}
-BAND_SOURCES = ("two_sided_gptq_b200/csrc/band_tc.cu", "two_sided_gptq_b200/csrc/common.cuh",
+BAND_TRAFFIC = {"sources_sha256": "bc8092fab082e3f7ffb530ebb380485e36c365dbbbf01ecb766ddcc6db7e5967",
+                "bytes_per_launch": 35.27e6, "profile": "profiles/band_4096_dram.md"}
+BAND_SOURCES = ("two_sided_gptq_b200/csrc/band_tc.cu", "two_sided_gptq_b200/csrc/band_fused.cu",
+                "two_sided_gptq_b200/csrc/tcgen05.cuh", "two_sided_gptq_b200/csrc/common.cuh",
                 "two_sided_gptq_b200/csrc/kernels.cuh")
 
 
@@ -293,12 +294,13 @@ L2_BYTES = 126e6
 
 def working_set_bytes(m, n, T=128):
     """Inputs (W, LA, LB), outputs (V, codes, steps) and the solve workspace
-    (Wt, Delta hi/lo, X^T hi/lo on the padded grid; both normalised factors with
-    their hi/lo parts) touched by one solve."""
+    (Wt, Delta hi/lo, X^T hi/lo and the exported in-tile R on the padded grid;
+    both normalised factors with their hi/lo parts; per-tile flags) touched by
+    one solve."""
     Mp, Np = -(-m // T) * T, -(-n // T) * T
     inputs = 4 * (m * n + n * n + m * m)
     outputs = 4 * m * n + m * n + 4 * m
-    workspace = 4 * (5 * Mp * Np + 3 * Np * Np + 3 * Mp * Mp)
+    workspace = 4 * (6 * Mp * Np + 3 * Np * Np + 3 * Mp * Mp) + 4 * ((Mp // T) * (Np // T) + (Mp + Np) // T)
     return inputs, outputs, workspace
 
 
@@ -492,7 +494,7 @@ def main():
         launches.append(bk.last_profile_launches())
     pr = {k: statistics.median(p[k] for p in prof) for k in prof[0]}
     levels = band_levels(launches)
-    plan = bk.plan_stats(m, n)
+    plan = bk.plan_stats(m, n, leaf=leaf)
     bf16, hbm, src = peaks()
     tf32_peak = bf16 * TF32_PER_BF16
     gemm_ms = pr["stage1_ms"] + pr["stage2_ms"] + pr["fused_ms"]
@@ -538,8 +540,8 @@ def main():
                      "launches_per_step": pr["leaf_launches"],
                      "achieved_gbs": leaf_bytes / (pr["leaf_ms"] / 1e3) / 1e9, "hbm_peak_gbs": hbm,
                      "bytes_per_step": leaf_bytes, "bound": "latency (dependent rounding steps)",
-                     "sequential_steps_per_leaf": LEAF_KERNELS[leaf][1],
-                     "ns_per_sequential_step": pr["leaf_ms"] * 1e6 / (pr["leaf_launches"] * LEAF_KERNELS[leaf][1]),
+                     "sequential_steps_per_tile_diagonal": LEAF_KERNELS[leaf][1],
+                     "ns_per_sequential_step": pr["leaf_ms"] * 1e6 / (plan["tile_diagonals"] * LEAF_KERNELS[leaf][1]),
                      "share_of_profiled_step": pr["leaf_ms"] / pr["total_ms"]},
             "profile_ms": pr,
             "factor_ms": factor_ms,

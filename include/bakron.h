@@ -86,7 +86,7 @@ typedef struct {
 } bakron_quantizer_t;
 
 /* Solver configuration (NULL = defaults; zero fields take defaults).
- * The environment can change the defaults of five fields: BAKRON_LEAF (0..6),
+ * The environment can change the defaults of five fields: BAKRON_LEAF (0..7),
  * BAKRON_GEMM (0..1), BAKRON_TIMEOUT_MS (1..600000), BAKRON_GRAPH (0..1,
  * ignored when profile = 1) and BAKRON_FUSE (1..65535, the default
  * fuse_width); a non-zero field set by the caller wins.  A
@@ -124,8 +124,12 @@ typedef struct {
                          3 with each tile on a cluster of four CTAs, one per
                          row block of sub-tiles; 6 = as 5 with a fourth warp
                          per CTA forming the older product terms of the next
-                         sub-tile during each sweep (bakron_tune_leaf picks
-                         one by measurement). */
+                         sub-tile during each sweep; 7 = as 6 with the two
+                         tile diagonals of every width-2 range of the
+                         recursion in one launch: the second diagonal's tiles
+                         wait (bounded, device flags) for their neighbours on
+                         the first and apply that node's updates themselves
+                         (bakron_tune_leaf picks one by measurement). */
     int32_t b_identity; /* 1: B = I (one-sided GPTQ with Hessian A, the case the
                            two-sided solve reduces to when B = I).  LB_dev may be
                            NULL and is not read; rows are independent, so the
@@ -141,6 +145,12 @@ typedef struct {
                            two launches.  0 = default (2), 1 = never fuse,
                            2..65535 = that width.  Ignored with gemm = 1 and on
                            the one-sided path. */
+    int32_t self_test_omit; /* self-test of the bounded waits of leaf structure
+                               7 only; 0 = off.  v > 0: the first-diagonal tile
+                               with row-major tile index v - 1 never raises its
+                               flag, so its neighbours' waits run out after
+                               timeout_ms and record BAKRON_ERR_DEVICE_TIMEOUT
+                               (the results are then not the solve's). */
 } bakron_config_t;
 
 /* Per-kernel-class device time of the latest profiled bakron_solve on the
@@ -233,7 +243,7 @@ bakron_status_t bakron_solve(const float *W_dev, int64_t m, int64_t n, const flo
  * bakron_solve on the caller's problem once per structure after one warm-up
  * solve, timing each with CUDA events on `stream` (the call synchronises
  * `stream`), and writes the fastest structure (a bakron_config_t.leaf value,
- * 1..6) to *leaf_out and the six times in ms to ms_out[0..5] (leaf 1..6;
+ * 1..7) to *leaf_out and the seven times in ms to ms_out[0..6] (leaf 1..7;
  * ms_out may be NULL).  Arguments as for bakron_solve; cfg->leaf is ignored
  * and cfg->profile must be 0.  V, codes and scales hold the last solve's
  * results (all structures give the same codes up to rounding ties).  Device
@@ -391,6 +401,9 @@ typedef struct {
                                 all band products: a product with the factor
                                 tile on the diagonal (lower triangular) counts
                                 T^2 (T+1)/2 of them instead of T^3 */
+    double leaf_update_flops; /* leaf structure 7: FLOPs of the width-2 nodes'
+                                 updates formed inside the leaf launches (2 T^3
+                                 per neighbour product); 0 otherwise */
 } bakron_plan_stats_t;
 bakron_status_t bakron_plan_stats(int64_t m, int64_t n, const bakron_config_t *cfg,
                                   bakron_plan_stats_t *out);

@@ -181,6 +181,39 @@ def test_plan_stats_matches_bruteforce_count(lib, shape):
     assert s.structural_flops == pytest.approx(fs, rel=0, abs=0)
 
 
+@pytest.mark.parametrize("shape", [(3, 3), (5, 8), (9, 4), (32, 32)])
+def test_plan_stats_two_diagonal_leaves(lib, shape):
+    """Leaf structure 7: the width-2 ranges of the recursion become single
+    launches whose updates move into the leaf (two T^3 products per
+    neighbour); every other node is counted as before."""
+    from two_sided_gptq_b200 import _native
+
+    Mt, Nt = shape
+    T = 128
+    base, pair = _native.PlanStats(), _native.PlanStats()
+    cfg = _native.Config(0, 0, 0, 0, None, 0, 7)
+    assert lib.bakron_plan_stats(Mt * T, Nt * T, None, ctypes.byref(base)) == 0
+    assert lib.bakron_plan_stats(Mt * T, Nt * T, ctypes.byref(cfg), ctypes.byref(pair)) == 0
+
+    def width2_ranges(k, l, out):
+        if l <= 1:
+            return
+        if l == 2:
+            out.append(k)
+            return
+        h = l // 2
+        width2_ranges(k, h, out)
+        width2_ranges(k + h, l - h, out)
+
+    ks = []
+    width2_ranges(0, Mt + Nt - 1, ks)
+    assert pair.nodes == base.nodes - len(ks)
+    assert pair.leaves == base.leaves - len(ks)
+    neighbours = sum((J >= 1) + (I >= 1) for k in ks for I in range(Mt) for J in [k + 1 - I] if 0 <= J < Nt)
+    assert pair.leaf_update_flops == 2.0 * T ** 3 * neighbours
+    assert pair.update_flops < base.update_flops
+
+
 def test_plan_stats_4096_cubic_work(lib):
     """O(mn(m+n)) work: the update FLOPs at 4096^2 lie between the
     mn(m+n) pull-form count and twice it, and grow ~8x per size doubling
@@ -257,9 +290,9 @@ def test_environment_overrides_are_validated():
     from two_sided_gptq_b200 import _native
 
     ok, bad = _native.Status.OK, _native.Status.ERR_INVALID_ARG
-    assert _plan_status_under_env({"BAKRON_LEAF": "6", "BAKRON_GEMM": "1", "BAKRON_TIMEOUT_MS": "50",
+    assert _plan_status_under_env({"BAKRON_LEAF": "7", "BAKRON_GEMM": "1", "BAKRON_TIMEOUT_MS": "50",
                                    "BAKRON_GRAPH": "1", "BAKRON_FUSE": "8"}) == ok
-    for env in ({"BAKRON_LEAF": "7"}, {"BAKRON_GEMM": "2"}, {"BAKRON_TIMEOUT_MS": "0"},
+    for env in ({"BAKRON_LEAF": "8"}, {"BAKRON_GEMM": "2"}, {"BAKRON_TIMEOUT_MS": "0"},
                 {"BAKRON_TIMEOUT_MS": "12ms"}, {"BAKRON_GRAPH": "-1"}, {"BAKRON_FUSE": "0"},
                 {"BAKRON_FUSE": "65536"}):
         assert _plan_status_under_env(env) == bad, env

@@ -25,7 +25,7 @@ __all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_pr
 
 
 # bakron_config_t.leaf values bakron_tune_leaf times (one ms_out entry each)
-LEAF_STRUCTURES = (1, 2, 3, 4, 5, 6)
+LEAF_STRUCTURES = (1, 2, 3, 4, 5, 6, 7)
 
 
 def _lib():
@@ -64,9 +64,10 @@ def _dev_f32(x, name):
     return x
 
 
-def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False, leaf=0, b_identity=False, graph=False, fuse_width=0):
+def _config(gemm=0, timeout_ms=0, wt_out=None, profile=False, leaf=0, b_identity=False, graph=False, fuse_width=0,
+            self_test_omit=0):
     return Config(0, int(gemm), 1 if graph else 0, int(timeout_ms), _ptr(wt_out), 1 if profile else 0, int(leaf),
-                  1 if b_identity else 0, int(fuse_width))
+                  1 if b_identity else 0, int(fuse_width), int(self_test_omit))
 
 
 def workspace(nbytes: int, device=None):
@@ -130,7 +131,7 @@ def solve_workspace_size(m: int, n: int, gemm: int = 0) -> int:
 
 def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None, out=None, stream=None,
           wt_out=None, check_status=True, timeout_ms=0, profile=False, leaf=0, shrink_grid=0, graph=False,
-          fuse_width=0):
+          fuse_width=0, self_test_omit=0):
     """BaKron solve on device tensors.  Returns ``(V, codes, scales)``.
 
     ``LB=None`` selects the one-sided path (B = I: GPTQ with Hessian A, over
@@ -143,7 +144,9 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     1 two-level CTA-wide, 2 single-level, 3 three warps per 32 x 32
     sub-tile, 4 six warps per 64 x 64 sub-tile, 5 as 3 with each tile on a
     cluster of four CTAs, 6 as 5 with the older product terms formed during
-    the sweeps; :func:`tune_leaf` picks one by measurement).  ``fuse_width`` (0 default, 1 never) runs the two band
+    the sweeps, 7 as 6 with two tile diagonals per launch (device flags, the
+    width-2 nodes' updates inside the leaf); :func:`tune_leaf` picks one by
+    measurement).  ``self_test_omit`` is a self-test hook of structure 7.  ``fuse_width`` (0 default, 1 never) runs the two band
     products of recursion nodes at most that many tile diagonals wide as one
     launch per target tile.  ``graph=True`` captures the solve's launches for this
     argument set into a CUDA graph on the first call and replays it on later
@@ -160,7 +163,7 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     m, n = W.shape
     if LA.shape != (n, n) or (not one_sided and LB.shape != (m, m)):
         raise ValueError("LA must be n x n and LB m x m")
-    cfg = _config(gemm, timeout_ms, wt_out, profile, leaf, one_sided, graph, fuse_width)
+    cfg = _config(gemm, timeout_ms, wt_out, profile, leaf, one_sided, graph, fuse_width, self_test_omit)
     if out is None:
         V = torch.empty((m, n), dtype=torch.float32, device=W.device)
         codes = torch.empty((m, n), dtype=torch.int8, device=W.device)
@@ -226,7 +229,7 @@ def tune_cache_put(path: str, key: str, leaf: int, ms) -> None:
 def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, timeout_ms=0, cache=None):
     """Leaf structure chosen by measurement (``bakron_tune_leaf``): one timed
     solve per structure on this problem.  Returns ``(leaf, [ms_leaf1, ...,
-    ms_leaf6])``; pass ``leaf`` to :func:`solve`.
+    ms_leaf7])``; pass ``leaf`` to :func:`solve`.
 
     ``cache`` (or the ``BAKRON_TUNE_CACHE`` environment variable) names a JSON
     file keyed by (m, n, bits, GPU name): a stored measurement is returned
@@ -388,10 +391,11 @@ def last_profile_launches() -> list:
              "structural_flops": r.structural_flops} for r in buf[:n]]
 
 
-def plan_stats(m: int, n: int, one_sided: bool = False) -> dict:
+def plan_stats(m: int, n: int, one_sided: bool = False, leaf: int = 0) -> dict:
     """Schedule statistics of an m x n solve (host only); ``one_sided`` for
-    the B = I schedule over column blocks."""
+    the B = I schedule over column blocks; ``leaf`` the leaf structure (7
+    moves the width-2 nodes' products into the leaf launches)."""
     s = PlanStats()
-    cfg = _config(b_identity=int(one_sided))
+    cfg = _config(b_identity=int(one_sided), leaf=leaf)
     check(_lib().bakron_plan_stats(m, n, ctypes.byref(cfg), ctypes.byref(s)), "bakron_plan_stats")
     return {f: getattr(s, f) for f, _ in PlanStats._fields_}

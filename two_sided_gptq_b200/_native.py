@@ -45,7 +45,8 @@ class BatchItem(ctypes.Structure):
 class Config(ctypes.Structure):
     _fields_ = [("tile", ctypes.c_int32), ("gemm", ctypes.c_int32), ("use_graph", ctypes.c_int32),
                 ("timeout_ms", ctypes.c_int32), ("wt_out", ctypes.c_void_p), ("profile", ctypes.c_int32),
-                ("leaf", ctypes.c_int32), ("b_identity", ctypes.c_int32), ("fuse_width", ctypes.c_int32)]
+                ("leaf", ctypes.c_int32), ("b_identity", ctypes.c_int32), ("fuse_width", ctypes.c_int32),
+                ("self_test_omit", ctypes.c_int32)]
 
 
 class Profile(ctypes.Structure):
@@ -60,7 +61,7 @@ class PlanStats(ctypes.Structure):
     _fields_ = [("tiles_m", ctypes.c_int64), ("tiles_n", ctypes.c_int64), ("tile_diagonals", ctypes.c_int64),
                 ("nodes", ctypes.c_int64), ("leaves", ctypes.c_int64), ("update_flops", ctypes.c_double),
                 ("stage1_flops", ctypes.c_double), ("stage2_flops", ctypes.c_double),
-                ("structural_flops", ctypes.c_double)]
+                ("structural_flops", ctypes.c_double), ("leaf_update_flops", ctypes.c_double)]
 
 
 # name -> (restype, argtypes); every function declared in include/bakron.h

@@ -30,8 +30,11 @@ constexpr const char *kVersion = "bakron-b200 0.2";
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Leaf structures bakron_tune_leaf times (bakron_config_t.leaf 1..6).
-constexpr int kLeafStructures = 6;
+// Leaf structures bakron_tune_leaf times (bakron_config_t.leaf 1..7).
+constexpr int kLeafStructures = 7;
+// 0-based leaf variant of structure 7: width-2 ranges of the recursion run as
+// one launch of two tile diagonals (structure 6's kernel for single ones).
+constexpr int kPairVariant = 6;
 
 // Nodes at most this many tile diagonals wide run fused by default (measured
 // on B200 at 4096^2: width 2 trims the profiled band time, wider fusing is
@@ -43,6 +46,7 @@ struct Config {
     // formed during the sweeps), the fastest measured
     int tile = kTile, gemm = 0, use_graph = 0, timeout_ms = 200, profile = 0, leaf = 5, b_identity = 0;
     int fuse_width = kDefaultFuseWidth;
+    int self_test_omit = 0;
     float *wt_out = nullptr;
 };
 
@@ -160,6 +164,8 @@ bakron_status_t read_config(const bakron_config_t *c, Config &out)
     out.b_identity = c->b_identity;
     if (c->fuse_width < 0 || c->fuse_width > 65535) return BAKRON_ERR_INVALID_ARG;
     if (c->fuse_width != 0) out.fuse_width = c->fuse_width;
+    if (c->self_test_omit < 0) return BAKRON_ERR_INVALID_ARG;
+    out.self_test_omit = c->self_test_omit;
     if (out.use_graph && out.profile) return BAKRON_ERR_INVALID_ARG;  // per-launch events cannot be replayed
     return BAKRON_OK;
 }
@@ -208,6 +214,7 @@ struct SolveCtx {
     GemmArgs s1, s2;
     TcMaps m1, m2;
     int gemm, leaf_variant, fuse_width;
+    int pair_slot;  // next ticket counter of a two-diagonal leaf launch
     cudaStream_t stream;
 };
 
@@ -221,11 +228,20 @@ cudaError_t run_band(const SolveCtx &c, int stage, const NodeParams &np)
     return e;
 }
 
-cudaError_t run_schedule(const SolveCtx &c, int k, int l)
+cudaError_t run_schedule(SolveCtx &c, int k, int l)
 {
     if (l <= 1) {
         t_prof.begin(1, NodeParams{k, 0, 1, c.leaf.Mt, c.leaf.Nt});
-        cudaError_t e = launch_leaf(c.leaf, k, c.leaf_variant, c.stream);
+        cudaError_t e = launch_leaf(c.leaf, k, c.leaf_variant == kPairVariant ? kPairVariant - 1 : c.leaf_variant,
+                                    c.stream);
+        t_prof.end();
+        return e;
+    }
+    if (l == 2 && c.leaf_variant == kPairVariant) {
+        // both tile diagonals in one launch; the second one's tiles apply the
+        // width-2 node's updates themselves
+        t_prof.begin(1, NodeParams{k, 1, 2, c.leaf.Mt, c.leaf.Nt});
+        cudaError_t e = launch_leaf_pair(c.leaf, k, c.pair_slot++, c.stream);
         t_prof.end();
         return e;
     }
@@ -368,7 +384,8 @@ bakron_status_t solve_device(const float *W, int64_t m, int64_t n, const float *
         for (int i = 0; i < 9; ++i) key.p[i] = ptrs[i];
         key.m = m; key.n = n; key.ws_bytes = ws_bytes;
         key.v[0] = qmin; key.v[1] = qmax; key.v[2] = q->row_scale ? 0 : q->shrink_grid; key.v[3] = conf.gemm;
-        key.v[4] = conf.leaf | (conf.fuse_width << 8); key.v[5] = conf.timeout_ms; key.v[6] = conf.b_identity;
+        key.v[4] = conf.leaf | (conf.fuse_width << 8); key.v[5] = conf.timeout_ms;
+        key.v[6] = conf.b_identity | (conf.self_test_omit << 1);
         if (cudaGetDevice(&key.v[7]) != cudaSuccess) return BAKRON_ERR_CUDA;
         return launch_graph(key, stream, [&](cudaStream_t cap) {
             return enqueue_solve(W, m, n, LA, LB, q, qmin, qmax, V, codes, scales, L, (char *)ws, conf, cap);
@@ -401,6 +418,7 @@ bakron_status_t enqueue_solve(const float *W, int64_t m, int64_t n, const float 
     c.gemm = conf.gemm;
     c.leaf_variant = conf.leaf;
     c.fuse_width = conf.fuse_width;
+    c.pair_slot = 0;
     c.stream = stream;
     c.leaf.LA32 = (const float *)(w + L.LA32);
     c.leaf.LB32 = (const float *)(w + L.LB32);
@@ -415,6 +433,14 @@ bakron_status_t enqueue_solve(const float *W, int64_t m, int64_t n, const float 
     c.leaf.qmin = qmin; c.leaf.qmax = qmax;
     c.leaf.st = st;
     c.leaf.wt_out = conf.wt_out;
+    c.leaf.Rx = (float *)(w + L.Rx);
+    c.leaf.flags = (int32_t *)(w + L.sync);
+    c.leaf.tickets = c.leaf.flags + L.Mt * L.Nt;
+    c.leaf.timeout_ms = conf.timeout_ms;
+    c.leaf.omit_flag = conf.self_test_omit;
+    if (!conf.b_identity && conf.leaf == kPairVariant &&
+        cudaMemsetAsync(w + L.sync, 0, L.sync_bytes, stream) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
     // stage 1: X^T (Np x Mp) = LtA (Np x Np) . Delta (Mp x Np)^T over tile columns
     c.s1 = GemmArgs{(const float *)(w + L.LAhi), (const float *)(w + L.LAlo),
                     (const float *)(w + L.Dhi), (const float *)(w + L.Dlo), L.Np, L.Np,
@@ -490,20 +516,31 @@ bakron_status_t bakron::solve_direct(const float *W, int64_t m, int64_t n, const
 
 namespace {
 
-void count_schedule(int k, int l, int Mt, int Nt, bakron_plan_stats_t *o)
+void count_schedule(int k, int l, int Mt, int Nt, bakron_plan_stats_t *o, bool pairs)
 {
     if (l <= 1) {
         o->leaves++;
         return;
     }
+    if (l == 2 && pairs) {
+        // one launch; each second-diagonal tile forms two T^3 products per
+        // neighbour it has on the first diagonal
+        o->leaves++;
+        const double t3 = 2.0 * kTile * (double)kTile * kTile;
+        for (int I = max(0, k + 1 - (Nt - 1)); I <= min(Mt - 1, k + 1); ++I) {
+            const int J = k + 1 - I;
+            o->leaf_update_flops += t3 * ((J >= 1 ? 1 : 0) + (I >= 1 ? 1 : 0));
+        }
+        return;
+    }
     const int h = l / 2;
-    count_schedule(k, h, Mt, Nt, o);
+    count_schedule(k, h, Mt, Nt, o, pairs);
     NodeParams np{k, h, l, Mt, Nt};
     o->stage1_flops += node_stage_flops(np, 1);
     o->stage2_flops += node_stage_flops(np, 2);
     o->structural_flops += node_stage_flops(np, 1, true) + node_stage_flops(np, 2, true);
     o->nodes++;
-    count_schedule(k + h, l - h, Mt, Nt, o);
+    count_schedule(k + h, l - h, Mt, Nt, o, pairs);
 }
 
 // One-sided path: the recursion over column blocks; every update counts as
@@ -885,7 +922,8 @@ bakron_status_t bakron_plan_stats(int64_t m, int64_t n, const bakron_config_t *c
     if (conf.b_identity)
         count_schedule_gptq(0, (int)out->tiles_n, (int)out->tiles_m, (int)out->tiles_n, out);
     else
-        count_schedule(0, (int)out->tile_diagonals, (int)out->tiles_m, (int)out->tiles_n, out);
+        count_schedule(0, (int)out->tile_diagonals, (int)out->tiles_m, (int)out->tiles_n, out,
+                       conf.leaf == kPairVariant);
     out->update_flops = out->stage1_flops + out->stage2_flops;
     return BAKRON_OK;
 }

@@ -98,7 +98,7 @@ __device__ __forceinline__ float div_rn_recip(float a, float b, float rb)
 // Layout of the solve workspace (all offsets multiples of kAlign).
 struct SolveLayout {
     int64_t m, n, T, Mt, Nt, Mp, Np;
-    size_t status, Wt, Dhi, Dlo, XThi, XTlo, LA32, LAhi, LAlo, LB32, LBhi, LBlo, total;
+    size_t status, Wt, Dhi, Dlo, XThi, XTlo, LA32, LAhi, LAlo, LB32, LBhi, LBlo, Rx, sync, sync_bytes, total;
 
     void compute(int64_t m_, int64_t n_, int64_t T_)
     {
@@ -113,6 +113,11 @@ struct SolveLayout {
         const size_t nn = (size_t)Np * Np * sizeof(float), mm = (size_t)Mp * Mp * sizeof(float);
         LA32 = take(nn); LAhi = take(nn); LAlo = take(nn);
         LB32 = take(mm); LBhi = take(mm); LBlo = take(mm);
+        // leaf structure 7: exported in-tile R, per-tile flags and per-launch
+        // tickets (zeroed by each solve)
+        Rx = take(mn);
+        sync_bytes = (size_t)(Mt * Nt + Mt + Nt) * sizeof(int32_t);
+        sync = take(sync_bytes);
         total = o;
     }
 };

@@ -15,6 +15,12 @@ struct LeafArgs {
     int Mt, Nt, qmin, qmax;
     DeviceStatus *st;
     float *wt_out;  // optional m x n pre-rounding values
+    // two tile diagonals per launch (leaf structure 7)
+    float *Rx;          // Mp x Np: each first-diagonal tile's in-tile R (read by its right neighbour)
+    int32_t *flags;     // Mt x Nt: CTAs of a first-diagonal tile that have published their outputs
+    int32_t *tickets;   // one counter per launch: clusters in the order they started
+    int timeout_ms;     // limit of the bounded waits on flags
+    int omit_flag;      // self-test only: first-diagonal tile (linear index + 1) that never publishes
 };
 
 // Operands of the band products.  Stage 1: A = LtA (Np x Np), B = Delta
@@ -41,6 +47,9 @@ cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stre
 // a fourth warp forms the older product terms during the sweeps.
 cudaError_t leaf_cluster_configure();
 cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, bool overlap, cudaStream_t stream);
+// Tile diagonals K and K+1 in one launch (leaf structure 7): ticket counter
+// `slot`; the second diagonal's clusters wait for their neighbours' flags.
+cudaError_t launch_leaf_pair(const LeafArgs &p, int K, int slot, cudaStream_t stream);
 
 // FP32 CUDA-core band products (reference kernels for the tensor-core path).
 cudaError_t launch_band_simt(int stage, const NodeParams &np, const GemmArgs &g, cudaStream_t stream);

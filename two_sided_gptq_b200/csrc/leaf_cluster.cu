@@ -29,6 +29,24 @@
 // sub-tile's Wt block and LtA strip and fetches the older D blocks from the
 // other CTAs), so between two sweeps only the newest terms remain, shared by
 // all four warps.
+//
+// Two tile diagonals per launch (kPair, structure 7): clusters take tickets
+// from a counter in the order they start; the first tickets take the tiles of
+// diagonal K, the rest those of K + 1, so a cluster only ever waits for
+// clusters that are already running.  A diagonal-K tile runs as above, then
+// exports its in-tile R (rows of its CTAs) and raises its flag (one increment
+// per CTA, after a device-scope fence).  A diagonal-(K+1) tile (I', J') waits,
+// bounded by a %globaltimer deadline, for the flags of its neighbours on K --
+// left (I', J'-1) and upper (I'-1, J') -- and then applies their share of
+// Proposition 3.1's updates itself, which for a width-2 node takes two plain
+// products instead of two chained ones:
+//     left:  sum_{r<=a, c} LtB[a,r] D_rc LtA[b,c] = (R_left LtA[J',J'-1]^T)[a,b],
+//            R_left the left tile's in-tile R, subtracted from Wt;
+//     upper: sum_{r, c<=b} LtB[a,r] D_rc LtA[b,c] = sum_{c<=b} S_up[a,c] LtA[b,c],
+//            S_up = LtB[I',I'-1] D_up, which enters the sweep's pull form
+//            exactly like the in-tile S (added into S before each sub-tile).
+// Both products run in FP32 on the CUDA cores of the tile's four CTAs (each
+// its own 32 rows) before the first phase.
 #include <cooperative_groups.h>
 
 #include <type_traits>
@@ -58,11 +76,33 @@ constexpr size_t kSmemC = ((size_t)(S3 + 1) * RSC + (size_t)(T + 1) * DSC + (siz
 // variant is one sub-tile sweep per SM.
 constexpr size_t kSmemCLaunch = 120 * 1024;
 static_assert(kSmemC <= kSmemCLaunch && 2 * kSmemCLaunch > 228 * 1024, "cluster leaf shared memory");
+// pair form: S_up rows (S3 x SUPS) and one staging chunk of the neighbour
+// products (R_left 32 x 32, LtA 128 x 32, LtB 32 x 32, D_up 32 x 128)
+constexpr int SUPS = T + 4;
+constexpr int CKS = 36;  // row stride of the staged 32-wide chunks
+constexpr size_t kSmemPairExtra = ((size_t)S3 * SUPS + 2 * S3 * CKS + (size_t)T * CKS + (size_t)S3 * T) * sizeof(float);
+constexpr size_t kSmemPairLaunch = align_up(kSmemC, 16) + kSmemPairExtra;
+static_assert(kSmemPairLaunch <= 232448, "pair leaf shared memory");
+
+// Bounded wait for a device-scope counter to reach `target`; false if the
+// deadline passed first.
+__device__ __forceinline__ bool wait_counter(const int32_t *ctr, int target, uint64_t deadline)
+{
+    for (;;) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= target) return true;
+        uint64_t t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t > deadline) return false;
+        __nanosleep(64);
+    }
+}
 }  // namespace
 
-template <bool kOverlap>
+template <bool kOverlap, bool kPair>
 __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kOverlap ? 128 : 96, 1)
-leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
+leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
 {
     constexpr int kThreadsC = kOverlap ? 128 : 96;
     cg::cluster_group cluster = cg::this_cluster();
@@ -83,13 +123,34 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
     float *sPS = rcp + S3;                    // 2 x S3: column-side partial sums by column
     float *sPU = sPS + 2 * S3;                // 2 x S3: row-side partial sums by column
     int8_t *sCode = (int8_t *)(sPU + 2 * S3); // S3 x T codes (+32 spare bytes)
+    // pair form: S_up rows of this row block, then the staging chunk
+    float *sSup = (float *)((uint8_t *)smem_f + align_up(kSmemC, 16));  // S3 x SUPS
+    float *cR = sSup + S3 * SUPS;             // S3 x CKS: R_left rows, 32-wide chunk
+    float *cB = cR + S3 * CKS;                // S3 x CKS: LtB[I', I'-1] rows, chunk
+    float *cA = cB + S3 * CKS;                // T x CKS: LtA[J', J'-1] rows, chunk
+    float *cD = cA + T * CKS;                 // S3 x T: D_up rows of the chunk
 
-    const int I = I_lo + (int)(blockIdx.x / 4), J = K - I;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // the cluster's tile: by launch position, or (pair form) by ticket
+    int Kd = K, I = I_lo + (int)(blockIdx.x / 4);
+    bool consumer = false;  // pair form: a tile of the second diagonal
+    if (kPair) {
+        __shared__ int ticket_sh;
+        pdl_wait();  // the ticket counter was cleared before this solve's first kernel
+        if (pp == 0 && tid == 0) ticket_sh = atomicAdd(&p.tickets[slot], 1);
+        cluster.sync();
+        const int tk = *cluster.map_shared_rank(&ticket_sh, 0);
+        const int lo0 = max(0, K - (p.Nt - 1)), n0 = min(p.Mt - 1, K) - lo0 + 1;
+        const int lo1 = max(0, K + 1 - (p.Nt - 1));
+        consumer = tk >= n0;
+        Kd = consumer ? K + 1 : K;
+        I = consumer ? lo1 + (tk - n0) : lo0 + tk;
+    }
+    const int J = Kd - I;
     const int64_t row0 = (int64_t)I * T, col0 = (int64_t)J * T;
     const int64_t brow0 = row0 + pp * S3;  // first row of this row block
     const int mr = (int)min64(T, p.m - row0), nc = (int)min64(T, p.n - col0);
     const int mrb = max(0, min(S3, mr - pp * S3));  // rows of this row block inside the matrix
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const float *LAt = p.LA32 + col0 * p.Np + col0;  // LtA diagonal block of the tile (global)
     const float *LBt = p.LB32 + row0 * p.Mp + row0;  // LtB diagonal block of the tile (global)
     const int lda_g = (int)p.Np, ldb_g = (int)p.Mp;
@@ -108,6 +169,97 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
         ((float4 *)sOS)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();  // R is zero before the first staged block lands in it
     pdl_wait();       // every global input (Wt, factors, steps) comes from earlier kernels
+    const bool has_left = kPair && consumer && J >= 1;  // neighbours on the first diagonal
+    const bool has_up = kPair && consumer && I >= 1;
+    if (kPair && consumer) {
+        // wait for the neighbours' outputs (bounded), then their share of the
+        // updates: P = R_left LtA[J',J'-1]^T off Wt, S_up = LtB[I',I'-1] D_up
+        if (tid == 0) {
+            const uint64_t deadline = [] { uint64_t t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t)); return t; }() +
+                                      (uint64_t)p.timeout_ms * 1000000ull;
+            bool ok = true;
+            if (has_left) ok = wait_counter(p.flags + (int64_t)I * p.Nt + (J - 1), 4, deadline);
+            if (ok && has_up) ok = wait_counter(p.flags + (int64_t)(I - 1) * p.Nt + J, 4, deadline);
+            if (!ok) record_error(p.st, BAKRON_ERR_DEVICE_TIMEOUT, 4000 + pp);
+            __threadfence();
+        }
+        __syncthreads();
+        // thread t: column j = t of P and S_up, rows a of this row block in pairs
+        float2 pa[S3 / 2], sa[S3 / 2];
+#pragma unroll
+        for (int i = 0; i < S3 / 2; ++i) pa[i] = sa[i] = make_float2(0.f, 0.f);
+        const int jj = tid;  // 128 threads = 128 columns
+        for (int kc = 0; kc < T / 32; ++kc) {
+            // stage the chunk of 32 contraction indices (L2-coherent loads)
+            const int64_t kx = (int64_t)kc * 32;
+            if (has_left) {
+                for (int c = tid; c < S3 * 8; c += kThreadsC) {
+                    const int r = c >> 3, k4 = c & 7;
+                    *(float4 *)(cR + r * CKS + 4 * k4) =
+                        __ldcg((const float4 *)(p.Rx + (brow0 + r) * p.Np + (col0 - T) + kx + 4 * k4));
+                }
+                for (int c = tid; c < T * 8; c += kThreadsC) {
+                    const int r = c >> 3, k4 = c & 7;
+                    *(float4 *)(cA + r * CKS + 4 * k4) =
+                        *(const float4 *)(p.LA32 + (col0 + r) * p.Np + (col0 - T) + kx + 4 * k4);
+                }
+            }
+            if (has_up) {
+                for (int c = tid; c < S3 * 8; c += kThreadsC) {
+                    const int r = c >> 3, k4 = c & 7;
+                    *(float4 *)(cB + r * CKS + 4 * k4) =
+                        *(const float4 *)(p.LB32 + (brow0 + r) * p.Mp + (row0 - T) + kx + 4 * k4);
+                }
+                for (int r = 0; r < S3; ++r) {
+                    const int64_t g = (row0 - T + kx + r) * p.Np + col0 + jj;
+                    cD[r * T + jj] = __ldcg(p.Dhi + g) + __ldcg(p.Dlo + g);
+                }
+            }
+            __syncthreads();
+#pragma unroll 2
+            for (int k = 0; k < 32; k += 4) {
+                if (has_left) {
+                    const float4 la4 = *(const float4 *)(cA + jj * CKS + k);
+#pragma unroll
+                    for (int i = 0; i < S3 / 2; ++i) {
+                        const float4 r0 = *(const float4 *)(cR + (2 * i) * CKS + k);
+                        const float4 r1 = *(const float4 *)(cR + (2 * i + 1) * CKS + k);
+                        pa[i] = ffma2(make_float2(r0.x, r1.x), make_float2(la4.x, la4.x), pa[i]);
+                        pa[i] = ffma2(make_float2(r0.y, r1.y), make_float2(la4.y, la4.y), pa[i]);
+                        pa[i] = ffma2(make_float2(r0.z, r1.z), make_float2(la4.z, la4.z), pa[i]);
+                        pa[i] = ffma2(make_float2(r0.w, r1.w), make_float2(la4.w, la4.w), pa[i]);
+                    }
+                }
+                if (has_up) {
+                    const float d0 = cD[(k + 0) * T + jj], d1 = cD[(k + 1) * T + jj];
+                    const float d2 = cD[(k + 2) * T + jj], d3 = cD[(k + 3) * T + jj];
+#pragma unroll
+                    for (int i = 0; i < S3 / 2; ++i) {
+                        const float4 b0 = *(const float4 *)(cB + (2 * i) * CKS + k);
+                        const float4 b1 = *(const float4 *)(cB + (2 * i + 1) * CKS + k);
+                        sa[i] = ffma2(make_float2(b0.x, b1.x), make_float2(d0, d0), sa[i]);
+                        sa[i] = ffma2(make_float2(b0.y, b1.y), make_float2(d1, d1), sa[i]);
+                        sa[i] = ffma2(make_float2(b0.z, b1.z), make_float2(d2, d2), sa[i]);
+                        sa[i] = ffma2(make_float2(b0.w, b1.w), make_float2(d3, d3), sa[i]);
+                    }
+                }
+            }
+            __syncthreads();  // the chunk buffers are refilled next
+        }
+        // Wt rows of this row block lose P (no other CTA reads them until this
+        // CTA stages them below); S_up waits in shared memory for the sweeps
+#pragma unroll
+        for (int i = 0; i < S3 / 2; ++i) {
+            if (has_left) {
+                float *w0 = p.Wt + (brow0 + 2 * i) * p.Np + col0 + jj;
+                w0[0] -= pa[i].x;
+                w0[p.Np] -= pa[i].y;
+            }
+            sSup[(2 * i) * SUPS + jj] = sa[i].x;
+            sSup[(2 * i + 1) * SUPS + jj] = sa[i].y;
+        }
+        __syncthreads();
+    }
 
     // Stage the sub-tile (pp, q) -- its Wt block into R's block (untouched
     // until then) and the strip LtA[q, 0:q] -- with threads [t0, t0 + nt).
@@ -169,12 +321,45 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
     }
     const bool exact_div = __syncthreads_or(out_of_range) != 0;
 
+    // row-side warp: LtA[q,q] row b (columns <= b-2); entry warp: LtA[b][b-1].
+    // Loaded for the CTA's next sub-tile as soon as the previous sweep ends, so
+    // the L2 latency overlaps the phase change.
+    float2 la[S3 / 2];
+    float la_new = 0.f;
+    auto load_la = [&](int q) {
+        if (q < 0 || q > 3) return;
+        if (role == 1) {
+#pragma unroll
+            for (int c = 0; c < S3 / 2; ++c) {
+                float2 v = *(const float2 *)(LAt + (q * S3 + lane) * lda_g + q * S3 + 2 * c);
+                v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
+                v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
+                la[c] = v;
+            }
+        }
+        if (role == 0 && lane > 0) la_new = LAt[(q * S3 + lane) * lda_g + q * S3 + lane - 1];
+    };
+    load_la(0 - pp);
+
     for (int e = 0; e < 7; ++e) {
         const int q = e - pp;
         const bool mine = q >= 0 && q <= 3;
         // Every CTA of the cluster has finished phase e - 1, so the D blocks
         // it rounded are final and visible (release / acquire at cluster scope).
-        cluster.sync();
+        // Overlapped form: the barrier is split; between arriving and waiting
+        // the CTA forms the newest row-side term R[p,q-1] LtA[q,q-1]^T, which
+        // needs only its own R (final since the last CTA barrier) and the LtA
+        // strip the product warp staged and waited for.
+        float au[2][4] = {};
+        if (kOverlap) {
+            asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+            if (mine && q > 0)
+                mma_block<2>(au, sR + S3 * (q - 1), RSC, sLA + S3 * (q - 1), S3 * q + 4, S3, 16 * (warp & 1),
+                             16 * (warp >> 1));
+            asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+        } else {
+            cluster.sync();
+        }
         asm volatile("cp.async.wait_all;" ::: "memory");  // this phase's staged Wt block and strip
         if (mine && pp > 0) {
             // D[p', q] of the row blocks above: all of them, or (overlapped
@@ -206,9 +391,8 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
             //   S = O_S + LtB[p,p-1] D[p-1,q],  U = O_U + R[p,q-1] LtA[q,q-1]^T,
             //   W0 = Wt - U - S into the slot, R's (p,q) block := S
             const int i0 = 16 * (warp & 1), j0 = 16 * (warp >> 1);
-            float as[2][4] = {}, au[2][4] = {};
+            float as[2][4] = {};
             if (pp > 0) mma_block<2>(as, sLBs + S3 * (pp - 1), S3 * pp + 4, sDr + S3 * (pp - 1), LSC, S3, i0, j0);
-            if (q > 0) mma_block<2>(au, sR + S3 * (q - 1), RSC, sLA + S3 * (q - 1), S3 * q + 4, S3, i0, j0);
             const int g = lane >> 2, t = lane & 3;
             float *rq = sR + q * S3;
 #pragma unroll
@@ -216,25 +400,13 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const int i = i0 + g + 8 * (h >> 1), j = j0 + nt * 8 + 2 * t + (h & 1);
-                    const float sv = sOS[i * WSC + j] + as[nt][h];
+                    float sv = sOS[i * WSC + j] + as[nt][h];
+                    if (has_up) sv += sSup[i * SUPS + q * S3 + j];
                     const float uv = sOU[i * WSC + j] + au[nt][h];
                     sW[i * WSC + j] = rq[i * RSC + j] - uv - sv;
                     rq[i * RSC + j] = sv;
                 }
         }
-        // row-side warp: LtA[q,q] row b (columns <= b-2); entry warp: LtA[b][b-1]
-        float2 la[S3 / 2];
-        float la_new = 0.f;
-        if (mine && role == 1) {
-#pragma unroll
-            for (int c = 0; c < S3 / 2; ++c) {
-                float2 v = *(const float2 *)(LAt + (q * S3 + lane) * lda_g + q * S3 + 2 * c);
-                v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
-                v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
-                la[c] = v;
-            }
-        }
-        if (mine && role == 0 && lane > 0) la_new = LAt[(q * S3 + lane) * lda_g + q * S3 + lane - 1];
         __syncthreads();
         if (!kOverlap) {
             stage_subtile(e + 1 - pp, 0, kThreadsC);  // lands while this phase sweeps
@@ -373,6 +545,7 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
                 }
             }
         }
+        load_la(q + 1);  // the next phase's sub-tile of this CTA
         __syncthreads();
         if (p.wt_out && mine) {  // the pre-rounding values of this phase's sub-tile
             for (int idx = tid; idx < S3 * S3; idx += kThreadsC) {
@@ -394,24 +567,48 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo)
         p.Dhi[gi * p.Np + gj] = hi;
         p.Dlo[gi * p.Np + gj] = lo;
     }
+    if (kPair && !consumer) {
+        // this row block's in-tile R for the right neighbour, then the flag
+        // (every thread fences its own writes before the CTA barrier)
+        for (int idx = tid; idx < S3 * T / 4; idx += kThreadsC) {
+            const int r = idx / (T / 4), c4 = idx % (T / 4);
+            *(float4 *)(p.Rx + (brow0 + r) * p.Np + col0 + 4 * c4) = *(const float4 *)(sR + r * RSC + 4 * c4);
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0 && p.omit_flag != I * p.Nt + J + 1) atomicAdd(p.flags + (int64_t)I * p.Nt + J, 1);
+    }
     // the other CTAs may still read this CTA's D until their last phase
     cluster.sync();
 }
 
 cudaError_t leaf_cluster_configure()
 {
-    cudaError_t e = cudaFuncSetAttribute(leaf_cluster_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemCLaunch);
+    cudaError_t e = cudaFuncSetAttribute(leaf_cluster_kernel<false, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCLaunch);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(leaf_cluster_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kSmemCLaunch);
+    e = cudaFuncSetAttribute(leaf_cluster_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemCLaunch);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(leaf_cluster_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSmemPairLaunch);
 }
 
 cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, bool overlap, cudaStream_t stream)
 {
     if (overlap)
-        return launch_pdl(leaf_cluster_kernel<true>, dim3(4 * tiles), dim3(128), kSmemCLaunch, stream, p, K, I_lo);
-    return launch_pdl(leaf_cluster_kernel<false>, dim3(4 * tiles), dim3(96), kSmemCLaunch, stream, p, K, I_lo);
+        return launch_pdl(leaf_cluster_kernel<true, false>, dim3(4 * tiles), dim3(128), kSmemCLaunch, stream, p, K,
+                          I_lo, 0);
+    return launch_pdl(leaf_cluster_kernel<false, false>, dim3(4 * tiles), dim3(96), kSmemCLaunch, stream, p, K, I_lo,
+                      0);
+}
+
+cudaError_t launch_leaf_pair(const LeafArgs &p, int K, int slot, cudaStream_t stream)
+{
+    auto tiles = [&](int k) { return min(p.Mt - 1, k) - max(0, k - (p.Nt - 1)) + 1; };
+    const int n = tiles(K) + tiles(K + 1);
+    return launch_pdl(leaf_cluster_kernel<true, true>, dim3(4 * n), dim3(128), kSmemPairLaunch, stream, p, K, 0,
+                      slot);
 }
 
 }  // namespace bakron
