@@ -32,8 +32,10 @@ TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 : BF16 tensor peak ratio
 FALLBACK_BF16_TFLOPS = 1590.0
 LEAF_BYTES_PER_WEIGHT = 25  # read Wt 4 + diagonal factor blocks 8; write code 1, V 4, D hi/lo 8
 LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 255), 3: ("leaf_warp_kernel", 7 * 63),
-                4: ("leaf_wide_kernel", 3 * 127), 5: ("leaf_cluster_kernel<false, false>", 7 * 63),
-                6: ("leaf_cluster_kernel<true, false>", 7 * 63), 7: ("leaf_cluster_kernel<true, true>", 7 * 63)}
+                4: ("leaf_wide_kernel", 3 * 127), 5: ("leaf_cluster_kernel<false, false, false>", 7 * 63),
+                6: ("leaf_cluster_kernel<true, false, false>", 7 * 63),
+                7: ("leaf_cluster_kernel<true, true, false>", 7 * 63),
+                8: ("leaf_cluster_kernel<true, false, true>", 7 * 63)}
 # DRAM traffic of the band products from an ncu capture of one solve's 93
 # band launches (profiles/band_4096_dram.md); reported only while the band
 # kernel sources hash to the value the capture was taken with.
@@ -163,6 +165,16 @@ def load_inputs(name, rank, dist):
     if dist is not None and rank == 0:
         dist.barrier()
     return W, A, B
+
+
+FP64_PEAK_NOMINAL = 37.0  # TFLOP/s, B200 FP64 (CUDA-core and tensor-core rates are the same)
+
+
+def factor_flops(d):
+    """Flops of chol(M^-1) for a d x d factor as the path computes it: the
+    Cholesky factorisation (d^3 / 6 multiply-adds) and the triangular inverse
+    (d^3 / 6 multiply-adds), two flops per multiply-add."""
+    return 2 * (d ** 3 / 6 + d ** 3 / 6)
 
 
 def oracle_factors(A, B):
@@ -545,6 +557,11 @@ def main():
                      "share_of_profiled_step": pr["leaf_ms"] / pr["total_ms"]},
             "profile_ms": pr,
             "factor_ms": factor_ms,
+            "factor": {"ms": factor_ms, "flops": factor_flops(n) + factor_flops(m),
+                       "fp64_tflops": (factor_flops(n) + factor_flops(m)) / (factor_ms / 1e3) / 1e12,
+                       "fp64_peak_tflops_nominal": FP64_PEAK_NOMINAL,
+                       "note": "chol(A^-1) and chol(B^-1) in FP64 (Cholesky d^3/6 + triangular inverse "
+                               "d^3/6 multiply-adds, 2 flops each, per factor); outside the metric"},
             "cpu_baseline": cb,
             "e2e": None if e2e_ms is None else {
                 "value": aggregate_rate(world, m, n, e2e_ms), "unit": "weights/s",

@@ -28,6 +28,17 @@ def _t(x):
     return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
 
 
+def fp64_then_rounded(Lg, Lo, label):
+    """The factor is computed in FP64 and rounded once to fp32: every entry
+    lies within half an fp32 ulp of the oracle's FP64 value, plus the FP64
+    path's own error (cond(M) * 2^-52 relative, far below 1e-9 of the largest
+    entry for these damped Gram factors)."""
+    excess = np.abs(Lg - Lo) - 2.0 ** -24 * np.abs(Lo) * (1 + 2.0 ** -20)
+    worst = float(excess.max()) / float(np.abs(Lo).max())
+    print(f"[{label}] max (|L - L_oracle| - half ulp) / max|L| = {worst:.3g}")
+    assert worst <= 1e-9
+
+
 @pytest.mark.parametrize("name", ["tiny", "mid"])
 def test_factor_matches_oracle(bk, name):
     W, A, B = workloads.generate(name)
@@ -40,6 +51,7 @@ def test_factor_matches_oracle(bk, name):
         print(name, "factor rel err", rel, "max |L L^T A - I|", resid)
         assert np.all(np.triu(Lg, 1) == 0) and np.all(np.diag(Lg) > 0)
         assert rel <= 1e-5
+        fp64_then_rounded(Lg, Lo, f"{name} {M.shape[0]}")
 
 
 @pytest.mark.slow
@@ -64,15 +76,19 @@ def test_factor_full_size_matches_oracle(bk, name, side):
     print(f"[{name} {side}, {M.shape[0]}] factor rel err {rel:.3g}, max |L L^T M - I| {resid:.3g}")
     assert np.all(np.triu(Lg, 1) == 0) and np.all(np.diag(Lg) > 0)
     assert rel <= 1e-5
+    fp64_then_rounded(Lg, Lo, f"{name} {side} {M.shape[0]}")
 
 
-@pytest.mark.parametrize("n", [1, 2, 63, 64, 65, 200, 513])
+# one panel, ragged panels, and sizes whose recursive inverse splits unevenly
+@pytest.mark.parametrize("n", [1, 2, 63, 64, 65, 127, 129, 200, 513, 1000, 2111])
 def test_factor_sizes(bk, n):
     _, A, _ = workloads.random_problem(2, n, seed=n)
     LA, _ = bk.factor(_t(A), None)
     Lg = LA.cpu().numpy().astype(np.float64)
     Lo = oracle.factor(A)
     assert np.linalg.norm(Lg - Lo) / np.linalg.norm(Lo) <= 1e-5
+    assert np.all(np.triu(Lg, 1) == 0)
+    fp64_then_rounded(Lg, Lo, f"n={n}")
 
 
 def test_factor_not_spd(bk):

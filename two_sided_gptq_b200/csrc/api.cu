@@ -30,8 +30,8 @@ constexpr const char *kVersion = "bakron-b200 0.2";
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Leaf structures bakron_tune_leaf times (bakron_config_t.leaf 1..7).
-constexpr int kLeafStructures = 7;
+// Leaf structures bakron_tune_leaf times (bakron_config_t.leaf 1..8).
+constexpr int kLeafStructures = 8;
 // 0-based leaf variant of structure 7: width-2 ranges of the recursion run as
 // one launch of two tile diagonals (structure 6's kernel for single ones).
 constexpr int kPairVariant = 6;
@@ -802,7 +802,7 @@ size_t bakron_factor_workspace_size(int64_t n, int64_t m)
 {
     if (n < 0 || m < 0 || (n == 0 && m == 0)) return 0;
     int64_t d = std::max(n, m);
-    return align_up(kStatusBytes) + align_up((size_t)2 * d * d * sizeof(double));
+    return align_up(kStatusBytes) + align_up(factor_work_doubles(d) * sizeof(double));
 }
 
 bakron_status_t bakron_factor(const float *A_dev, int64_t n, const float *B_dev, int64_t m,

@@ -43,10 +43,11 @@ cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, c
 
 cudaError_t leaf_configure();
 cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stream);
-// Leaf with one tile per cluster of four CTAs (leaf_cluster.cu); overlap:
-// a fourth warp forms the older product terms during the sweeps.
+// Leaf with one tile per cluster of four CTAs (leaf_cluster.cu); form 0:
+// three sweep warps, 1: a fourth warp forms the older product terms during
+// the sweeps, 2: as 1 with the sweep warps handing over through mbarriers.
 cudaError_t leaf_cluster_configure();
-cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, bool overlap, cudaStream_t stream);
+cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, int form, cudaStream_t stream);
 // Tile diagonals K and K+1 in one launch (leaf structure 7): ticket counter
 // `slot`; the second diagonal's clusters wait for their neighbours' flags.
 cudaError_t launch_leaf_pair(const LeafArgs &p, int K, int slot, cudaStream_t stream);
@@ -92,7 +93,9 @@ int64_t proxy_loss_parts(int64_t m, int64_t n);
 cudaError_t launch_proxy_loss(const float *W, const float *V, const float *A, const float *B,
                               int64_t m, int64_t n, double *out, double *part, cudaStream_t stream);
 
-// FP64 factorisation: L (n x n, fp32) = chol(A^{-1}); work = n*n doubles.
+// FP64 factorisation: L (n x n, fp32) = chol(A^{-1}); work holds
+// factor_work_doubles(n) doubles.
+size_t factor_work_doubles(int64_t n);
 cudaError_t launch_factor(const float *A, int64_t n, float *L, double *work, DeviceStatus *st,
                           cudaStream_t stream);
 
