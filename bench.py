@@ -32,10 +32,8 @@ TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 : BF16 tensor peak ratio
 FALLBACK_BF16_TFLOPS = 1590.0
 LEAF_BYTES_PER_WEIGHT = 25  # read Wt 4 + diagonal factor blocks 8; write code 1, V 4, D hi/lo 8
 LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 255), 3: ("leaf_warp_kernel", 7 * 63),
-                4: ("leaf_wide_kernel", 3 * 127), 5: ("leaf_cluster_kernel<false, false, false>", 7 * 63),
-                6: ("leaf_cluster_kernel<true, false, false>", 7 * 63),
-                7: ("leaf_cluster_kernel<true, true, false>", 7 * 63),
-                8: ("leaf_cluster_kernel<true, false, true>", 7 * 63)}
+                4: ("leaf_wide_kernel", 3 * 127), 5: ("leaf_cluster_kernel<false, false>", 7 * 63),
+                6: ("leaf_cluster_kernel<true, false>", 7 * 63), 7: ("leaf_cluster_kernel<true, true>", 7 * 63)}
 # DRAM traffic of the band products from an ncu capture of one solve's 93
 # band launches (profiles/band_4096_dram.md); reported only while the band
 # kernel sources hash to the value the capture was taken with.
@@ -167,7 +165,7 @@ def load_inputs(name, rank, dist):
     return W, A, B
 
 
-FP64_PEAK_NOMINAL = 37.0  # TFLOP/s, B200 FP64 (CUDA-core and tensor-core rates are the same)
+FP64_PEAK_NOMINAL = 37.0  # TFLOP/s, nominal B200 FP64
 
 
 def factor_flops(d):

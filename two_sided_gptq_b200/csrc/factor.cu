@@ -42,6 +42,24 @@ __global__ void rev_copy_kernel(const float *__restrict__ A, int64_t n, double *
     }
 }
 
+// 1/sqrt(d) to FP64 accuracy by Newton's iteration for the reciprocal square
+// root, y <- y + y (1 - d y^2) / 2, from the single-precision estimate: each
+// step squares the relative error (about 2^-22, 2^-44, then FP64 rounding).
+// Pivots outside the range where the single-precision estimate is safe take
+// the IEEE square root and division.
+__device__ __forceinline__ double rsqrt_fp64(double d)
+{
+    if (!(d > 1e-30 && d < 1e30)) return 1.0 / sqrt(d);
+    double y = (double)rsqrtf((float)d);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const double h = d * y;
+        const double r = fma(-h, y, 1.0);
+        y = fma(0.5 * y, r, y);
+    }
+    return y;
+}
+
 // Diagonal block [kb, kb+bs): its Cholesky factor C_kk into X and C_kk^-1
 // into Y (both lower; Y's block gets explicit zeros above the diagonal).  256
 // threads, each holding a 4 x 4 set of the 64 x 64 block in registers (rows
@@ -55,6 +73,7 @@ __global__ void __launch_bounds__(256) potrf_inv_kernel(double *X, double *Y, in
 {
     __shared__ double vec[2][NB];
     __shared__ double cf[NB][NB + 1];
+    __shared__ double rdiag[NB];  // 1 / C_kk[j][j]
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     double a[4][4];
 #pragma unroll
@@ -75,7 +94,8 @@ __global__ void __launch_bounds__(256) potrf_inv_kernel(double *X, double *Y, in
             if (tid == 0) record_error(st, BAKRON_ERR_NOT_SPD, (int)(kb + j));
             d = 1.0;
         }
-        const double piv = sqrt(d), rp = 1.0 / piv;
+        const double rp = rsqrt_fp64(d), piv = d * rp;
+        if (tid == 0) rdiag[j] = rp;
         double li[4], lk[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) li[r] = ty + 16 * r > j ? cj[ty + 16 * r] * rp : 0.0;
@@ -122,7 +142,7 @@ __global__ void __launch_bounds__(256) potrf_inv_kernel(double *X, double *Y, in
     __syncthreads();
     for (int t = 0; t < NB; ++t) {
         const double *yt = vec[t & 1];
-        const double rd = 1.0 / cf[t][t];
+        const double rd = rdiag[t];
         double v[4], ci[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) v[c] = yt[tx + 16 * c] * rd;

@@ -43,11 +43,10 @@ cudaError_t launch_prep(const float *W, int64_t m, int64_t n, const float *LA, c
 
 cudaError_t leaf_configure();
 cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stream);
-// Leaf with one tile per cluster of four CTAs (leaf_cluster.cu); form 0:
-// three sweep warps, 1: a fourth warp forms the older product terms during
-// the sweeps, 2: as 1 with the sweep warps handing over through mbarriers.
+// Leaf with one tile per cluster of four CTAs (leaf_cluster.cu); overlap:
+// a fourth warp forms the older product terms during the sweeps.
 cudaError_t leaf_cluster_configure();
-cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, int form, cudaStream_t stream);
+cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, bool overlap, cudaStream_t stream);
 // Tile diagonals K and K+1 in one launch (leaf structure 7): ticket counter
 // `slot`; the second diagonal's clusters wait for their neighbours' flags.
 cudaError_t launch_leaf_pair(const LeafArgs &p, int K, int slot, cudaStream_t stream);

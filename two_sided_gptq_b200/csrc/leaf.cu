@@ -980,8 +980,8 @@ cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stre
 {
     int I_lo = max(0, K - (p.Nt - 1)), I_hi = min(p.Mt - 1, K);
     if (I_hi < I_lo) return cudaSuccess;
-    if (variant == 4 || variant == 5 || variant == 7)
-        return launch_leaf_cluster(p, K, I_lo, I_hi - I_lo + 1, variant == 7 ? 2 : variant == 5 ? 1 : 0, stream);
+    if (variant == 4 || variant == 5)
+        return launch_leaf_cluster(p, K, I_lo, I_hi - I_lo + 1, variant == 5, stream);
     if (variant == 3)
         return launch_pdl(leaf_wide_kernel, dim3(I_hi - I_lo + 1), dim3(kThreadsWide), kSmemWide, stream, p, K, I_lo);
     if (variant == 2)

@@ -30,17 +30,6 @@
 // other CTAs), so between two sweeps only the newest terms remain, shared by
 // all four warps.
 //
-// Decoupled sweep (kDec, structure 8, on top of the overlapped form): the
-// three sweep warps no longer meet at a barrier every step.  The side warps
-// work three steps ahead of need: the sums they hand over leave out the two
-// newest terms of each side, which the entry warp adds itself from its own
-// registers -- D[a-1][b] and D[a-2][b] are its own last two results, R[a][b-1]
-// and R[a][b-2] the last results of the lanes one and two columns over
-// (shuffles).  Hand-offs go through four mbarrier slots: "done" (the entry
-// warp finished step g, so its R and D are in shared memory) and "full" (both
-// side warps wrote their sums for step g); a side warp producing step g waits
-// for done[g-3], the entry warp for full[g].  Every wait is bounded.
-//
 // Two tile diagonals per launch (kPair, structure 7): clusters take tickets
 // from a counter in the order they start; the first tickets take the tiles of
 // diagonal K, the rest those of K + 1, so a cluster only ever waits for
@@ -65,7 +54,6 @@
 #include "common.cuh"
 #include "kernels.cuh"
 #include "leaf_common.cuh"
-#include "tcgen05.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -112,14 +100,11 @@ __device__ __forceinline__ bool wait_counter(const int32_t *ctr, int target, uin
 }
 }  // namespace
 
-template <bool kOverlap, bool kPair, bool kDec>
+template <bool kOverlap, bool kPair>
 __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kOverlap ? 128 : 96, 1)
 leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
 {
-    static_assert(!kDec || (kOverlap && !kPair), "the decoupled sweep builds on the overlapped single-diagonal form");
     constexpr int kThreadsC = kOverlap ? 128 : 96;
-    // the side warps' sums leave out this many newest terms of each side
-    constexpr int kLag = kDec ? 3 : 2;
     cg::cluster_group cluster = cg::this_cluster();
     const int pp = (int)cluster.block_rank();  // row block of sub-tiles
 
@@ -144,13 +129,6 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
     float *cB = cR + S3 * CKS;                // S3 x CKS: LtB[I', I'-1] rows, chunk
     float *cA = cB + S3 * CKS;                // T x CKS: LtA[J', J'-1] rows, chunk
     float *cD = cA + T * CKS;                 // S3 x T: D_up rows of the chunk
-
-    // decoupled sweep: mbarriers full[0..3], done[0..3]; the side warps' sums
-    // in four step slots; LtB[r][r-2] inside the row block; the abort flag of
-    // a wait that ran out
-    __shared__ __align__(8) uint64_t sbar[8];
-    __shared__ float sPS4[kDec ? 4 * S3 : 1], sPU4[kDec ? 4 * S3 : 1], sLBd2[kDec ? S3 : 1];
-    __shared__ int sabort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // the cluster's tile: by launch position, or (pair form) by ticket
@@ -189,16 +167,6 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
         ((float4 *)sDt)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int idx = tid; idx < 2 * S3 * WSC / 4; idx += kThreadsC)  // O_S, O_U
         ((float4 *)sOS)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (kDec) {
-        if (tid == 0) {
-            for (int i = 0; i < 4; ++i) {
-                tc::mbar_init(tc::smem_u32(&sbar[i]), 2 * 32);  // full: both side warps
-                tc::mbar_init(tc::smem_u32(&sbar[4 + i]), 32);  // done: the entry warp
-            }
-            sabort = 0;
-        }
-        for (int idx = tid; idx < 4 * S3; idx += kThreadsC) sPS4[idx] = sPU4[idx] = 0.f;
-    }
     __syncthreads();  // R is zero before the first staged block lands in it
     pdl_wait();       // every global input (Wt, factors, steps) comes from earlier kernels
     const bool has_left = kPair && consumer && J >= 1;  // neighbours on the first diagonal
@@ -328,17 +296,16 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
     if (tid < S3) sLBd[tid] = tid > 0 ? LBt[(pp * S3 + tid) * ldb_g + pp * S3 + tid - 1] : 0.f;
-    if (kDec && tid < S3) sLBd2[tid] = tid > 1 ? LBt[(pp * S3 + tid) * ldb_g + pp * S3 + tid - 2] : 0.f;
     const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
     const int role = warp;  // 0 entries, 1 row side, 2 column side, 3 (overlapped form) older products
-    // column-side warp: its LtB[p,p] row rho (columns <= rho-kLag), fixed for the kernel
+    // column-side warp: its LtB[p,p] row rho (columns <= rho-2), fixed for the kernel
     float2 lbr[S3 / 2];
     if (role == 2) {
 #pragma unroll
         for (int c = 0; c < S3 / 2; ++c) {
             float2 v = *(const float2 *)(LBt + (pp * S3 + lane) * ldb_g + pp * S3 + 2 * c);
-            v.x = 2 * c + 0 <= lane - kLag ? v.x : 0.f;
-            v.y = 2 * c + 1 <= lane - kLag ? v.y : 0.f;
+            v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
+            v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
             lbr[c] = v;
         }
     }
@@ -354,29 +321,26 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
     }
     const bool exact_div = __syncthreads_or(out_of_range) != 0;
 
-    // row-side warp: LtA[q,q] row b (columns <= b-kLag); entry warp: LtA[b][b-1]
-    // (and LtA[b][b-2] for the decoupled sweep).  Loaded for the CTA's next
-    // sub-tile as soon as the previous sweep ends, so the L2 latency overlaps
-    // the phase change.
+    // row-side warp: LtA[q,q] row b (columns <= b-2); entry warp: LtA[b][b-1].
+    // Loaded for the CTA's next sub-tile as soon as the previous sweep ends, so
+    // the L2 latency overlaps the phase change.
     float2 la[S3 / 2];
-    float la_new = 0.f, la_new2 = 0.f;
+    float la_new = 0.f;
     auto load_la = [&](int q) {
         if (q < 0 || q > 3) return;
         if (role == 1) {
 #pragma unroll
             for (int c = 0; c < S3 / 2; ++c) {
                 float2 v = *(const float2 *)(LAt + (q * S3 + lane) * lda_g + q * S3 + 2 * c);
-                v.x = 2 * c + 0 <= lane - kLag ? v.x : 0.f;
-                v.y = 2 * c + 1 <= lane - kLag ? v.y : 0.f;
+                v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
+                v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
                 la[c] = v;
             }
         }
         if (role == 0 && lane > 0) la_new = LAt[(q * S3 + lane) * lda_g + q * S3 + lane - 1];
-        if (kDec && role == 0 && lane > 1) la_new2 = LAt[(q * S3 + lane) * lda_g + q * S3 + lane - 2];
     };
     load_la(0 - pp);
 
-    int gstep = 0;  // decoupled sweep: steps this CTA has swept so far (mbarrier phases)
     for (int e = 0; e < 7; ++e) {
         const int q = e - pp;
         const bool mine = q >= 0 && q <= 3;
@@ -468,146 +432,7 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
                 }
             }
         }
-        if (kDec && mine && role < 3) {
-            const uint32_t bar_full = tc::smem_u32(&sbar[0]), bar_done = tc::smem_u32(&sbar[4]);
-            // bounded wait: after a wait ran out every later one returns at
-            // once (the sweep finishes with garbage, the cluster barriers stay
-            // balanced, the status says why)
-            auto wait_bar = [&](uint32_t bar, int g, int where) {
-                const uint32_t parity = (uint32_t)(g >> 2) & 1u;
-                if (tc::mbar_try_wait(bar, parity)) return;
-                const uint64_t deadline = tc::now_ns() + (uint64_t)p.timeout_ms * 1000000ull;
-                while (!tc::mbar_try_wait(bar, parity)) {
-                    if (*(volatile int *)&sabort != 0) return;
-                    if (tc::now_ns() > deadline) {
-                        if (atomicExch(&sabort, 1) == 0) record_error(p.st, BAKRON_ERR_DEVICE_TIMEOUT, where);
-                        return;
-                    }
-                }
-            };
-            if (role == 0) {
-                // ---- entry warp (lane = column b): rounds entry (d - b, b) at step d
-                const int b = lane, tb = q * S3 + b;
-                auto row_consts = [&](int a, float &w0, float &l1, float &l2, float &sv, float &rv_, float &s0) {
-                    const int ac = min(max(a, 0), S3 - 1);
-                    w0 = sW[ac * WSC + b];
-                    l1 = sLBd[ac];
-                    l2 = sLBd2[ac];
-                    sv = scale[ac];
-                    rv_ = rcp[ac];
-                    s0 = sR[ac * RSC + tb];  // S[a][b] until this entry overwrites it
-                };
-                auto sweep = [&](auto ieee_tag) {
-                    constexpr bool kIeee = decltype(ieee_tag)::value;
-                    float w0, lb1, lb2, sc_s, sc_r, s_ab;
-                    row_consts(-b, w0, lb1, lb2, sc_s, sc_r, s_ab);
-                    // own D of the last two steps (rows a-1, a-2 of column b), own R of
-                    // the last two steps, and the R of lanes b-1 / b-2 for this step
-                    float d1 = 0.f, d2 = 0.f, r1 = 0.f, r2 = 0.f, rl1 = 0.f, rl2 = 0.f;
-                    wait_bar(bar_full + 8 * (gstep & 3), gstep, 5000 + 10 * pp);
-                    float ps_in = sPS4[(gstep & 3) * S3 + b], pu_in = sPU4[(gstep & 3) * S3 + b];
-#pragma unroll 2
-                    for (int d = 0; d < 2 * S3 - 1; ++d) {
-                        const int g = gstep + d;
-                        const int a = d - b;
-                        const int ac = min(max(a, 0), S3 - 1);
-                        float w0n, l1n, l2n, sn, rn, s_n;
-                        row_consts(a + 1, w0n, l1n, l2n, sn, rn, s_n);
-                        const float sc = fmaf(lb1, d1, fmaf(lb2, d2, ps_in));
-                        const float wt = w0 - fmaf(rl1, la_new, fmaf(rl2, la_new2, pu_in)) - sc;
-                        // clamp(rint(wt / s)) with the correctly rounded fp32 quotient
-                        const float qf = kIeee ? __fdiv_rn(wt, sc_s) : div_rn_recip(wt, sc_s, sc_r);
-                        const float cq = fminf(fmaxf(rintf(qf), fqmin), fqmax);
-                        const bool valid = a >= 0 && a < mrb && tb < nc;
-                        const float dl = valid ? fmaf(-sc_s, cq, wt) : 0.f;
-                        const float rr = s_ab + sc + dl;
-                        d2 = d1; d1 = dl; r2 = r1; r1 = rr;
-                        rl1 = __shfl_up_sync(0xffffffffu, r1, 1);  // R[a+1][b-1] for the next step
-                        rl2 = __shfl_up_sync(0xffffffffu, r2, 2);  // R[a+1][b-2]
-                        // invalid lanes write to spare slots instead of branching
-                        const int iR = valid ? a * RSC + tb : S3 * RSC + lane;
-                        const int iD = valid ? tb * DSC + a : T * DSC + lane;
-                        const int iC = valid ? a * T + tb : S3 * T + lane;
-                        const int iW = valid ? a * WSC + b : ac * WSC + S3 + (lane & 3);  // row padding
-                        sR[iR] = rr;
-                        sDt[iD] = dl;
-                        sCode[iC] = code_byte(cq);
-                        sW[iW] = wt;  // pre-rounding value, copied out when requested
-                        tc::mbar_arrive(bar_done + 8 * (g & 3));
-                        if (d + 1 < 2 * S3 - 1) {
-                            wait_bar(bar_full + 8 * ((g + 1) & 3), g + 1, 5000 + 10 * pp);
-                            ps_in = sPS4[((g + 1) & 3) * S3 + b];
-                            pu_in = sPU4[((g + 1) & 3) * S3 + b];
-                        }
-                        w0 = w0n; lb1 = l1n; lb2 = l2n; sc_s = sn; sc_r = rn; s_ab = s_n;
-                    }
-                };
-                if (exact_div)
-                    sweep(std::true_type{});
-                else
-                    sweep(std::false_type{});
-            } else if (role == 1) {
-                // ---- row-side warp (lane = column b): sum_{c <= b-3} R[a][c] LtA[b][c]
-                // for the entry (a, b) of step d, once the entry warp finished step d-3
-                const int b = lane;
-                float4 rv[S3 / 4];
-#pragma unroll
-                for (int c = 0; c < S3 / 4; ++c) rv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-                for (int d = 0; d < 2 * S3 - 1; ++d) {
-                    const int g = gstep + d;
-                    if (d >= kLag) wait_bar(bar_done + 8 * ((g - kLag) & 3), g - kLag, 5001 + 10 * pp);
-                    const int an = min(max(d - b, 0), S3 - 1);
-                    const float *Rn = sR + an * RSC + q * S3;
-#pragma unroll
-                    for (int c = 0; c < S3 / 4; ++c)
-                        if (4 * c <= b - kLag) rv[c] = *(const float4 *)(Rn + 4 * c);
-                    float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
-                    float2 u2 = make_float2(0.f, 0.f), u3 = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int c = 0; c < S3 / 4; c += 2) {
-                        u0 = ffma2(make_float2(rv[c].x, rv[c].y), la[2 * c], u0);
-                        u1 = ffma2(make_float2(rv[c].z, rv[c].w), la[2 * c + 1], u1);
-                        u2 = ffma2(make_float2(rv[c + 1].x, rv[c + 1].y), la[2 * c + 2], u2);
-                        u3 = ffma2(make_float2(rv[c + 1].z, rv[c + 1].w), la[2 * c + 3], u3);
-                    }
-                    sPU4[(g & 3) * S3 + b] = ((u0.x + u1.x) + (u2.x + u3.x)) + ((u0.y + u1.y) + (u2.y + u3.y));
-                    tc::mbar_arrive(bar_full + 8 * (g & 3));
-                }
-            } else {
-                // ---- column-side warp (lane = row rho): sum_{r <= rho-3} LtB[rho][r] D[r][b]
-                // for the entry (rho, b = d - rho) of step d
-                const int rho = lane;
-                float4 dv[S3 / 4];
-#pragma unroll
-                for (int c = 0; c < S3 / 4; ++c) dv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-                for (int d = 0; d < 2 * S3 - 1; ++d) {
-                    const int g = gstep + d;
-                    if (d >= kLag) wait_bar(bar_done + 8 * ((g - kLag) & 3), g - kLag, 5002 + 10 * pp);
-                    const int b = d - rho;
-                    const int bc = min(max(b, 0), S3 - 1);
-                    const float *Dc = sDt + (q * S3 + bc) * DSC;
-#pragma unroll
-                    for (int c = 0; c < S3 / 4; ++c)
-                        if (4 * c <= rho - kLag) dv[c] = *(const float4 *)(Dc + 4 * c);
-                    float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
-                    float2 s2 = make_float2(0.f, 0.f), s3 = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int c = 0; c < S3 / 4; c += 2) {
-                        s0 = ffma2(make_float2(dv[c].x, dv[c].y), lbr[2 * c], s0);
-                        s1 = ffma2(make_float2(dv[c].z, dv[c].w), lbr[2 * c + 1], s1);
-                        s2 = ffma2(make_float2(dv[c + 1].x, dv[c + 1].y), lbr[2 * c + 2], s2);
-                        s3 = ffma2(make_float2(dv[c + 1].z, dv[c + 1].w), lbr[2 * c + 3], s3);
-                    }
-                    if (b == bc)
-                        sPS4[(g & 3) * S3 + b] = ((s0.x + s1.x) + (s2.x + s3.x)) + ((s0.y + s1.y) + (s2.y + s3.y));
-                    tc::mbar_arrive(bar_full + 8 * (g & 3));
-                }
-            }
-        }
-        if (kDec && mine) gstep += 2 * S3 - 1;
-        if (!kDec && mine && role < 3) {
+        if (mine && role < 3) {
             float *ps_buf = sPS, *pu_buf = sPU;
             if (role == 0) {
                 // ---- entry warp (lane = column b): rounds entry (d - b, b) at step d
@@ -759,37 +584,31 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
 
 cudaError_t leaf_cluster_configure()
 {
-    cudaError_t e = cudaFuncSetAttribute(leaf_cluster_kernel<false, false, false>,
+    cudaError_t e = cudaFuncSetAttribute(leaf_cluster_kernel<false, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCLaunch);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(leaf_cluster_kernel<true, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(leaf_cluster_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemCLaunch);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(leaf_cluster_kernel<true, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemCLaunch);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(leaf_cluster_kernel<true, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(leaf_cluster_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kSmemPairLaunch);
 }
 
-cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, int form, cudaStream_t stream)
+cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, bool overlap, cudaStream_t stream)
 {
-    if (form == 2)
-        return launch_pdl(leaf_cluster_kernel<true, false, true>, dim3(4 * tiles), dim3(128), kSmemCLaunch, stream,
-                          p, K, I_lo, 0);
-    if (form == 1)
-        return launch_pdl(leaf_cluster_kernel<true, false, false>, dim3(4 * tiles), dim3(128), kSmemCLaunch, stream,
-                          p, K, I_lo, 0);
-    return launch_pdl(leaf_cluster_kernel<false, false, false>, dim3(4 * tiles), dim3(96), kSmemCLaunch, stream, p,
-                      K, I_lo, 0);
+    if (overlap)
+        return launch_pdl(leaf_cluster_kernel<true, false>, dim3(4 * tiles), dim3(128), kSmemCLaunch, stream, p, K,
+                          I_lo, 0);
+    return launch_pdl(leaf_cluster_kernel<false, false>, dim3(4 * tiles), dim3(96), kSmemCLaunch, stream, p, K, I_lo,
+                      0);
 }
 
 cudaError_t launch_leaf_pair(const LeafArgs &p, int K, int slot, cudaStream_t stream)
 {
     auto tiles = [&](int k) { return min(p.Mt - 1, k) - max(0, k - (p.Nt - 1)) + 1; };
     const int n = tiles(K) + tiles(K + 1);
-    return launch_pdl(leaf_cluster_kernel<true, true, false>, dim3(4 * n), dim3(128), kSmemPairLaunch, stream, p, K,
-                      0, slot);
+    return launch_pdl(leaf_cluster_kernel<true, true>, dim3(4 * n), dim3(128), kSmemPairLaunch, stream, p, K, 0,
+                      slot);
 }
 
 }  // namespace bakron
