@@ -10,11 +10,11 @@
 //
 // Blocked right-looking Cholesky on 64-wide panels (the diagonal block's
 // factor and its inverse in one CTA; the panel solve and the trailing
-// symmetric update as GEMMs) and a recursive triangular
-// inverse, inv([[A, 0], [B, C]]) = [[A^-1, 0], [-C^-1 B A^-1, C^-1]], whose
-// merges are two GEMMs each; all FP64 on the CUDA cores.  The GEMM is one
-// register-blocked kernel (128 x 128 or 64 x 64 output tiles) that skips the
-// zero halves of triangular operands.
+// symmetric update as GEMMs) and a triangular inverse built bottom-up from
+// the diagonal blocks' inverses, inv([[A, 0], [B, C]]) = [[A^-1, 0],
+// [-C^-1 B A^-1, C^-1]], each level's merges two batched GEMMs; all FP64.
+// The GEMM runs on the FP64 tensor cores (128 x 128 or 64 x 64 output tiles)
+// and skips the zero halves of triangular operands.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -175,129 +175,168 @@ __global__ void __launch_bounds__(256) potrf_inv_kernel(double *X, double *Y, in
 }
 
 // C[i][j] = alpha sum_k A[i][k] B'[k][j] + beta C[i][j] for an M x N output,
-// with A row-major (lda) and B' = B row-major K x N (ldb) or, with
-// B_KMAJOR, B' = B^T for B row-major N x K.  flags: kLowerOut computes and
-// writes only entries with j <= i (tiles above the diagonal are skipped);
-// kLowerA (A[i][k] = 0 for k > i) and kLowerB (B'[k][j] = 0 for j > k) shorten
-// each tile's contraction range to the part that can be non-zero.  256 threads
-// per 16R x 16R tile, R x R outputs each (rows ty + 16 r, columns tx + 16 c),
-// K in steps of 16 through shared memory, the next step's tiles fetched into
-// registers while the current one is consumed.  Every CTA reads all the A
-// rows it writes before its first store (the last barrier of the K loop
-// separates them), so C may be A itself when N fits one tile column.
+// with A row-major (lda) and B' = B row-major K x N (ldb) or, with B_KMAJOR,
+// B' = B^T for B row-major N x K; on the FP64 tensor cores
+// (mma.sync.m8n8k4.f64).  flags: kLowerOut computes and writes only entries
+// with j <= i (tiles above the diagonal are skipped); kLowerA
+// (A[i][k] = 0 for k > i) and kLowerB (B'[k][j] = 0 for j > k) shorten each
+// tile's contraction range to the part that can be non-zero.  Batched over
+// blockIdx.z: problem z reads A + z sA, B + z sB and writes C + z sC, the last
+// one with M_last rows and contraction length K_last.  256 threads per
+// TM x TN tile as 2 x 4 warps; K in steps of 16 through shared memory (k-major
+// rows padded by 8 doubles so the fragment loads take two wavefronts), the
+// next step's tiles fetched into registers while the current one is
+// consumed.  Every CTA reads all the A rows it writes before its first store
+// (the last barrier of the K loop separates them), so C may be A itself when
+// N fits one tile column.
 namespace {
 constexpr int GK = 16;
 constexpr int kLowerOut = 1, kLowerA = 2, kLowerB = 4;
-}
 
-template <bool B_KMAJOR, int R>
-__global__ void __launch_bounds__(256) dgemm_kernel(int M, int N, int K, const double *A, int64_t lda,
-                                                    const double *__restrict__ B, int64_t ldb, double *C,
-                                                    int64_t ldc, double alpha, double beta, int flags)
+struct GemmD {
+    int M, N, K, M_last, K_last;
+    const double *A;
+    int64_t lda, sA;
+    const double *B;
+    int64_t ldb, sB;
+    double *C;
+    int64_t ldc, sC;
+    double alpha, beta;
+    int flags;
+};
+
+__device__ __forceinline__ void dmma(double (&c)[2], double a, double b)
 {
-    constexpr int GT = 16 * R;
-    const int i0 = blockIdx.y * GT, j0 = blockIdx.x * GT;
-    if ((flags & kLowerOut) && j0 > i0 + GT - 1) return;
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(c[0]), "+d"(c[1])
+                 : "d"(a), "d"(b));
+}
+}  // namespace
+
+template <bool B_KMAJOR, int TM, int TN>
+__global__ void __launch_bounds__(256) dgemm_kernel(GemmD g)
+{
+    constexpr int WTM = TM / 2, WTN = TN / 4, MT = WTM / 8, NT = WTN / 8;
+    constexpr int EA = TM / 16, EB = TN / 16;  // elements per thread of an A / B step tile
+    const int z = blockIdx.z;
+    const bool last = z == (int)gridDim.z - 1;
+    const int M = last ? g.M_last : g.M, N = g.N, K = last ? g.K_last : g.K;
+    const double *A = g.A + z * g.sA, *B = g.B + z * g.sB;
+    double *C = g.C + z * g.sC;
+    const int i0 = blockIdx.y * TM, j0 = blockIdx.x * TN;
+    if (i0 >= M) return;
+    if ((g.flags & kLowerOut) && j0 > i0 + TM - 1) return;
     int k_lo = 0, k_hi = K;
-    if (flags & kLowerB) k_lo = j0;                          // B'[k][j] = 0 for k < j
-    if (flags & kLowerA) k_hi = min(K, i0 + GT);             // A[i][k] = 0 for k > i
+    if (g.flags & kLowerB) k_lo = j0;                  // B'[k][j] = 0 for k < j
+    if (g.flags & kLowerA) k_hi = min(K, i0 + TM);     // A[i][k] = 0 for k > i
     k_lo = (k_lo / GK) * GK;
-    __shared__ double As[GK][GT + 2];
-    __shared__ double Bs[GK][GT + 2];
-    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-    double acc[R][R];
+    __shared__ double As[GK][TM + 8];
+    __shared__ double Bs[GK][TN + 8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int wm = warp >> 2, wn = warp & 3;
+    double acc[MT][NT][2];
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+    for (int a = 0; a < MT; ++a)
 #pragma unroll
-        for (int c = 0; c < R; ++c) acc[r][c] = 0.0;
-    // tile loads: A rows (i0 + lr, k0 + lk .. + R-1), one R-wide strip per thread
-    const int lr = tid / (GK / R), lk = (tid % (GK / R)) * R;
-    double ra[R], rb[R];
+        for (int b = 0; b < NT; ++b) acc[a][b][0] = acc[a][b][1] = 0.0;
+    // step tiles: A rows (i0 + lr, k0 + lk .. + EA-1) per thread; B likewise
+    const int lr = tid / (GK / EA), lk = (tid % (GK / EA)) * EA;
+    const int br = tid / (GK / EB), bk = (tid % (GK / EB)) * EB;
+    double ra[EA], rb[EB];
     auto fetch = [&](int k0) {
 #pragma unroll
-        for (int u = 0; u < R; ++u) {
+        for (int u = 0; u < EA; ++u) {
             const int i = i0 + lr, k = k0 + lk + u;
-            ra[u] = (i < M && k < k_hi) ? A[(int64_t)i * lda + k] : 0.0;
+            ra[u] = (i < M && k < k_hi) ? A[(int64_t)i * g.lda + k] : 0.0;
         }
         if (B_KMAJOR) {
 #pragma unroll
-            for (int u = 0; u < R; ++u) {
-                const int j = j0 + lr, k = k0 + lk + u;
-                rb[u] = (j < N && k < k_hi) ? B[(int64_t)j * ldb + k] : 0.0;
+            for (int u = 0; u < EB; ++u) {
+                const int j = j0 + br, k = k0 + bk + u;
+                rb[u] = (j < N && k < k_hi) ? B[(int64_t)j * g.ldb + k] : 0.0;
             }
         } else {
-            // B rows k0 + (tid >> 4), columns j0 + (tid & 15) * R .. + R-1
-            const int k = k0 + (tid >> 4), jb = j0 + (tid & 15) * R;
+            // B rows k0 + (tid >> 4), columns j0 + (tid & 15) * EB .. + EB-1
+            const int k = k0 + (tid >> 4), jb = j0 + (tid & 15) * EB;
 #pragma unroll
-            for (int u = 0; u < R; ++u)
-                rb[u] = (k < k_hi && jb + u < N) ? B[(int64_t)k * ldb + jb + u] : 0.0;
+            for (int u = 0; u < EB; ++u)
+                rb[u] = (k < k_hi && jb + u < N) ? B[(int64_t)k * g.ldb + jb + u] : 0.0;
         }
     };
     auto stash = [&]() {
 #pragma unroll
-        for (int u = 0; u < R; ++u) As[lk + u][lr] = ra[u];
+        for (int u = 0; u < EA; ++u) As[lk + u][lr] = ra[u];
         if (B_KMAJOR) {
 #pragma unroll
-            for (int u = 0; u < R; ++u) Bs[lk + u][lr] = rb[u];
+            for (int u = 0; u < EB; ++u) Bs[bk + u][br] = rb[u];
         } else {
 #pragma unroll
-            for (int u = 0; u < R; ++u) Bs[tid >> 4][(tid & 15) * R + u] = rb[u];
+            for (int u = 0; u < EB; ++u) Bs[tid >> 4][(tid & 15) * EB + u] = rb[u];
         }
     };
+    // fragment coordinates: A (8 x 4) row lane/4, column lane%4; B (4 x 8)
+    // row lane%4, column lane/4; C (8 x 8) row lane/4, columns 2 (lane%4) + e
+    const int fr = lane >> 2, fk = lane & 3;
     if (k_lo < k_hi) fetch(k_lo);
     for (int k0 = k_lo; k0 < k_hi; k0 += GK) {
         stash();
         __syncthreads();
         if (k0 + GK < k_hi) fetch(k0 + GK);  // in flight while this step is consumed
 #pragma unroll
-        for (int kk = 0; kk < GK; ++kk) {
-            double a[R], b[R];
+        for (int kk = 0; kk < GK; kk += 4) {
+            double af[MT], bf[NT];
 #pragma unroll
-            for (int r = 0; r < R; ++r) a[r] = As[kk][ty + 16 * r];
+            for (int a = 0; a < MT; ++a) af[a] = As[kk + fk][wm * WTM + a * 8 + fr];
 #pragma unroll
-            for (int c = 0; c < R; ++c) b[c] = Bs[kk][tx + 16 * c];
+            for (int b = 0; b < NT; ++b) bf[b] = Bs[kk + fk][wn * WTN + b * 8 + fr];
 #pragma unroll
-            for (int r = 0; r < R; ++r)
+            for (int a = 0; a < MT; ++a)
 #pragma unroll
-                for (int c = 0; c < R; ++c) acc[r][c] = fma(a[r], b[c], acc[r][c]);
+                for (int b = 0; b < NT; ++b) dmma(acc[a][b], af[a], bf[b]);
         }
         __syncthreads();
     }
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+    for (int a = 0; a < MT; ++a)
 #pragma unroll
-        for (int c = 0; c < R; ++c) {
-            const int i = i0 + ty + 16 * r, j = j0 + tx + 16 * c;
-            if (i >= M || j >= N) continue;
-            if ((flags & kLowerOut) && j > i) continue;
-            double *o = C + (int64_t)i * ldc + j;
-            *o = beta == 0.0 ? alpha * acc[r][c] : fma(alpha, acc[r][c], beta * *o);
-        }
+        for (int b = 0; b < NT; ++b)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int i = i0 + wm * WTM + a * 8 + fr, j = j0 + wn * WTN + b * 8 + 2 * fk + e;
+                if (i >= M || j >= N) continue;
+                if ((g.flags & kLowerOut) && j > i) continue;
+                double *o = C + (int64_t)i * g.ldc + j;
+                *o = g.beta == 0.0 ? g.alpha * acc[a][b][e] : fma(g.alpha, acc[a][b][e], g.beta * *o);
+            }
 }
 
 namespace {
-template <int R>
-cudaError_t dgemm_r(int M, int N, int K, const double *A, int64_t lda, const double *B, int64_t ldb, bool b_kmajor,
-                    double *C, int64_t ldc, double alpha, double beta, int flags, cudaStream_t stream)
+template <int TM, int TN>
+cudaError_t dgemm_t(const GemmD &g, bool b_kmajor, int nz, cudaStream_t stream)
 {
-    if (M <= 0 || N <= 0) return cudaSuccess;
-    constexpr int GT = 16 * R;
-    const dim3 grid((unsigned)((N + GT - 1) / GT), (unsigned)((M + GT - 1) / GT));
+    const int Mmax = max(g.M, g.M_last);
+    if (Mmax <= 0 || g.N <= 0 || nz <= 0) return cudaSuccess;
+    const dim3 grid((unsigned)((g.N + TN - 1) / TN), (unsigned)((Mmax + TM - 1) / TM), (unsigned)nz);
     if (b_kmajor)
-        dgemm_kernel<true, R><<<grid, 256, 0, stream>>>(M, N, K, A, lda, B, ldb, C, ldc, alpha, beta, flags);
+        dgemm_kernel<true, TM, TN><<<grid, 256, 0, stream>>>(g);
     else
-        dgemm_kernel<false, R><<<grid, 256, 0, stream>>>(M, N, K, A, lda, B, ldb, C, ldc, alpha, beta, flags);
+        dgemm_kernel<false, TM, TN><<<grid, 256, 0, stream>>>(g);
     return cudaGetLastError();
 }
 
-// 128 x 128 tiles where the output fills enough of them, 64 x 64 otherwise
+// 128 x 128 tiles where the outputs fill enough of them, 64 x 64 otherwise
+cudaError_t dgemm_batched(const GemmD &g, bool b_kmajor, int nz, cudaStream_t stream)
+{
+    const int64_t big = (int64_t)nz * ((g.M + 127) / 128) * ((g.N + 127) / 128);
+    if (big >= 148 && g.N > 64) return dgemm_t<128, 128>(g, b_kmajor, nz, stream);
+    return dgemm_t<64, 64>(g, b_kmajor, nz, stream);
+}
+
 cudaError_t dgemm(int M, int N, int K, const double *A, int64_t lda, const double *B, int64_t ldb, bool b_kmajor,
                   double *C, int64_t ldc, double alpha, double beta, int flags, cudaStream_t stream)
 {
-    const int64_t big = (int64_t)((M + 127) / 128) * ((N + 127) / 128);
-    if (big >= 148 && N > 64)
-        return dgemm_r<8>(M, N, K, A, lda, B, ldb, b_kmajor, C, ldc, alpha, beta, flags, stream);
-    return dgemm_r<4>(M, N, K, A, lda, B, ldb, b_kmajor, C, ldc, alpha, beta, flags, stream);
+    const GemmD g{M, N, K, M, K, A, lda, 0, B, ldb, 0, C, ldc, 0, alpha, beta, flags};
+    return dgemm_batched(g, b_kmajor, 1, stream);
 }
 }  // namespace
 
@@ -313,22 +352,26 @@ __global__ void write_factor_kernel(const double *__restrict__ Y, int64_t n, flo
 }
 
 namespace {
-// Y[i0:i0+len, i0:i0+len] = C[...]^-1 (lower) given the inverses of its
-// 64 x 64 diagonal blocks in Y: split at a multiple of 64 near the middle,
-// invert both halves, then Y21 = -Y22 (C21 Y11) through T.
-cudaError_t trinv_rec(const double *C, double *Y, double *T, int64_t ld, int64_t i0, int64_t len,
-                      cudaStream_t stream)
+// Y = C^-1 (lower, n x n, leading dimension n) given the inverses of C's
+// 64 x 64 diagonal blocks in Y, bottom-up: at block size s every pair of
+// neighbouring blocks [i0, i0+s), [i0+s, min(i0+2s, n)) with i0 a multiple of
+// 2s is merged, Y21 = -Y22 (C21 Y11), all merges of a level in one batched
+// launch per product (T holds C21 Y11, s x s per merge).
+cudaError_t trinv_levels(const double *C, double *Y, double *T, int64_t n, cudaStream_t stream)
 {
-    if (len <= NB) return cudaSuccess;
-    const int64_t h = ((len + 2 * NB - 1) / (2 * NB)) * NB;
-    cudaError_t e = trinv_rec(C, Y, T, ld, i0, h, stream);
-    if (e == cudaSuccess) e = trinv_rec(C, Y, T, ld, i0 + h, len - h, stream);
-    if (e != cudaSuccess) return e;
-    const int m2 = (int)(len - h), m1 = (int)h;
-    e = dgemm(m2, m1, m1, C + (i0 + h) * ld + i0, ld, Y + i0 * ld + i0, ld, false, T, m1, 1.0, 0.0, kLowerB, stream);
-    if (e != cudaSuccess) return e;
-    return dgemm(m2, m1, m2, Y + (i0 + h) * ld + (i0 + h), ld, T, m1, false, Y + (i0 + h) * ld + i0, ld, -1.0, 0.0,
-                 kLowerA, stream);
+    for (int64_t s = NB; s < n; s *= 2) {
+        const int nz = (int)((n - s + 2 * s - 1) / (2 * s));
+        const int m2_last = (int)min64(s, n - ((int64_t)(nz - 1) * 2 * s + s));
+        const int64_t step = 2 * s * (n + 1);  // from one merge's block to the next
+        const int si = (int)s;
+        const GemmD g1{si, si, si, m2_last, si, C + s * n, n, step, Y, n, step, T, s, s * s, 1.0, 0.0, kLowerB};
+        cudaError_t e = dgemm_batched(g1, false, nz, stream);
+        if (e != cudaSuccess) return e;
+        const GemmD g2{si, si, si, m2_last, m2_last, Y + s * n + s, n, step, T, s, s * s, Y + s * n, n, step,
+                       -1.0, 0.0, kLowerA};
+        if ((e = dgemm_batched(g2, false, nz, stream)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 }  // namespace
 
@@ -361,7 +404,7 @@ cudaError_t launch_factor(const float *A, int64_t n, float *L, double *work, Dev
         }
     }
     // Y = C^-1 from the diagonal blocks' inverses
-    if ((e = trinv_rec(C, Y, T, n, 0, n, stream)) != cudaSuccess) return e;
+    if ((e = trinv_levels(C, Y, T, n, stream)) != cudaSuccess) return e;
     write_factor_kernel<<<g, 256, 0, stream>>>(Y, n, L);
     return cudaGetLastError();
 }
