@@ -37,8 +37,8 @@ LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 25
 # DRAM traffic of the band products from an ncu capture of one solve's 93
 # band launches (profiles/band_4096_dram.md); reported only while the band
 # kernel sources hash to the value the capture was taken with.
-BAND_TRAFFIC = {"sources_sha256": "bc8092fab082e3f7ffb530ebb380485e36c365dbbbf01ecb766ddcc6db7e5967",
-                "bytes_per_launch": 35.27e6, "profile": "profiles/band_4096_dram.md"}
+BAND_TRAFFIC = {"sources_sha256": "c8a98f27876dc4766db47327de718f4a109755d7c42c85a2c6f85990ab2d3051",
+                "bytes_per_launch": 35.06e6, "profile": "profiles/band_4096_dram.md"}
 BAND_SOURCES = ("two_sided_gptq_b200/csrc/band_tc.cu", "two_sided_gptq_b200/csrc/band_fused.cu",
                 "two_sided_gptq_b200/csrc/tcgen05.cuh", "two_sided_gptq_b200/csrc/common.cuh",
                 "two_sided_gptq_b200/csrc/kernels.cuh")
@@ -410,6 +410,29 @@ def extra_measurements(args, bk, w, Wd, LA, LB, W, codes, ws, stream, dev, dist,
     return e2e_ms, batch_ms, one_ms
 
 
+def proxy_loss_timing(bk, Wd, V, Ad, Bd, stream, dist, dev):
+    """bakron_proxy_loss of the solve's V (its result is copied to the host,
+    so each call ends synchronised): value and ms per call (CUDA events on the
+    stream, median of five after one warm-up), max over ranks."""
+    import torch
+
+    m, n = Wd.shape
+    value = bk.proxy_loss(Wd, V, Ad, Bd, stream=stream)
+    times = []
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        bk.proxy_loss(Wd, V, Ad, Bd, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = max_over_ranks(statistics.median(times), dist, dev)
+    flops = 2.0 * m * n * (m + n)
+    return {"value": value, "ms": ms, "flops": flops, "tflops": flops / (ms / 1e3) / 1e12,
+            "note": "tr((W-V)^T B (W-V) A): FP32 CUDA-core products B(W-V) and (W-V)A per 64 x 64 tile, "
+                    "FP64 fixed-order reduction; outside the metric"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -519,6 +542,7 @@ def main():
     if not args.no_extras:
         e2e_ms, batch_ms, one_ms = extra_measurements(args, bk, w, Wd, LA, LB, W, codes, ws, stream, dev, dist,
                                                       leaf, fw, n_batch)
+    loss = proxy_loss_timing(bk, Wd, V, Ad, Bd, stream, dist, dev)
 
     line = None
     if rank == 0:
@@ -555,6 +579,7 @@ def main():
                      "share_of_profiled_step": pr["leaf_ms"] / pr["total_ms"]},
             "profile_ms": pr,
             "factor_ms": factor_ms,
+            "proxy_loss": loss,
             "factor": {"ms": factor_ms, "flops": factor_flops(n) + factor_flops(m),
                        "fp64_tflops": (factor_flops(n) + factor_flops(m)) / (factor_ms / 1e3) / 1e12,
                        "fp64_peak_tflops_nominal": FP64_PEAK_NOMINAL,

@@ -281,9 +281,14 @@ size_t bakron_solve_host_workspace_size(int64_t m, int64_t n, const bakron_confi
 
 /* bakron_solve on HOST buffers: copies W_host, LA_host, LB_host to device
  * staging inside ws_dev, solves, and copies V, codes and scales back, all
- * enqueued on `stream` (pinned host memory makes the copies asynchronous;
- * the results are valid after the stream is synchronised).  q->row_scale,
- * if not NULL, is a HOST pointer here. */
+ * ordered on `stream` (pinned host memory makes the copies asynchronous;
+ * the results are valid after the stream is synchronised).  In the
+ * two-sided solve each 128-row block of V and codes is copied back as soon
+ * as the tile diagonal that completes it has been rounded, on a copy stream
+ * of the library's own that `stream` waits for at the end, so those copies
+ * overlap the rest of the solve; the launches are then always direct
+ * (cfg->use_graph is ignored).  q->row_scale, if not NULL, is a HOST pointer
+ * here. */
 bakron_status_t bakron_solve_host(const float *W_host, int64_t m, int64_t n, const float *LA_host,
                                   const float *LB_host, const bakron_quantizer_t *q, float *V_host,
                                   int8_t *codes_host, float *scales_host, void *ws_dev,
@@ -335,18 +340,23 @@ bakron_status_t bakron_solve_noalloc(const float *W_dev, int64_t m, int64_t n, c
                                      bakron_stream_t stream, int32_t *device_status_host);
 
 /* ------------------------------------------------------------ proxy loss */
-/* Bytes of workspace bakron_proxy_loss needs: the status block plus one FP64
- * partial sum per 64 x 64 tile of W. */
+/* Bytes of workspace bakron_proxy_loss needs: the status block, TF32 hi / lo
+ * parts of W - V (both orientations), A and B padded to whole 128 x 128
+ * tiles, the two products (fp32) and 592 FP64 partial sums; about
+ * 4 (6 Mp Np + 2 Mp^2 + 2 Np^2) bytes, Mp, Np = m, n rounded up to 128. */
 size_t bakron_proxy_loss_workspace_size(int64_t m, int64_t n);
 
 /* Proxy loss l = tr((W-V)^T B (W-V) A) = ||B^{1/2}(V-W)A^{1/2}||_F^2
  * (Corollary 3.4's distortion; the review's "||vec(W)-vec(V)||_H^2",
- * H = A (x) B).  W_dev, V_dev m x n; A_dev n x n; B_dev m x m (symmetric).
- * Products in FP32 on the GPU, reduction in FP64: each 64 x 64 tile's sum
- * goes to its own slot in the workspace and the slots are added in a fixed
- * order, so repeated calls give bit-identical results.  The result is
+ * H = A (x) B).  W_dev, V_dev m x n; A_dev n x n (symmetric: its rows serve as
+ * the columns of A); B_dev m x m.  Computed as sum_ij (B E)_ij (E A)_ij,
+ * E = W - V: both products on the tensor cores in 3xTF32 (about FP32
+ * accuracy), the elementwise products and their sum in FP64, each of 592
+ * fixed shares of the entries summed in index order and the shares added in
+ * index order, so repeated calls give bit-identical results.  The result is
  * written to *out_dev (a device double) and, if out_host is not NULL, also
- * to *out_host, in which case the call synchronises `stream`. */
+ * to *out_host, in which case the call synchronises `stream`.  The
+ * workspace must be 1024-byte aligned. */
 bakron_status_t bakron_proxy_loss(const float *W_dev, const float *V_dev, const float *A_dev,
                                   const float *B_dev, int64_t m, int64_t n, double *out_dev,
                                   double *out_host, void *ws_dev, size_t ws_bytes,

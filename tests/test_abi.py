@@ -53,8 +53,11 @@ def test_host_only_queries(lib):
     assert ws >= 4 * (5 * 4096 * 4096 + 6 * 4096 * 4096)
     assert lib.bakron_solve_host_workspace_size(100, 70, None) > lib.bakron_solve_workspace_size(100, 70, None)
     assert lib.bakron_factor_workspace_size(300, 200) >= 2 * 300 * 300 * 8
-    assert lib.bakron_proxy_loss_workspace_size(3, 4) == 1024 + 8  # status block (aligned) + one tile sum
-    assert lib.bakron_proxy_loss_workspace_size(4096, 4096) == 1024 + 8 * 64 * 64
+    # status block; E, E^T, B, A hi / lo and the two products, each padded to
+    # 128-multiples; 592 FP64 partial sums (1024-byte aligned)
+    assert lib.bakron_proxy_loss_workspace_size(3, 4) == 1024 + 10 * 128 * 128 * 4 + 5120
+    assert lib.bakron_proxy_loss_workspace_size(4096, 4096) == 1024 + 10 * 4096 * 4096 * 4 + 5120
+    assert lib.bakron_proxy_loss_workspace_size(200, 300) == 1024 + (6 * 256 * 384 + 2 * 256 * 256 + 2 * 384 * 384) * 4 + 5120
     bad = _native.Config(64, 0, 0, 0, None)  # unsupported tile
     assert lib.bakron_solve_workspace_size(10, 10, ctypes.byref(bad)) == 0
 

@@ -125,9 +125,17 @@ def test_solve_device_errors(bk):
     bk.solve(_t(W), _t(LA), _t(LB))
 
 
-@pytest.mark.parametrize("name", ["tiny", "mid"])
+@pytest.mark.parametrize("name", ["tiny", "mid", (200, 333), (129, 1), (1, 130),
+                                  pytest.param("bench", marks=pytest.mark.slow)])
 def test_proxy_loss_matches_oracle(bk, name):
-    W, A, B = workloads.generate(name)
+    """bakron_proxy_loss (both products on the tensor cores in 3xTF32, FP64
+    dot) against the oracle's FP64 tr((W-V)^T B (W-V) A); ragged shapes pad
+    every operand to whole tiles with zeros."""
+    if isinstance(name, tuple):
+        m, n = name
+        W, A, B = workloads.random_problem(m, n, seed=m + n)
+    else:
+        W, A, B = workloads.generate(name)
     LA = oracle.factor(A).astype(np.float32)
     LB = oracle.factor(B).astype(np.float32)
     Wd = _t(W)

@@ -84,6 +84,37 @@ struct Profiler {
     }
 };
 thread_local Profiler t_prof;
+
+// Host-buffer solves: the rows of V and codes go back to the host as soon as
+// the tile diagonal that completes them has been rounded (row block I is
+// final after tile diagonal I + Nt - 1), on a copy stream that follows the
+// solve's stream through one event, so the device-to-host copies of all but
+// the last row block overlap the rest of the solve.
+struct RowCopy {
+    cudaStream_t cs = nullptr;
+    cudaEvent_t ev = nullptr;
+    float *V_host = nullptr;
+    int8_t *codes_host = nullptr;
+    const float *V_dev = nullptr;
+    const int8_t *codes_dev = nullptr;
+    int64_t m = 0, n = 0;
+    int Mt = 0, Nt = 0, next_block = 0;
+    bool failed = false;
+    // copy the row blocks completed by tile diagonals <= k (issued on `main`)
+    void upto_diagonal(int k, cudaStream_t main)
+    {
+        const int last = std::min(k - (Nt - 1), Mt - 1);
+        if (failed || last < next_block) return;
+        const int64_t r0 = (int64_t)next_block * kTile, r1 = std::min<int64_t>((int64_t)(last + 1) * kTile, m);
+        failed = cudaEventRecord(ev, main) != cudaSuccess || cudaStreamWaitEvent(cs, ev, 0) != cudaSuccess ||
+                 cudaMemcpyAsync(V_host + r0 * n, V_dev + r0 * n, (size_t)(r1 - r0) * n * sizeof(float),
+                                 cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+                 cudaMemcpyAsync(codes_host + r0 * n, codes_dev + r0 * n, (size_t)(r1 - r0) * n,
+                                 cudaMemcpyDeviceToHost, cs) != cudaSuccess;
+        next_block = last + 1;
+    }
+};
+thread_local RowCopy *t_rowcopy = nullptr;
 thread_local bakron_profile_t t_last_profile = {};
 thread_local std::vector<bakron_profile_launch_t> t_last_launches;
 
@@ -235,6 +266,7 @@ cudaError_t run_schedule(SolveCtx &c, int k, int l)
         cudaError_t e = launch_leaf(c.leaf, k, c.leaf_variant == kPairVariant ? kPairVariant - 1 : c.leaf_variant,
                                     c.stream);
         t_prof.end();
+        if (t_rowcopy && e == cudaSuccess) t_rowcopy->upto_diagonal(k, c.stream);
         return e;
     }
     if (l == 2 && c.leaf_variant == kPairVariant) {
@@ -243,6 +275,7 @@ cudaError_t run_schedule(SolveCtx &c, int k, int l)
         t_prof.begin(1, NodeParams{k, 1, 2, c.leaf.Mt, c.leaf.Nt});
         cudaError_t e = launch_leaf_pair(c.leaf, k, c.pair_slot++, c.stream);
         t_prof.end();
+        if (t_rowcopy && e == cudaSuccess) t_rowcopy->upto_diagonal(k + 1, c.stream);
         return e;
     }
     const int h = l / 2;
@@ -786,16 +819,55 @@ bakron_status_t bakron_solve_host(const float *W_host, int64_t m, int64_t n, con
         if (!h2d(H.uscales, q->row_scale, (size_t)m * 4)) return BAKRON_ERR_CUDA;
         qd.row_scale = (const float *)(w + H.uscales);
     }
+    if (one_sided) {
+        // rows are final only at the end of the column-block recursion
+        bakron_status_t r = solve_device((const float *)(w + H.W), m, n, (const float *)(w + H.LA),
+                                         (const float *)(w + H.LB), &qd, (float *)(w + H.V),
+                                         (int8_t *)(w + H.codes), (float *)(w + H.scales), w + H.solve, sb,
+                                         cfg, s, true);
+        if (r != BAKRON_OK) return r;
+        if (cudaMemcpyAsync(V_host, w + H.V, (size_t)m * n * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaMemcpyAsync(codes_host, w + H.codes, (size_t)m * n, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaMemcpyAsync(scales_host, w + H.scales, (size_t)m * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return BAKRON_ERR_CUDA;
+        return BAKRON_OK;
+    }
+    // two-sided: row blocks stream back during the solve (direct launches)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BAKRON_ERR_CUDA;
+    thread_local cudaStream_t copy_stream[64] = {};
+    thread_local cudaEvent_t copy_event[64] = {};
+    if (!copy_stream[dev] && cudaStreamCreateWithFlags(&copy_stream[dev], cudaStreamNonBlocking) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
+    if (!copy_event[dev] && cudaEventCreateWithFlags(&copy_event[dev], cudaEventDisableTiming) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
+    RowCopy rc;
+    rc.cs = copy_stream[dev];
+    rc.ev = copy_event[dev];
+    rc.V_host = V_host;
+    rc.codes_host = codes_host;
+    rc.V_dev = (const float *)(w + H.V);
+    rc.codes_dev = (const int8_t *)(w + H.codes);
+    rc.m = m;
+    rc.n = n;
+    rc.Mt = (int)((m + kTile - 1) / kTile);
+    rc.Nt = (int)((n + kTile - 1) / kTile);
+    t_rowcopy = &rc;
     bakron_status_t r = solve_device((const float *)(w + H.W), m, n, (const float *)(w + H.LA),
                                      (const float *)(w + H.LB), &qd, (float *)(w + H.V),
                                      (int8_t *)(w + H.codes), (float *)(w + H.scales), w + H.solve, sb,
-                                     cfg, s, true);
-    if (r != BAKRON_OK) return r;
-    if (cudaMemcpyAsync(V_host, w + H.V, (size_t)m * n * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(codes_host, w + H.codes, (size_t)m * n, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(scales_host, w + H.scales, (size_t)m * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+                                     cfg, s, true, true);
+    t_rowcopy = nullptr;
+    // whatever was issued, `s` ends after the copy stream's work: the rows not
+    // yet copied and the steps follow the last kernel
+    rc.upto_diagonal(rc.Mt + rc.Nt - 2, s);
+    const bool ok = !rc.failed && r == BAKRON_OK &&
+                    cudaMemcpyAsync(scales_host, w + H.scales, (size_t)m * 4, cudaMemcpyDeviceToHost, rc.cs) ==
+                        cudaSuccess;
+    if (cudaEventRecord(rc.ev, rc.cs) != cudaSuccess || cudaStreamWaitEvent(s, rc.ev, 0) != cudaSuccess)
         return BAKRON_ERR_CUDA;
-    return BAKRON_OK;
+    if (r != BAKRON_OK) return r;
+    return ok ? BAKRON_OK : BAKRON_ERR_CUDA;
 }
 
 size_t bakron_factor_workspace_size(int64_t n, int64_t m)
@@ -829,7 +901,9 @@ bakron_status_t bakron_factor(const float *A_dev, int64_t n, const float *B_dev,
 size_t bakron_proxy_loss_workspace_size(int64_t m, int64_t n)
 {
     if (m < 1 || n < 1 || m > kMaxSide || n > kMaxSide) return 0;
-    return align_up(kStatusBytes) + (size_t)proxy_loss_parts(m, n) * sizeof(double);
+    ProxyLayout L;
+    L.compute(m, n);
+    return L.total;
 }
 
 bakron_status_t bakron_proxy_loss(const float *W_dev, const float *V_dev, const float *A_dev,
@@ -840,13 +914,16 @@ bakron_status_t bakron_proxy_loss(const float *W_dev, const float *V_dev, const 
     if (m < 1 || n < 1 || m > kMaxSide || n > kMaxSide) return BAKRON_ERR_INVALID_ARG;
     if (!W_dev || !V_dev || !A_dev || !B_dev || !out_dev) return BAKRON_ERR_INVALID_ARG;
     if (!ws_dev || ws_bytes < bakron_proxy_loss_workspace_size(m, n)) return BAKRON_ERR_WORKSPACE;
-    if (!aligned16(W_dev) || !aligned16(V_dev) || !aligned16(A_dev) || !aligned16(B_dev) || !aligned16(ws_dev) ||
-        ((uintptr_t)out_dev & 7u))
+    if (!aligned16(W_dev) || !aligned16(V_dev) || !aligned16(A_dev) || !aligned16(B_dev) ||
+        ((uintptr_t)ws_dev & (kAlign - 1)) || ((uintptr_t)out_dev & 7u))
         return BAKRON_ERR_ALIGNMENT;
+    if (configure_device() != cudaSuccess) return BAKRON_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
+    ProxyLayout L;
+    L.compute(m, n);
     if (cudaMemsetAsync(ws_dev, 0, kStatusBytes, s) != cudaSuccess) return BAKRON_ERR_CUDA;
-    double *part = (double *)((char *)ws_dev + align_up(kStatusBytes));
-    if (launch_proxy_loss(W_dev, V_dev, A_dev, B_dev, m, n, out_dev, part, s) != cudaSuccess) return BAKRON_ERR_CUDA;
+    if (launch_proxy_loss(W_dev, V_dev, A_dev, B_dev, L, (char *)ws_dev, out_dev, s) != cudaSuccess)
+        return BAKRON_ERR_CUDA;
     if (out_host) {
         if (cudaMemcpyAsync(out_host, out_dev, sizeof(double), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
             cudaStreamSynchronize(s) != cudaSuccess)

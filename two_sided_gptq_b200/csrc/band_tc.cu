@@ -49,11 +49,13 @@ template <int STAGE>
 __global__ void __launch_bounds__(kThreads, 1)
 band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
 {
-    // STAGE 1, 2: the band products; 3: Gram tiles; 4: the one-sided update
+    // STAGE 1, 2: the band products; 3: Gram tiles; 4: the one-sided update;
+    // 5: full GEMM tiles (the proxy loss's products)
     const Item it = STAGE == 1   ? stage1_item(np, blockIdx.x, blockIdx.y)
                     : STAGE == 2 ? stage2_item(np, blockIdx.x, blockIdx.y)
                     : STAGE == 3 ? gram_item(np, blockIdx.x, blockIdx.y)
-                                 : gptq_item(np, blockIdx.x, blockIdx.y);
+                    : STAGE == 4 ? gptq_item(np, blockIdx.x, blockIdx.y)
+                                 : full_item(np, blockIdx.x, blockIdx.y);
     if (!it.valid) return;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -348,6 +350,8 @@ cudaError_t band_tc_configure()
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(band_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(band_tc_kernel<5>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(band_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
 }
 
@@ -391,6 +395,25 @@ cudaError_t launch_band_abort_selftest(DeviceStatus *st, float *buf, int timeout
     if (!make_tc_maps(1, 2, 2, g, &maps)) return cudaErrorInvalidValue;
     const NodeParams np{0, 1, 2, 2, 2};
     return launch_band_tc(1, np, g, maps, stream);
+}
+
+// Full GEMM D (Mo x No) = A (Mo x K) B (No x K)^T, operands as TF32 hi / lo
+// parts, K-major with row stride K; D stored with row stride No.  All sizes
+// multiples of the tile.
+bool make_full_maps(const float *a_hi, const float *a_lo, const float *b_hi, const float *b_lo, float *D, int64_t Mo,
+                    int64_t No, int64_t K, TcMaps *m)
+{
+    return make_map(&m->a_hi, a_hi, Mo, K, K) && make_map(&m->a_lo, a_lo, Mo, K, K) &&
+           make_map(&m->b_hi, b_hi, No, K, K) && make_map(&m->b_lo, b_lo, No, K, K) &&
+           make_map(&m->o0, D, Mo, No, No, 32) && make_map(&m->o1, D, Mo, No, No, 32);
+}
+
+cudaError_t launch_full_tc(int64_t Mo, int64_t No, int64_t K, const GemmArgs &g, const TcMaps &maps,
+                           cudaStream_t stream)
+{
+    const NodeParams np{0, 0, (int)(K / T), (int)(Mo / T), (int)(No / T)};
+    return launch_pdl(band_tc_kernel<5>, dim3((unsigned)np.Nt, (unsigned)np.Mt), dim3(kThreads), kSmem, stream, maps,
+                      np, g);
 }
 
 cudaError_t launch_gram_tc(const NodeParams &np, const GemmArgs &g, const TcMaps &maps, cudaStream_t stream)

@@ -186,4 +186,13 @@ __host__ __device__ inline Item gram_item(const NodeParams &p, int J, int I)
     return it;
 }
 
+// Full GEMM tile (I, J) of D = A B^T: A rows = output rows (p.Mt tiles),
+// B rows = output columns (p.Nt tiles), contraction over p.l tiles of K.
+// Grid: x = J, y = I.
+__host__ __device__ inline Item full_item(const NodeParams &p, int J, int I)
+{
+    Item it{I, J, 0, p.l, I < p.Mt && J < p.Nt && p.l > 0};
+    return it;
+}
+
 }  // namespace bakron

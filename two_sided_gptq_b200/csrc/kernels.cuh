@@ -86,11 +86,21 @@ cudaError_t launch_gram_prep(const float *X, int64_t N, int64_t d, int64_t Dp, i
 cudaError_t launch_gram_finish(const float *G, int64_t d, int64_t Dp, int64_t N, float damping, float *A,
                                cudaStream_t stream);
 
-// Proxy loss (FP32 products, FP64 reduction) into *out (device double);
-// `part` holds proxy_loss_parts(m, n) doubles (per-tile partial sums).
-int64_t proxy_loss_parts(int64_t m, int64_t n);
-cudaError_t launch_proxy_loss(const float *W, const float *V, const float *A, const float *B,
-                              int64_t m, int64_t n, double *out, double *part, cudaStream_t stream);
+// Full GEMM tiles on the tensor cores (band_tc.cu, stage 5): D = A B^T.
+bool make_full_maps(const float *a_hi, const float *a_lo, const float *b_hi, const float *b_lo, float *D, int64_t Mo,
+                    int64_t No, int64_t K, TcMaps *m);
+cudaError_t launch_full_tc(int64_t Mo, int64_t No, int64_t K, const GemmArgs &g, const TcMaps &maps,
+                           cudaStream_t stream);
+
+// Proxy loss tr((W-V)^T B (W-V) A) (proxy_loss.cu): the two products on the
+// tensor cores in 3xTF32, the elementwise dot in FP64 with a fixed order.
+struct ProxyLayout {
+    int64_t m, n, Mp, Np;
+    size_t status, Ehi, Elo, EThi, ETlo, Bhi, Blo, Ahi, Alo, P, Q, parts, total;
+    void compute(int64_t m_, int64_t n_);
+};
+cudaError_t launch_proxy_loss(const float *W, const float *V, const float *A, const float *B, const ProxyLayout &L,
+                              char *ws, double *out, cudaStream_t stream);
 
 // FP64 factorisation: L (n x n, fp32) = chol(A^{-1}); work holds
 // factor_work_doubles(n) doubles.
