@@ -167,8 +167,62 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
         ((float4 *)sDt)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int idx = tid; idx < 2 * S3 * WSC / 4; idx += kThreadsC)  // O_S, O_U
         ((float4 *)sOS)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
-    __syncthreads();  // R is zero before the first staged block lands in it
-    pdl_wait();       // every global input (Wt, factors, steps) comes from earlier kernels
+    // The factors and the steps come from the preparation kernel at the start
+    // of the solve, which has completed before this kernel's predecessor
+    // passed its own dependency wait: they are read before this kernel's
+    // wait, overlapping the predecessor's tail.  Only Wt (and the pair form's
+    // neighbour data) depend on the predecessor.
+    if (pp > 0) {  // LtB[p, 0:p], fixed for the kernel
+        const int ld = S3 * pp + 4, c4 = 8 * pp;
+        for (int c = tid; c < S3 * c4; c += kThreadsC) {
+            const int i = c / c4, k4 = c - i * c4;
+            cp_async16(sLBs + i * ld + 4 * k4, LBt + (pp * S3 + i) * ldb_g + 4 * k4);
+        }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (tid < S3) sLBd[tid] = tid > 0 ? LBt[(pp * S3 + tid) * ldb_g + pp * S3 + tid - 1] : 0.f;
+    const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
+    const int role = warp;  // 0 entries, 1 row side, 2 column side, 3 (overlapped form) older products
+    // column-side warp: its LtB[p,p] row rho (columns <= rho-2), fixed for the kernel
+    float2 lbr[S3 / 2];
+    if (role == 2) {
+#pragma unroll
+        for (int c = 0; c < S3 / 2; ++c) {
+            float2 v = *(const float2 *)(LBt + (pp * S3 + lane) * ldb_g + pp * S3 + 2 * c);
+            v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
+            v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
+            lbr[c] = v;
+        }
+    }
+    // Steps of this row block and their correctly rounded reciprocals; a step
+    // outside [2^-60, 2^60] switches the row block to the IEEE division (both
+    // give the correctly rounded quotient, so the choice never shows).
+    bool out_of_range = false;
+    if (tid < S3) {
+        const float s = tid < mrb ? p.scales[brow0 + tid] : 1.f;
+        scale[tid] = s;
+        rcp[tid] = __frcp_rn(s);
+        out_of_range = !(s >= 0x1p-60f && s <= 0x1p60f);
+    }
+    // (this barrier also orders the zeroing above before the first staged block)
+    const bool exact_div = __syncthreads_or(out_of_range) != 0;
+
+    // row-side warp: LtA[q,q] row b (used for columns <= b-2, masked when its
+    // sweep starts, so no instruction waits for these loads before then);
+    // entry warp: LtA[b][b-1].  Loaded for the CTA's next sub-tile as soon as
+    // the previous sweep ends, so the L2 latency overlaps the phase change.
+    float2 la[S3 / 2];
+    float la_new = 0.f;
+    auto load_la = [&](int q) {
+        if (q < 0 || q > 3) return;
+        if (role == 1) {
+#pragma unroll
+            for (int c = 0; c < S3 / 2; ++c) la[c] = *(const float2 *)(LAt + (q * S3 + lane) * lda_g + q * S3 + 2 * c);
+        }
+        if (role == 0 && lane > 0) la_new = LAt[(q * S3 + lane) * lda_g + q * S3 + lane - 1];
+    };
+    load_la(0 - pp);
+    pdl_wait();  // Wt comes from the previous kernel
     const bool has_left = kPair && consumer && J >= 1;  // neighbours on the first diagonal
     const bool has_up = kPair && consumer && I >= 1;
     if (kPair && consumer) {
@@ -286,60 +340,24 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
             *(float4 *)(sDr + j * LSC + pr * S3 + 4 * r4) = *(const float4 *)src;
         }
     };
-    stage_subtile(0 - pp, 0, kThreadsC);
-    if (pp > 0) {  // LtB[p, 0:p], fixed for the kernel
-        const int ld = S3 * pp + 4, c4 = 8 * pp;
-        for (int c = tid; c < S3 * c4; c += kThreadsC) {
-            const int i = c / c4, k4 = c - i * c4;
-            cp_async16(sLBs + i * ld + 4 * k4, LBt + (pp * S3 + i) * ldb_g + 4 * k4);
+    // V = s * code and the residual's TF32 split for columns [c0, c1) of this
+    // row block, with threads [t0, t0 + nt)
+    auto write_out = [&](int c0, int c1, int t0, int nt) {
+        const int w = c1 - c0;
+        for (int idx = tid - t0; idx < S3 * w; idx += nt) {
+            const int r = idx / w, c = c0 + idx % w;
+            if (r >= mrb || c >= nc) continue;
+            const int64_t gi = brow0 + r, gj = col0 + c;
+            const int8_t code = sCode[r * T + c];
+            p.codes[gi * p.n + gj] = code;
+            p.V[gi * p.n + gj] = scale[r] * (float)code;
+            float hi, lo;
+            split_tf32(sDt[c * DSC + r], hi, lo);
+            p.Dhi[gi * p.Np + gj] = hi;
+            p.Dlo[gi * p.Np + gj] = lo;
         }
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    if (tid < S3) sLBd[tid] = tid > 0 ? LBt[(pp * S3 + tid) * ldb_g + pp * S3 + tid - 1] : 0.f;
-    const float fqmin = (float)p.qmin, fqmax = (float)p.qmax;
-    const int role = warp;  // 0 entries, 1 row side, 2 column side, 3 (overlapped form) older products
-    // column-side warp: its LtB[p,p] row rho (columns <= rho-2), fixed for the kernel
-    float2 lbr[S3 / 2];
-    if (role == 2) {
-#pragma unroll
-        for (int c = 0; c < S3 / 2; ++c) {
-            float2 v = *(const float2 *)(LBt + (pp * S3 + lane) * ldb_g + pp * S3 + 2 * c);
-            v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
-            v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
-            lbr[c] = v;
-        }
-    }
-    // Steps of this row block and their correctly rounded reciprocals; a step
-    // outside [2^-60, 2^60] switches the row block to the IEEE division (both
-    // give the correctly rounded quotient, so the choice never shows).
-    bool out_of_range = false;
-    if (tid < S3) {
-        const float s = tid < mrb ? p.scales[brow0 + tid] : 1.f;
-        scale[tid] = s;
-        rcp[tid] = __frcp_rn(s);
-        out_of_range = !(s >= 0x1p-60f && s <= 0x1p60f);
-    }
-    const bool exact_div = __syncthreads_or(out_of_range) != 0;
-
-    // row-side warp: LtA[q,q] row b (columns <= b-2); entry warp: LtA[b][b-1].
-    // Loaded for the CTA's next sub-tile as soon as the previous sweep ends, so
-    // the L2 latency overlaps the phase change.
-    float2 la[S3 / 2];
-    float la_new = 0.f;
-    auto load_la = [&](int q) {
-        if (q < 0 || q > 3) return;
-        if (role == 1) {
-#pragma unroll
-            for (int c = 0; c < S3 / 2; ++c) {
-                float2 v = *(const float2 *)(LAt + (q * S3 + lane) * lda_g + q * S3 + 2 * c);
-                v.x = 2 * c + 0 <= lane - 2 ? v.x : 0.f;
-                v.y = 2 * c + 1 <= lane - 2 ? v.y : 0.f;
-                la[c] = v;
-            }
-        }
-        if (role == 0 && lane > 0) la_new = LAt[(q * S3 + lane) * lda_g + q * S3 + lane - 1];
     };
-    load_la(0 - pp);
+    stage_subtile(0 - pp, 0, kThreadsC);
 
     for (int e = 0; e < 7; ++e) {
         const int q = e - pp;
@@ -491,6 +509,11 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
                 // for the entry warp's next entry (a+1, b); column b-1 of that R
                 // row is written during this step, its coefficient here is zero
                 const int b = lane;
+#pragma unroll
+                for (int c = 0; c < S3 / 2; ++c) {
+                    la[c].x = 2 * c + 0 <= b - 2 ? la[c].x : 0.f;
+                    la[c].y = 2 * c + 1 <= b - 2 ? la[c].y : 0.f;
+                }
                 float4 rv[S3 / 4];
 #pragma unroll
                 for (int c = 0; c < S3 / 4; ++c) rv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -555,18 +578,7 @@ leaf_cluster_kernel(LeafArgs p, int K, int I_lo, int slot)
         }
     }
     pdl_trigger();
-    for (int idx = tid; idx < S3 * T; idx += kThreadsC) {  // V = s * code, residual split
-        const int r = idx / T, c = idx % T;
-        if (r >= mrb || c >= nc) continue;
-        const int64_t gi = brow0 + r, gj = col0 + c;
-        const int8_t code = sCode[r * T + c];
-        p.codes[gi * p.n + gj] = code;
-        p.V[gi * p.n + gj] = scale[r] * (float)code;
-        float hi, lo;
-        split_tf32(sDt[c * DSC + r], hi, lo);
-        p.Dhi[gi * p.Np + gj] = hi;
-        p.Dlo[gi * p.Np + gj] = lo;
-    }
+    write_out(0, T, 0, kThreadsC);
     if (kPair && !consumer) {
         // this row block's in-tile R for the right neighbour, then the flag
         // (every thread fences its own writes before the CTA barrier)
