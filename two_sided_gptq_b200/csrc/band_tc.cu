@@ -50,9 +50,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 band_tc_kernel(const __grid_constant__ TcMaps maps, NodeParams np, GemmArgs g)
 {
     // STAGE 1, 2: the band products; 3: Gram tiles; 4: the one-sided update;
-    // 5: full GEMM tiles (the proxy loss's products)
-    const Item it = STAGE == 1   ? stage1_item(np, blockIdx.x, blockIdx.y)
-                    : STAGE == 2 ? stage2_item(np, blockIdx.x, blockIdx.y)
+    // 5: full GEMM tiles (the proxy loss's products).  With np.lpt the band
+    // products run on a (row tile, key offset) grid with the key offset
+    // descending along y: CTAs are dispatched x-fastest, so the items with
+    // the longest contractions (the largest offsets) start first and the
+    // short ones fill the tail of the last wave.
+    const bool lpt = STAGE <= 2 && np.lpt;
+    const int bx = lpt ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.x;
+    const int by = lpt ? (int)blockIdx.x : (int)blockIdx.y;
+    const Item it = STAGE == 1   ? stage1_item(np, bx, by)
+                    : STAGE == 2 ? stage2_item(np, bx, by)
                     : STAGE == 3 ? gram_item(np, blockIdx.x, blockIdx.y)
                     : STAGE == 4 ? gptq_item(np, blockIdx.x, blockIdx.y)
                                  : full_item(np, blockIdx.x, blockIdx.y);
@@ -441,8 +448,15 @@ bool make_tc_maps(int stage, int Mt, int Nt, const GemmArgs &g, TcMaps *maps)
 cudaError_t launch_band_tc(int stage, const NodeParams &np, const GemmArgs &g, const TcMaps &maps,
                            cudaStream_t stream)
 {
-    if (stage == 1) return launch_pdl(band_tc_kernel<1>, dim3(np.l, np.Mt), dim3(kThreads), kSmem, stream, maps, np, g);
-    return launch_pdl(band_tc_kernel<2>, dim3(np.l - np.h, np.Mt), dim3(kThreads), kSmem, stream, maps, np, g);
+    // Longest-first order measured faster for nodes up to 40 tile diagonals
+    // wide (levels 32 and 16 at 4096^2, 36 and 18 at 14336 x 4096) and slower
+    // for the widest, whose row-tile-major order keeps operands in L2.
+    NodeParams q = np;
+    q.lpt = np.l <= 40;
+    const unsigned nx = (unsigned)(stage == 1 ? np.l : np.l - np.h);
+    const dim3 grid = q.lpt ? dim3((unsigned)np.Mt, nx) : dim3(nx, (unsigned)np.Mt);
+    if (stage == 1) return launch_pdl(band_tc_kernel<1>, grid, dim3(kThreads), kSmem, stream, maps, q, g);
+    return launch_pdl(band_tc_kernel<2>, grid, dim3(kThreads), kSmem, stream, maps, q, g);
 }
 
 }  // namespace bakron

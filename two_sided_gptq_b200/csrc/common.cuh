@@ -126,6 +126,7 @@ struct SolveLayout {
 // over tile diagonals key(I,J) = I + J.
 struct NodeParams {
     int k, h, l, Mt, Nt;
+    int lpt = 0;  // band products: grid laid out longest contraction first (set at launch)
 };
 
 // One work item of a band GEMM: output tile (ra, rb), contraction over tile
