@@ -356,7 +356,8 @@ def solve_host(W, LA, LB, bits=4, *, V=None, codes=None, scales=None, gemm=0, ws
 
 
 def proxy_loss(W, V, A, B, *, stream=None) -> float:
-    """``tr((W-V)^T B (W-V) A)`` computed on the device (FP32 products, FP64 sum)."""
+    """``tr((W-V)^T B (W-V) A)`` computed on the device (both products on the
+    tensor cores in 3xTF32, the elementwise dot in FP64 in a fixed order)."""
     torch = _torch()
     lib = _lib()
     m, n = W.shape
