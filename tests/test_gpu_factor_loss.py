@@ -168,14 +168,22 @@ def test_end_to_end_gpu_factors(bk, name):
     assert r["failures"] == 0 and r["ties"] <= tie_cap(W.size)
 
 
-def test_solve_host_buffers(bk):
+@pytest.mark.parametrize("shape,leaf", [((150, 270), 0), ((1000, 300), 0), ((300, 1000), 6), ((640, 384), 7),
+                                        ((129, 1), 5), ((1, 257), 3)])
+def test_solve_host_buffers(bk, shape, leaf):
+    """bakron_solve_host (row blocks of V and codes copied back while the solve
+    runs, on the library's copy stream) equals the device solve, for tall and
+    wide shapes and for leaf structures whose launches cover one or two tile
+    diagonals; pinned host buffers, so the copies are asynchronous."""
     import torch
 
-    W, A, B = workloads.random_problem(150, 270, seed=8)
+    m, n = shape
+    W, A, B = workloads.random_problem(m, n, seed=m + 3 * n)
     LA = oracle.factor(A).astype(np.float32)
     LB = oracle.factor(B).astype(np.float32)
-    Vh, ch, sh = bk.solve_host(torch.from_numpy(W), torch.from_numpy(LA), torch.from_numpy(LB), bits=4)
-    Vd, cd, sd = bk.solve(_t(W), _t(LA), _t(LB), bits=4)
+    pin = lambda x: torch.from_numpy(x).pin_memory()
+    Vh, ch, sh = bk.solve_host(pin(W), pin(LA), pin(LB), bits=4, leaf=leaf)
+    Vd, cd, sd = bk.solve(_t(W), _t(LA), _t(LB), bits=4, leaf=leaf)
     assert np.array_equal(ch.numpy(), cd.cpu().numpy())
     assert np.array_equal(Vh.numpy(), Vd.cpu().numpy())
     assert np.array_equal(sh.numpy(), sd.cpu().numpy())
