@@ -33,7 +33,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 LEAF_BYTES_PER_WEIGHT = 25  # read Wt 4 + diagonal factor blocks 8; write code 1, V 4, D hi/lo 8
 LEAF_KERNELS = {1: ("leaf_nested_kernel", 3 * 127), 2: ("leaf_single_kernel", 255), 3: ("leaf_warp_kernel", 7 * 63),
                 4: ("leaf_wide_kernel", 3 * 127), 5: ("leaf_cluster_kernel<false, false>", 7 * 63),
-                6: ("leaf_cluster_kernel<true, false>", 7 * 63), 7: ("leaf_cluster_kernel<true, true>", 7 * 63)}
+                6: ("leaf_cluster_kernel<true, false>", 7 * 63), 7: ("leaf_cluster_kernel<true, true>", 7 * 63),
+                8: ("leaf_wave_kernel", 3 * 48 + 159)}
 # DRAM traffic of the band products from an ncu capture of one solve's 93
 # band launches (profiles/band_4096_dram.md); reported only while the band
 # kernel sources hash to the value the capture was taken with.
@@ -429,8 +430,8 @@ def proxy_loss_timing(bk, Wd, V, Ad, Bd, stream, dist, dev):
     ms = max_over_ranks(statistics.median(times), dist, dev)
     flops = 2.0 * m * n * (m + n)
     return {"value": value, "ms": ms, "flops": flops, "tflops": flops / (ms / 1e3) / 1e12,
-            "note": "tr((W-V)^T B (W-V) A): FP32 CUDA-core products B(W-V) and (W-V)A per 64 x 64 tile, "
-                    "FP64 fixed-order reduction; outside the metric"}
+            "note": "tr((W-V)^T B (W-V) A): the products B(W-V) and (W-V)A on the tcgen05 tensor cores in "
+                    "3xTF32, the elementwise dot in FP64 with a fixed order; outside the metric"}
 
 
 def main():

@@ -86,7 +86,7 @@ typedef struct {
 } bakron_quantizer_t;
 
 /* Solver configuration (NULL = defaults; zero fields take defaults).
- * The environment can change the defaults of five fields: BAKRON_LEAF (0..7),
+ * The environment can change the defaults of five fields: BAKRON_LEAF (0..8),
  * BAKRON_GEMM (0..1), BAKRON_TIMEOUT_MS (1..600000), BAKRON_GRAPH (0..1,
  * ignored when profile = 1) and BAKRON_FUSE (1..65535, the default
  * fuse_width); a non-zero field set by the caller wins.  A
@@ -128,7 +128,12 @@ typedef struct {
                          tile diagonals of every width-2 range of the
                          recursion in one launch: the second diagonal's tiles
                          wait (bounded, device flags) for their neighbours on
-                         the first and apply that node's updates themselves
+                         the first and apply that node's updates themselves;
+                         8 = each CTA of the cluster rounds its 32-row strip
+                         in one continuous sweep, 48 steps behind the CTA
+                         above (no sub-tile phases; the CTA above pushes its
+                         rounded residuals and its progress into the CTA
+                         below, bounded waits)
                          (bakron_tune_leaf picks one by measurement). */
     int32_t b_identity; /* 1: B = I (one-sided GPTQ with Hessian A, the case the
                            two-sided solve reduces to when B = I).  LB_dev may be
@@ -244,7 +249,7 @@ bakron_status_t bakron_solve(const float *W_dev, int64_t m, int64_t n, const flo
  * bakron_solve on the caller's problem once per structure after one warm-up
  * solve, timing each with CUDA events on `stream` (the call synchronises
  * `stream`), and writes the fastest structure (a bakron_config_t.leaf value,
- * 1..7) to *leaf_out and the seven times in ms to ms_out[0..6] (leaf 1..7;
+ * 1..8) to *leaf_out and the eight times in ms to ms_out[0..7] (leaf 1..8;
  * ms_out may be NULL).  Arguments as for bakron_solve; cfg->leaf is ignored
  * and cfg->profile must be 0.  V, codes and scales hold the last solve's
  * results (all structures give the same codes up to rounding ties).  Device

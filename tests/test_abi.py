@@ -293,9 +293,9 @@ def test_environment_overrides_are_validated():
     from two_sided_gptq_b200 import _native
 
     ok, bad = _native.Status.OK, _native.Status.ERR_INVALID_ARG
-    assert _plan_status_under_env({"BAKRON_LEAF": "7", "BAKRON_GEMM": "1", "BAKRON_TIMEOUT_MS": "50",
+    assert _plan_status_under_env({"BAKRON_LEAF": "8", "BAKRON_GEMM": "1", "BAKRON_TIMEOUT_MS": "50",
                                    "BAKRON_GRAPH": "1", "BAKRON_FUSE": "8"}) == ok
-    for env in ({"BAKRON_LEAF": "8"}, {"BAKRON_GEMM": "2"}, {"BAKRON_TIMEOUT_MS": "0"},
+    for env in ({"BAKRON_LEAF": "9"}, {"BAKRON_GEMM": "2"}, {"BAKRON_TIMEOUT_MS": "0"},
                 {"BAKRON_TIMEOUT_MS": "12ms"}, {"BAKRON_GRAPH": "-1"}, {"BAKRON_FUSE": "0"},
                 {"BAKRON_FUSE": "65536"}):
         assert _plan_status_under_env(env) == bad, env

@@ -62,7 +62,7 @@ def test_ragged_shapes(shape, gemm):
     check_solve(W, LA, LB, 4, gemm=gemm, label=f"{m}x{n}/gemm{gemm}")
 
 
-@pytest.mark.parametrize("leaf", [3, 5, 6, 7])
+@pytest.mark.parametrize("leaf", [3, 5, 6, 7, 8])
 @pytest.mark.parametrize("shape", RAGGED)
 def test_ragged_shapes_canary_write_only_their_buffers(shape, leaf):
     """Canary-padded workspace and outputs (guard zones of a known byte
@@ -124,7 +124,7 @@ def test_leaf_variants(case):
         W, A, B = workloads.random_problem(m, n, seed=m + 7 * n)
         LA, LB = oracle_factors(A, B)
         label = f"{m}x{n}"
-    for leaf in (1, 2, 3, 4, 5, 6, 7):
+    for leaf in (1, 2, 3, 4, 5, 6, 7, 8):
         check_solve(W, LA, LB, 4, leaf=leaf, label=f"{label}/leaf{leaf}")
 
 
@@ -183,7 +183,7 @@ def test_tune_leaf_picks_a_measured_structure():
     W, A, B, LA, LB = named("mid")
     Wd, LAd, LBd = (torch.from_numpy(x).cuda() for x in (W, LA.astype(np.float32), LB.astype(np.float32)))
     leaf, ms = bk.tune_leaf(Wd, LAd, LBd, bits=4)
-    assert leaf in (1, 2, 3, 4, 5, 6, 7) and all(t > 0 for t in ms)
+    assert leaf in (1, 2, 3, 4, 5, 6, 7, 8) and all(t > 0 for t in ms)
     assert ms[leaf - 1] == min(ms)
     check_solve(W, LA, LB, 4, leaf=leaf, label=f"mid/tuned-leaf{leaf}")
 

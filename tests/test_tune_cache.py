@@ -30,5 +30,5 @@ def test_bad_files_and_entries_are_misses(tmp_path):
     assert bk.tune_cache_get(path, "k") is None
     bk.tune_cache_put(path, "k", 2, [1.0])  # a corrupt file is replaced
     assert bk.tune_cache_get(path, "k") == (2, [1.0])
-    json.dump({"k": {"leaf": 8, "ms": []}, "j": "x"}, open(path, "w"))  # no structure 8
+    json.dump({"k": {"leaf": 9, "ms": []}, "j": "x"}, open(path, "w"))  # no structure 9
     assert bk.tune_cache_get(path, "k") is None and bk.tune_cache_get(path, "j") is None

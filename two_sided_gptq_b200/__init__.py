@@ -25,7 +25,7 @@ __all__ = ["factor", "solve", "solve_host", "proxy_loss", "plan_stats", "last_pr
 
 
 # bakron_config_t.leaf values bakron_tune_leaf times (one ms_out entry each)
-LEAF_STRUCTURES = (1, 2, 3, 4, 5, 6, 7)
+LEAF_STRUCTURES = (1, 2, 3, 4, 5, 6, 7, 8)
 
 
 def _lib():
@@ -145,7 +145,8 @@ def solve(W, LA, LB, bits=4, *, qmin=0, qmax=0, row_scale=None, gemm=0, ws=None,
     sub-tile, 4 six warps per 64 x 64 sub-tile, 5 as 3 with each tile on a
     cluster of four CTAs, 6 as 5 with the older product terms formed during
     the sweeps, 7 as 6 with two tile diagonals per launch (device flags, the
-    width-2 nodes' updates inside the leaf); :func:`tune_leaf` picks one by
+    width-2 nodes' updates inside the leaf), 8 continuous strip sweeps, one
+    per CTA, staggered by 48 steps; :func:`tune_leaf` picks one by
     measurement).  ``self_test_omit`` is a self-test hook of structure 7.  ``fuse_width`` (0 default, 1 never) runs the two band
     products of recursion nodes at most that many tile diagonals wide as one
     launch per target tile.  ``graph=True`` captures the solve's launches for this
@@ -229,7 +230,7 @@ def tune_cache_put(path: str, key: str, leaf: int, ms) -> None:
 def tune_leaf(W, LA, LB, bits=4, *, ws=None, out=None, stream=None, gemm=0, timeout_ms=0, cache=None):
     """Leaf structure chosen by measurement (``bakron_tune_leaf``): one timed
     solve per structure on this problem.  Returns ``(leaf, [ms_leaf1, ...,
-    ms_leaf7])``; pass ``leaf`` to :func:`solve`.
+    ms_leaf8])``; pass ``leaf`` to :func:`solve`.
 
     ``cache`` (or the ``BAKRON_TUNE_CACHE`` environment variable) names a JSON
     file keyed by (m, n, bits, GPU name): a stored measurement is returned

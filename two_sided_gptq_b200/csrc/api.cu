@@ -30,8 +30,8 @@ constexpr const char *kVersion = "bakron-b200 0.2";
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Leaf structures bakron_tune_leaf times (bakron_config_t.leaf 1..7).
-constexpr int kLeafStructures = 7;
+// Leaf structures bakron_tune_leaf times (bakron_config_t.leaf 1..8).
+constexpr int kLeafStructures = 8;
 // 0-based leaf variant of structure 7: width-2 ranges of the recursion run as
 // one launch of two tile diagonals (structure 6's kernel for single ones).
 constexpr int kPairVariant = 6;

@@ -973,13 +973,15 @@ cudaError_t leaf_configure()
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(leaf_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemSingle);
     if (e != cudaSuccess) return e;
-    return leaf_cluster_configure();
+    if ((e = leaf_cluster_configure()) != cudaSuccess) return e;
+    return leaf_wave_configure();
 }
 
 cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stream)
 {
     int I_lo = max(0, K - (p.Nt - 1)), I_hi = min(p.Mt - 1, K);
     if (I_hi < I_lo) return cudaSuccess;
+    if (variant == 7) return launch_leaf_wave(p, K, I_lo, I_hi - I_lo + 1, stream);
     if (variant == 4 || variant == 5)
         return launch_leaf_cluster(p, K, I_lo, I_hi - I_lo + 1, variant == 5, stream);
     if (variant == 3)
