@@ -14,7 +14,8 @@
 // are split by where their terms come from:
 //   row side   sum_{c' < c} R[a][c'] LtA[c][c']:  the current sub-tile's columns
 //              (side warp 1, without the newest c-1), the previous sub-tile's
-//              32 columns (side warp 2), the older sub-tiles (the product warp,
+//              32 columns (side warp 2; both read R and LtA rows from shared
+//              memory each step), the older sub-tiles (the product warp,
 //              per half sub-tile, subtracted from the staged Wt), and R[a][c-1]
 //              (the entry warp, from the lane to its left);
 //   column side sum_{r < a} LtB[a][r] D[r][c] over this row block (side warp 3,
@@ -148,7 +149,13 @@ leaf_wave_kernel(LeafArgs p, int K, int I_lo)
         const int r = pp * S3 + tid;  // row within the tile
         sRowC[tid] = make_float4(tid > 0 ? sLB[tid * RSC + r - 1] : 0.f, step_s, __frcp_rn(step_s), 0.f);
     }
-    for (int c = tid; c < T; c += kThreadsW) sLAsub[c] = c > 0 ? sLA[c * LAS + c - 1] : 0.f;
+    for (int c = tid; c < T; c += kThreadsW) {
+        sLAsub[c] = c > 0 ? sLA[c * LAS + c - 1] : 0.f;
+        // the row side's sums leave out the newest column (the entry warp's
+        // term) and never need the diagonal: both zero in the staged block
+        if (c > 0) sLA[c * LAS + c - 1] = 0.f;
+        sLA[c * LAS + c] = 0.f;
+    }
     // the other CTAs write into this one's shared memory from here on
     cluster.sync();
     pdl_wait();  // Wt comes from the previous kernel
@@ -319,19 +326,16 @@ leaf_wave_kernel(LeafArgs p, int K, int I_lo)
             sweep(std::false_type{});
     } else if (role == 1 || role == 2) {
         // ---- row side (lane = entry lane b): role 1 the current sub-tile's
-        // columns 32 q .. c-2, role 2 the previous sub-tile's 32 columns
-        // (without c-1 for b = 0); LtA row c of that block in registers,
-        // reloaded when the lane moves on to the next sub-tile
+        // columns, role 2 the previous sub-tile's 32 columns, both rows (R row
+        // a and LtA row c) read from shared memory each step.  The staged LtA
+        // block holds zeros on its diagonal and sub-diagonal (the newest
+        // column c-1 is the entry warp's term, written during this step) and
+        // above the diagonal, and R is still zero from column c on, so no
+        // lane masks its operands and none branches when it moves on to the
+        // next sub-tile; role 1 skips the 4-column groups past c-2
         const int b = lane;
         const int off = role == 1 ? 0 : 1;
-        float2 la[S3 / 2];
-#pragma unroll
-        for (int k = 0; k < S3 / 2; ++k) la[k] = make_float2(0.f, 0.f);
-        float4 rv[S3 / 4];
-#pragma unroll
-        for (int k = 0; k < S3 / 4; ++k) rv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-        int cur_q = -1;
-        const int lim = role == 1 ? b - 2 : (b == 0 ? S3 - 2 : S3 - 1);  // last column index used in the block
+        const int lim = role == 1 ? b - 2 : S3 - 1;  // last column of the block with a term
         for (int s = -1; s < kSteps; ++s) {
             const int act = s + 1 - b;
             const bool live = s + 1 < kSteps && act >= 0 && act < T;
@@ -339,29 +343,23 @@ leaf_wave_kernel(LeafArgs p, int K, int I_lo)
             const int a1 = ac & (S3 - 1), q1 = ac >> 5, qb = q1 - off;
             float sum = 0.f;
             if (live && qb >= 0) {
-                if (q1 != cur_q) {
-                    cur_q = q1;
-                    const float *lrow = sLA + (b + S3 * q1) * LAS + S3 * qb;
-#pragma unroll
-                    for (int k = 0; k < S3 / 2; ++k) {
-                        float2 v = *(const float2 *)(lrow + 2 * k);
-                        v.x = 2 * k + 0 <= lim ? v.x : 0.f;
-                        v.y = 2 * k + 1 <= lim ? v.y : 0.f;
-                        la[k] = v;
-                    }
-                }
                 const float *Rn = sR + a1 * RSC + S3 * qb;
+                const float *Ln = sLA + (b + S3 * q1) * LAS + S3 * qb;
+                float4 rv[S3 / 4], lv[S3 / 4];
 #pragma unroll
-                for (int k = 0; k < S3 / 4; ++k)
-                    if (4 * k <= lim) rv[k] = *(const float4 *)(Rn + 4 * k);
+                for (int k = 0; k < S3 / 4; ++k) {
+                    const bool use = 4 * k <= lim;
+                    rv[k] = use ? *(const float4 *)(Rn + 4 * k) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    lv[k] = use ? *(const float4 *)(Ln + 4 * k) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
                 float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
                 float2 u2 = make_float2(0.f, 0.f), u3 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int k = 0; k < S3 / 4; k += 2) {
-                    u0 = ffma2(make_float2(rv[k].x, rv[k].y), la[2 * k], u0);
-                    u1 = ffma2(make_float2(rv[k].z, rv[k].w), la[2 * k + 1], u1);
-                    u2 = ffma2(make_float2(rv[k + 1].x, rv[k + 1].y), la[2 * k + 2], u2);
-                    u3 = ffma2(make_float2(rv[k + 1].z, rv[k + 1].w), la[2 * k + 3], u3);
+                    u0 = ffma2(make_float2(rv[k].x, rv[k].y), make_float2(lv[k].x, lv[k].y), u0);
+                    u1 = ffma2(make_float2(rv[k].z, rv[k].w), make_float2(lv[k].z, lv[k].w), u1);
+                    u2 = ffma2(make_float2(rv[k + 1].x, rv[k + 1].y), make_float2(lv[k + 1].x, lv[k + 1].y), u2);
+                    u3 = ffma2(make_float2(rv[k + 1].z, rv[k + 1].w), make_float2(lv[k + 1].z, lv[k + 1].w), u3);
                 }
                 sum = ((u0.x + u1.x) + (u2.x + u3.x)) + ((u0.y + u1.y) + (u2.y + u3.y));
             }
