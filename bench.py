@@ -577,6 +577,8 @@ def main():
                      "bytes_per_step": leaf_bytes, "bound": "latency (dependent rounding steps)",
                      "sequential_steps_per_tile_diagonal": LEAF_KERNELS[leaf][1],
                      "ns_per_sequential_step": pr["leaf_ms"] * 1e6 / (plan["tile_diagonals"] * LEAF_KERNELS[leaf][1]),
+                     "dependent_steps_per_solve": {str(k): plan["tile_diagonals"] * v[1] for k, v in LEAF_KERNELS.items()},
+                     "dependent_steps_minimum": m + n - 1,
                      "share_of_profiled_step": pr["leaf_ms"] / pr["total_ms"]},
             "profile_ms": pr,
             "factor_ms": factor_ms,
