@@ -20,9 +20,9 @@
 //              (the entry warp, from the lane to its left);
 //   column side sum_{r < a} LtB[a][r] D[r][c] over this row block (side warp 3,
 //              without the newest a-1, which the entry warp adds from its own
-//              previous result), the row block above (side warp 4, from D
-//              columns the CTA above pushes into this CTA's shared memory each
-//              step), and the older row blocks (the product warp, per sub-tile,
+//              previous result), the row block above (side warp 4, from the
+//              D values the CTA above pushes into this CTA's shared memory as
+//              it rounds them), and the older row blocks (the product warp, per sub-tile,
 //              from the other CTAs' shared memory);
 // with R[a][c] = (all column-side terms) + D[a][c].  The side warps form step
 // s+1's sums during step s; the five sweep warps meet at one named barrier per
