@@ -47,11 +47,6 @@ cudaError_t launch_leaf(const LeafArgs &p, int K, int variant, cudaStream_t stre
 // a fourth warp forms the older product terms during the sweeps.
 cudaError_t leaf_cluster_configure();
 cudaError_t launch_leaf_cluster(const LeafArgs &p, int K, int I_lo, int tiles, bool overlap, cudaStream_t stream);
-// Continuous strip sweep (leaf structure 8, leaf_wave.cu): each CTA of a
-// tile's cluster rounds its 32-row strip in one sweep, 48 steps behind the
-// CTA above.
-cudaError_t leaf_wave_configure();
-cudaError_t launch_leaf_wave(const LeafArgs &p, int K, int I_lo, int tiles, cudaStream_t stream);
 // Tile diagonals K and K+1 in one launch (leaf structure 7): ticket counter
 // `slot`; the second diagonal's clusters wait for their neighbours' flags.
 cudaError_t launch_leaf_pair(const LeafArgs &p, int K, int slot, cudaStream_t stream);

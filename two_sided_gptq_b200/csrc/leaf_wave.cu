@@ -39,6 +39,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "leaf_wave.cuh"
 #include "leaf_common.cuh"
 
 namespace cg = cooperative_groups;
