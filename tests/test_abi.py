@@ -299,3 +299,18 @@ def test_environment_overrides_are_validated():
                 {"BAKRON_TIMEOUT_MS": "12ms"}, {"BAKRON_GRAPH": "-1"}, {"BAKRON_FUSE": "0"},
                 {"BAKRON_FUSE": "65536"}):
         assert _plan_status_under_env(env) == bad, env
+
+
+@pytest.mark.parametrize("shape", [(3, 3), (5, 8), (32, 32)])
+def test_plan_stats_strip_sweep_leaf_keeps_the_schedule(lib, shape):
+    """Leaf structure 8 changes only how a tile diagonal is swept: the
+    recursion, its leaves, nodes and update FLOPs are those of the default."""
+    from two_sided_gptq_b200 import _native
+
+    Mt, Nt = shape
+    base, wave = _native.PlanStats(), _native.PlanStats()
+    cfg = _native.Config(0, 0, 0, 0, None, 0, 8)
+    assert lib.bakron_plan_stats(Mt * 128, Nt * 128, None, ctypes.byref(base)) == 0
+    assert lib.bakron_plan_stats(Mt * 128, Nt * 128, ctypes.byref(cfg), ctypes.byref(wave)) == 0
+    for f, _ in _native.PlanStats._fields_:
+        assert getattr(wave, f) == getattr(base, f), f
