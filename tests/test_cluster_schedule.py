@@ -28,18 +28,12 @@ import workloads
 T, S3, NB = 128, 32, 4
 
 
-def replay(W, LtA, LtB, s_rows, qmin, qmax, mistake=None):
-    """Codes and pre-rounding values of one tile (m, n <= 128).  ``mistake``
-    plants one error in the replay (for the sensitivity test)."""
-    m, n = W.shape
-    Wp = np.zeros((T, T))
-    Wp[:m, :n] = W
-    LA = np.zeros((T, T))
-    LA[:n, :n] = LtA
-    LB = np.zeros((T, T))
-    LB[:m, :m] = LtB
-    step = np.ones(T, np.float32)
-    step[:m] = s_rows
+def sweep_tile(Wp, LA, LB, step, m, n, qmin, qmax, S_extra=None, mistake=None):
+    """One 128 x 128 tile by the phase schedule: staged Wt ``Wp``, the tile's
+    diagonal factor blocks ``LA`` (columns) and ``LB`` (rows), row steps, the
+    extent (m, n) inside the matrix.  ``S_extra`` (the pair form's upper
+    neighbour share) is added into S before each sub-tile.  Returns (codes,
+    pre-rounding values, D, in-tile R), all 128 x 128."""
     D = np.zeros((T, T))
     R = np.zeros((T, T))
     phase_of = np.full((T, T), 1 << 20)  # phase that produced D / R (block-wise)
@@ -79,6 +73,8 @@ def replay(W, LtA, LtB, s_rows, qmin, qmax, mistake=None):
             if q >= 1:
                 assert phase_of[S3 * p, S3 * (q - 1)] == e - 1
                 U += R[blk(p), blk(q - 1)] @ LA[blk(q), blk(q - 1)].T
+            if S_extra is not None:
+                S += S_extra[blk(p), blk(q)]
             W0[p] = Wp[blk(p), blk(q)] - U - S
             R[blk(p), blk(q)] = S  # R's block starts as S
         # the sweeps: 63 steps, every CTA of the phase in parallel
@@ -119,7 +115,23 @@ def replay(W, LtA, LtB, s_rows, qmin, qmax, mistake=None):
                         wt_out[r, c] = wt
                     rstep[a, b] = d
             phase_of[blk(p), blk(q)] = e
-    return codes[:m, :n], wt_out[:m, :n]
+    return codes, wt_out, D, R
+
+
+def replay(W, LtA, LtB, s_rows, qmin, qmax, mistake=None):
+    """Codes and pre-rounding values of one tile (m, n <= 128).  ``mistake``
+    plants one error in the replay (for the sensitivity test)."""
+    m, n = W.shape
+    Wp = np.zeros((T, T))
+    Wp[:m, :n] = W
+    LA = np.zeros((T, T))
+    LA[:n, :n] = LtA
+    LB = np.zeros((T, T))
+    LB[:m, :m] = LtB
+    step = np.ones(T, np.float32)
+    step[:m] = s_rows
+    codes, wt, _, _ = sweep_tile(Wp, LA, LB, step, m, n, qmin, qmax, mistake=mistake)
+    return codes[:m, :n], wt[:m, :n]
 
 
 @pytest.mark.parametrize("shape", [(128, 128), (100, 77), (33, 128), (128, 5)])
